@@ -1,0 +1,563 @@
+// Causal attention backward on tcgen05 for the folded layer.
+//
+// With s = q.k / sqrt(dh) (log2-domain LSE from the forward), per head:
+//   P = exp(s - LSE),  Delta_q = rowsum(dO * O),  dS = P * (dO V^T - Delta),
+//   dV = P^T dO,  dK = dS^T Q / sqrt(dh),  dQ = dS K / sqrt(dh).
+// Key-side gradients gather contributions from every rank's queries and are
+// written at the key owner's local row: the reverse of the forward's K/V
+// all-gather ("Zyphra TSP folds TP+SP onto one GPU axis", zubnet.ai,
+// paragraph 2 gives the forward exchange; its reverse is the reading taken
+// for the backward).
+//
+// Three kernels, no atomics (deterministic):
+//   attn_delta   Delta[h][row] = sum_d dO * O (bf16 inputs, fp32 sum).
+//   attn_dkdv    one item = (head, 128-key tile); loops over the 128-row query
+//                tiles that see any of its keys.  S^T = K Q^T and dP^T = V dO^T
+//                in TMEM; P^T, dS^T written to smem as bf16; dV += P^T dO and
+//                dK += dS^T Q accumulate in TMEM for the whole item.
+//   attn_dq      one item = (head, 128-row query tile); loops over key tiles.
+//                S = Q K^T, dP = dO V^T in TMEM; dS to smem; dQ += dS K.
+// Warp roles as in the forward: warp 0 TMA, warp 1 TMEM + MMA, warps 2-5
+// element-wise (thread = TMEM lane = row of the 128-row tile).
+#include "common.cuh"
+#include "internal.h"
+
+namespace tsp {
+namespace {
+
+constexpr int kBwdThreads = 192;
+
+__device__ __forceinline__ float ex2b(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void spin_drain(uint64_t *bar, uint32_t parity, long long limit) {
+    long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity) && clock64() - t0 < limit) {
+    }
+}
+
+template <int DH>
+struct BCfg {
+    static constexpr int SWB = DH * 2 < 128 ? DH * 2 : 128;
+    static constexpr int ATOM_COLS = SWB / 2;
+    static constexpr int NATOM = DH / ATOM_COLS;
+    static constexpr int TILE_BYTES = 128 * DH * 2;
+    static constexpr int ATOM_BYTES = 128 * SWB;
+    static constexpr uint32_t LAYOUT = SWB == 128 ? kSwizzle128 : (SWB == 64 ? kSwizzle64 : kSwizzle32);
+    static constexpr int SQ_BYTES = 128 * 128 * 2;  // a 128 x 128 bf16 operand (P^T, dS^T or dS)
+};
+
+template <int DH>
+__device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
+    using C = BCfg<DH>;
+    const int col = kk * 16;
+    return sdesc(base + (col / C::ATOM_COLS) * C::ATOM_BYTES + (col % C::ATOM_COLS) * 2, 16, 8 * C::SWB, C::LAYOUT);
+}
+template <int DH>
+__device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk) {
+    using C = BCfg<DH>;
+    return sdesc(base + kk * 16 * C::SWB, C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
+}
+__device__ __forceinline__ uint64_t sq_desc(uint32_t base, int kk) {
+    const int col = kk * 16;
+    return sdesc(base + (col / 64) * 16384 + (col % 64) * 2, 16, 1024, kSwizzle128);
+}
+// Write 32 consecutive bf16 values (columns c0..c0+31 of a 128-column row) of
+// a K-major 128B-swizzled 128x128 operand.
+__device__ __forceinline__ void store_row32(uint8_t *tile, int row, int c0, const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int col = c0 + q * 8;
+        uint4 w;
+        w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+        const int atom = col >> 6, chunk = ((col & 63) >> 3) ^ (row & 7);
+        *reinterpret_cast<uint4 *>(tile + atom * 16384 + row * 128 + chunk * 16) = w;
+    }
+}
+
+template <int DH>
+CUtensorMapSwizzle swz_of() {
+    return BCfg<DH>::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+           : BCfg<DH>::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// ---------------------------------------------------------------------------
+__global__ void attn_delta_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *dout, float *delta, int S, int H,
+                                  int dh) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32, lane = threadIdx.x % 32;
+    if (warp >= S * H) return;
+    const int row = warp / H, head = warp % H;
+    const int64_t base = static_cast<int64_t>(row) * H * dh + head * dh;
+    float s = 0.f;
+    for (int c = lane * 2; c < dh; c += 64) {
+        uint32_t a = *reinterpret_cast<const uint32_t *>(o + base + c);
+        uint32_t b = *reinterpret_cast<const uint32_t *>(dout + base + c);
+        s += bf16_lo(a) * bf16_lo(b) + bf16_hi(a) * bf16_hi(b);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) delta[static_cast<int64_t>(head) * S + row] = s;
+}
+
+// ---------------------------------------------------------------------------
+struct BwdParams {
+    AttnBwdDesc d;
+    const int *zig;          // local row -> global position (device copy of the map)
+    const int *qtile_maxpos; // per 128-row local query tile, largest global position
+    int num_items;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_dkdv_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
+                     const BwdParams bp, const DevErr err) {
+    using C = BCfg<DH>;
+    const AttnBwdDesc &a = bp.d;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *sK = smem;
+    uint8_t *sV = sK + C::TILE_BYTES;
+    uint8_t *sQ = sV + C::TILE_BYTES;
+    uint8_t *sdO = sQ + C::TILE_BYTES;
+    uint8_t *sPt = sdO + C::TILE_BYTES;
+    uint8_t *sdSt = sPt + C::SQ_BYTES;
+    float *sLse = reinterpret_cast<float *>(sdSt + C::SQ_BYTES);
+    float *sDelta = sLse + 128;
+    int *sPos = reinterpret_cast<int *>(sDelta + 128);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sPos + 128);
+    uint64_t *kv_full = bars + 0, *kv_empty = bars + 1, *q_full = bars + 2, *step_done = bars + 3,
+             *s_full = bars + 4, *p_full = bars + 5, *drain = bars + 6;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int h = a.H * DH;
+    const int nqt = a.S / 128;
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
+    const float scale = rsqrtf(static_cast<float>(DH));
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        mbar_init(kv_empty, 1);
+        mbar_init(q_full, 1);
+        mbar_init(step_done, 1);
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int item_iter = 0, step = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
+                if (!mbar_wait(kv_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
+                mbar_arrive_tx(kv_full, 2 * C::TILE_BYTES);
+                for (int t = 0; t < C::NATOM; ++t) {
+                    tma_load_2d(sK + t * C::ATOM_BYTES, &mK, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
+                    tma_load_2d(sV + t * C::ATOM_BYTES, &mV, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
+                }
+                for (int qt = 0; qt < nqt; ++qt) {
+                    if (bp.qtile_maxpos[qt] < kt * 128) continue;
+                    if (!mbar_wait(step_done, (step & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(q_full, 2 * C::TILE_BYTES + 3 * 512);
+                    for (int t = 0; t < C::NATOM; ++t) {
+                        tma_load_2d(sQ + t * C::ATOM_BYTES, &mQ, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
+                        tma_load_2d(sdO + t * C::ATOM_BYTES, &mdO, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
+                    }
+                    bulk_load(sLse, a.lse + static_cast<int64_t>(head) * a.S + qt * 128, 512, q_full);
+                    bulk_load(sDelta, a.delta + static_cast<int64_t>(head) * a.S + qt * 128, 512, q_full);
+                    bulk_load(sPos, bp.zig + qt * 128, 512, q_full);
+                    ++step;
+                }
+            }
+            if (item_iter > 0) spin_drain(kv_full, (item_iter - 1) & 1, err.wait_limit);
+            if (step > 0) spin_drain(q_full, (step - 1) & 1, err.wait_limit);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
+            const uint32_t k_b = smem_u32(sK), v_b = smem_u32(sV), q_b = smem_u32(sQ), do_b = smem_u32(sdO);
+            const uint32_t pt_b = smem_u32(sPt), dst_b = smem_u32(sdSt);
+            int item_iter = 0, step = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kt = a.kv_order[it] / a.H;
+                if (!mbar_wait(kv_full, item_iter & 1, abort_flag, err)) break;
+                bool first = true;
+                for (int qt = 0; qt < nqt; ++qt) {
+                    if (bp.qtile_maxpos[qt] < kt * 128) continue;
+                    if (!mbar_wait(q_full, step & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 0, kdesc<DH>(k_b, kk), kdesc<DH>(q_b, kk), idS, kk > 0);
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 128, kdesc<DH>(v_b, kk), kdesc<DH>(do_b, kk), idS, kk > 0);
+                    umma_commit(s_full);
+                    if (!mbar_wait(p_full, step & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(tmem + 256, sq_desc(pt_b, kk), mndesc<DH>(do_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(tmem + 384, sq_desc(dst_b, kk), mndesc<DH>(q_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
+                    umma_commit(step_done);
+                    first = false;
+                    ++step;
+                }
+                umma_commit(kv_empty);
+            }
+            if (!ok || *abort_flag) {
+                umma_commit(drain);
+                spin_drain(drain, 0, err.wait_limit);
+            }
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int trow = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        int step = 0;
+        for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
+            const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
+            const int key = kt * 128 + trow;
+            bool ok = true, any = false;
+            for (int qt = 0; qt < nqt; ++qt) {
+                if (bp.qtile_maxpos[qt] < kt * 128) continue;
+                any = true;
+                if (!mbar_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                // previous step's MMAs must be done reading P^T / dS^T
+                if (step > 0 && !mbar_wait(step_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float s[32], dp[32];
+                    tmem_ld32(tmem + lane_off + c * 32, s);
+                    tmem_ld32(tmem + lane_off + 128 + c * 32, dp);
+                    tmem_ld_wait();
+                    float pv[32], dsv[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int q = c * 32 + e;
+                        const float p = (key <= sPos[q]) ? ex2b(s[e] * sl2 - sLse[q]) : 0.f;
+                        pv[e] = p;
+                        dsv[e] = p * (dp[e] - sDelta[q]);
+                    }
+                    store_row32(sPt, trow, c * 32, pv);
+                    store_row32(sdSt, trow, c * 32, dsv);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+                ++step;
+            }
+            if (!ok) break;
+            if (!any) continue;
+            if (!mbar_wait(step_done, (step - 1) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            const int lrow = a.inv_map[key];
+            __nv_bfloat16 *dvrow = static_cast<__nv_bfloat16 *>(a.dv) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+            __nv_bfloat16 *dkrow = static_cast<__nv_bfloat16 *>(a.dk) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+                float v[32], k[32];
+                tmem_ld32(tmem + lane_off + 256 + c * 32, v);
+                tmem_ld32(tmem + lane_off + 384 + c * 32, k);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) k[e] *= scale;
+                uint4 *dv4 = reinterpret_cast<uint4 *>(dvrow + c * 32);
+                uint4 *dk4 = reinterpret_cast<uint4 *>(dkrow + c * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    dv4[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                        pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+                    dk4[q] = make_uint4(pack_bf16(k[8 * q], k[8 * q + 1]), pack_bf16(k[8 * q + 2], k[8 * q + 3]),
+                                        pack_bf16(k[8 * q + 4], k[8 * q + 5]), pack_bf16(k[8 * q + 6], k[8 * q + 7]));
+                }
+            }
+            tc_fence_before();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+template <int DH>
+struct DqCfg {
+    using C = BCfg<DH>;
+    static constexpr int KVST = 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_DO = OFF_Q + C::TILE_BYTES;
+    static constexpr int OFF_K = OFF_DO + C::TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + KVST * C::TILE_BYTES;
+    static constexpr int OFF_DS = OFF_V + KVST * C::TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_DS + C::SQ_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_dq_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                   const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
+                   const BwdParams bp, const DevErr err) {
+    using C = BCfg<DH>;
+    using Q = DqCfg<DH>;
+    const AttnBwdDesc &a = bp.d;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Q::OFF_BAR);
+    uint64_t *q_full = bars + 0, *q_empty = bars + 1, *kv_full = bars + 2, *kv_empty = bars + 4,
+             *s_full = bars + 6, *p_full = bars + 7, *ds_done = bars + 8, *drain = bars + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int h = a.H * DH;
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
+    const float scale = rsqrtf(static_cast<float>(DH));
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(ds_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto item_nkv = [&](int qt) { return bp.qtile_maxpos[qt] / 128 + 1; };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int item_iter = 0, kvc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
+                if (!mbar_wait(q_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
+                mbar_arrive_tx(q_full, 2 * C::TILE_BYTES);
+                for (int t = 0; t < C::NATOM; ++t) {
+                    tma_load_2d(smem + Q::OFF_Q + t * C::ATOM_BYTES, &mQ, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
+                    tma_load_2d(smem + Q::OFF_DO + t * C::ATOM_BYTES, &mdO, q_full, head * DH + t * C::ATOM_COLS,
+                                qt * 128);
+                }
+                const int nkv = item_nkv(qt);
+                for (int j = 0; j < nkv; ++j) {
+                    const int s = kvc % Q::KVST;
+                    if (!mbar_wait(&kv_empty[s], ((kvc / Q::KVST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(&kv_full[s], 2 * C::TILE_BYTES);
+                    for (int t = 0; t < C::NATOM; ++t) {
+                        tma_load_2d(smem + Q::OFF_K + s * C::TILE_BYTES + t * C::ATOM_BYTES, &mK, &kv_full[s],
+                                    head * DH + t * C::ATOM_COLS, j * 128);
+                        tma_load_2d(smem + Q::OFF_V + s * C::TILE_BYTES + t * C::ATOM_BYTES, &mV, &kv_full[s],
+                                    head * DH + t * C::ATOM_COLS, j * 128);
+                    }
+                    ++kvc;
+                }
+            }
+            for (int s = 0; s < Q::KVST; ++s)
+                if (kvc > s) {
+                    const int last = kvc - 1 - ((kvc - 1 - s) % Q::KVST);
+                    spin_drain(&kv_full[s], (last / Q::KVST) & 1, err.wait_limit);
+                }
+            if (item_iter > 0) spin_drain(q_full, (item_iter - 1) & 1, err.wait_limit);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
+            const uint32_t q_b = smem_u32(smem + Q::OFF_Q), do_b = smem_u32(smem + Q::OFF_DO);
+            const uint32_t ds_b = smem_u32(smem + Q::OFF_DS);
+            int item_iter = 0, kvc = 0, step = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int qt = a.q_order[it] / a.H;
+                if (!mbar_wait(q_full, item_iter & 1, abort_flag, err)) break;
+                const int nkv = item_nkv(qt);
+                for (int j = 0; j < nkv; ++j, ++step) {
+                    const int s = kvc % Q::KVST;
+                    if (!mbar_wait(&kv_full[s], (kvc / Q::KVST) & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * C::TILE_BYTES);
+                    const uint32_t v_b = smem_u32(smem + Q::OFF_V + s * C::TILE_BYTES);
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 0, kdesc<DH>(q_b, kk), kdesc<DH>(k_b, kk), idS, kk > 0);
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 128, kdesc<DH>(do_b, kk), kdesc<DH>(v_b, kk), idS, kk > 0);
+                    umma_commit(s_full);
+                    if (!mbar_wait(p_full, step & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(tmem + 256, sq_desc(ds_b, kk), mndesc<DH>(k_b, kk), idG, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(ds_done);
+                    umma_commit(&kv_empty[s]);
+                    ++kvc;
+                }
+                umma_commit(q_empty);
+            }
+            if (!ok || *abort_flag) {
+                umma_commit(drain);
+                spin_drain(drain, 0, err.wait_limit);
+            }
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int trow = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        uint8_t *sDS = smem + Q::OFF_DS;
+        int step = 0;
+        for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
+            const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
+            const int lrow = qt * 128 + trow;
+            const int pos = bp.zig[lrow];
+            const float lse = a.lse[static_cast<int64_t>(head) * a.S + lrow];
+            const float dl = a.delta[static_cast<int64_t>(head) * a.S + lrow];
+            const int nkv = item_nkv(qt);
+            bool ok = true;
+            for (int j = 0; j < nkv; ++j, ++step) {
+                if (!mbar_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                if (step > 0 && !mbar_wait(ds_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float s[32], dp[32], dsv[32];
+                    tmem_ld32(tmem + lane_off + c * 32, s);
+                    tmem_ld32(tmem + lane_off + 128 + c * 32, dp);
+                    tmem_ld_wait();
+                    const int k0 = j * 128 + c * 32;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float p = (k0 + e <= pos) ? ex2b(s[e] * sl2 - lse) : 0.f;
+                        dsv[e] = p * (dp[e] - dl);
+                    }
+                    store_row32(sDS, trow, c * 32, dsv);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            if (!mbar_wait(ds_done, (step - 1) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            __nv_bfloat16 *dqrow = static_cast<__nv_bfloat16 *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + 256 + c * 32, v);
+                tmem_ld_wait();
+                uint4 *d4 = reinterpret_cast<uint4 *>(dqrow + c * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    d4[q] = make_uint4(pack_bf16(v[8 * q] * scale, v[8 * q + 1] * scale),
+                                       pack_bf16(v[8 * q + 2] * scale, v[8 * q + 3] * scale),
+                                       pack_bf16(v[8 * q + 4] * scale, v[8 * q + 5] * scale),
+                                       pack_bf16(v[8 * q + 6] * scale, v[8 * q + 7] * scale));
+            }
+            tc_fence_before();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int DH>
+cudaError_t launch_bwd_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
+                            const int *zig, const int *qtile_maxpos) {
+    using C = BCfg<DH>;
+    const int h = a.H * DH;
+    CUtensorMap mq, mk, mv, mdo;
+    const auto swz = swz_of<DH>();
+    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+    ok = ok && encode_tensor_map_2d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+    ok = ok && encode_tensor_map_2d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+    ok = ok && encode_tensor_map_2d(&mdo, a.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+    if (!ok) return cudaErrorInvalidValue;
+
+    const int warps = a.S * a.H;
+    attn_delta_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.o),
+                                                                 static_cast<const __nv_bfloat16 *>(a.dout), a.delta,
+                                                                 a.S, a.H, DH);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    BwdParams bp;
+    bp.d = a;
+    bp.zig = zig;
+    bp.qtile_maxpos = qtile_maxpos;
+    bp.num_items = (a.S / 128) * a.H;
+    const int grid = bp.num_items < num_sms ? bp.num_items : num_sms;
+
+    const int smem_kv = 4 * C::TILE_BYTES + 2 * C::SQ_BYTES + 3 * 512 + 128 + 1024;
+    auto k1 = attn_dkdv_kernel<DH>;
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
+    if (e != cudaSuccess) return e;
+    k1<<<grid, kBwdThreads, smem_kv, st>>>(mq, mk, mv, mdo, bp, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    auto k2 = attn_dq_kernel<DH>;
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<DH>::SMEM);
+    if (e != cudaSuccess) return e;
+    k2<<<grid, kBwdThreads, DqCfg<DH>::SMEM, st>>>(mq, mk, mv, mdo, bp, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
+                                 const int *zig, const int *qtile_maxpos) {
+    switch (a.dh) {
+        case 32: return launch_bwd_impl<32>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 64: return launch_bwd_impl<64>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 128: return launch_bwd_impl<128>(a, err, num_sms, st, zig, qtile_maxpos);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace tsp

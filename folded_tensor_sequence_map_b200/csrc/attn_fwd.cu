@@ -1,0 +1,409 @@
+// Causal flash attention forward on tcgen05 for the folded layer.
+//
+// Queries are the ranks' local tokens (rank-major zigzag rows); keys and values
+// are the all-gathered K/V in global order ("Zyphra TSP folds TP+SP onto one
+// GPU axis", zubnet.ai, paragraph 2).  Every query row carries its own global
+// position p (from the zigzag map), and key k is visible iff k <= p.
+//
+// Work item = (head, block of 256 local query rows) = two 128-row query tiles.
+// CTA layout (10 warps, persistent, one CTA per SM):
+//   warp 0     TMA producer: the two Q tiles of the item, then K_j / V_j tiles
+//              of 128 keys (K ring of 2, V ring of 1 or 2 slots).
+//   warp 1     TMEM owner and MMA issuer: S_w = Q_w K_j^T (128x128, fp32 in
+//              TMEM) and O_w += P_w V_j (128 x dh, fp32 in TMEM) for w = 0, 1,
+//              ordered so that S of the next tile overlaps the softmax of the
+//              other tile (ping-pong between the two softmax groups).
+//   warps 2-5  softmax group 0 (query tile 0), warps 6-9 group 1: thread =
+//              query row; online softmax in the log2 domain, P written to
+//              shared memory as bf16 in the MMA's 128B-swizzled K-major
+//              layout; O rescaled in TMEM when the running max grows; final
+//              O / l written as bf16 and LSE (log2 domain) as fp32.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+dh), O1 [384,384+dh).
+#include "common.cuh"
+#include "internal.h"
+
+namespace tsp {
+namespace {
+
+constexpr int kFwdThreads = 320;
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Global position of local (rank-major) row i under the zigzag partition.
+__device__ __forceinline__ int zig_pos(int i, int L, int D, int c) {
+    const int r = i / L;
+    const int j = i - r * L;
+    return (j < c) ? r * c + j : (2 * D - 1 - r) * c + (j - c);
+}
+
+template <int DH>
+struct FwdCfg {
+    static constexpr int SWB = DH * 2 < 128 ? DH * 2 : 128;   // swizzle span in bytes
+    static constexpr int ATOM_COLS = SWB / 2;                 // bf16 columns per swizzle atom
+    static constexpr int NATOM = DH / ATOM_COLS;
+    static constexpr int TILE_BYTES = 128 * DH * 2;           // one 128-row tile of Q, K or V
+    static constexpr int ATOM_BYTES = 128 * SWB;
+    static constexpr uint32_t LAYOUT = SWB == 128 ? kSwizzle128 : (SWB == 64 ? kSwizzle64 : kSwizzle32);
+    static constexpr int KST = 2;
+    static constexpr int VST = DH == 128 ? 1 : 2;
+    static constexpr int P_BYTES = 128 * 128 * 2;
+    // smem map (1024-aligned pieces)
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
+    static constexpr int OFF_P = OFF_V + VST * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+};
+
+// K-major descriptor of a [128 rows][DH] bf16 tile for K step kk (16 columns).
+template <int DH>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
+    using C = FwdCfg<DH>;
+    const int col = kk * 16;
+    const uint32_t off = (col / C::ATOM_COLS) * C::ATOM_BYTES + (col % C::ATOM_COLS) * 2;
+    return sdesc(base + off, 16, 8 * C::SWB, C::LAYOUT);
+}
+// MN-major descriptor of V[128 keys][DH] (N = DH contiguous) for K step kk (16 keys).
+template <int DH>
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
+    using C = FwdCfg<DH>;
+    return sdesc(base + kk * 16 * C::SWB, C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
+}
+// P[128 rows][128 keys] bf16, K-major with 128B swizzle (two 64-key atoms).
+__device__ __forceinline__ uint64_t p_desc(uint32_t base, int kk) {
+    const int col = kk * 16;
+    return sdesc(base + (col / 64) * 16384 + (col % 64) * 2, 16, 1024, kSwizzle128);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                    const __grid_constant__ CUtensorMap mapV, const AttnDesc a, const DevErr err) {
+    using C = FwdCfg<DH>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *q_full = bars + 0;
+    uint64_t *q_empty = bars + 1;
+    uint64_t *k_full = bars + 2;            // [KST]
+    uint64_t *k_empty = k_full + C::KST;    // [KST]
+    uint64_t *v_full = k_empty + C::KST;    // [VST]
+    uint64_t *v_empty = v_full + C::VST;    // [VST]
+    uint64_t *s_full = v_empty + C::VST;    // [2]
+    uint64_t *p_full = s_full + 2;          // [2]
+    uint64_t *o_done = p_full + 2;          // [2]
+    uint64_t *drain = o_done + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int h = a.H * DH;
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < C::KST; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::VST; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&s_full[w], 1);
+            mbar_init(&p_full[w], 128);
+            mbar_init(&o_done[w], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&mapQ);
+        tma_prefetch_desc(&mapK);
+        tma_prefetch_desc(&mapV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int kcount = 0, vcount = 0, item_iter = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < a.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int qb = a.order[2 * it] / a.H, head = a.order[2 * it] % a.H, nkv = a.order[2 * it + 1];
+                if (!mbar_wait(q_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
+                mbar_arrive_tx(q_full, 2 * C::TILE_BYTES);
+                for (int w = 0; w < 2; ++w)
+                    for (int t = 0; t < C::NATOM; ++t)
+                        tma_load_2d(smem + C::OFF_Q + w * C::TILE_BYTES + t * C::ATOM_BYTES, &mapQ, q_full,
+                                    head * DH + t * C::ATOM_COLS, qb * 256 + w * 128);
+                for (int j = 0; j < nkv; ++j) {
+                    const int ks = kcount % C::KST;
+                    if (!mbar_wait(&k_empty[ks], ((kcount / C::KST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(&k_full[ks], C::TILE_BYTES);
+                    for (int t = 0; t < C::NATOM; ++t)
+                        tma_load_2d(smem + C::OFF_K + ks * C::TILE_BYTES + t * C::ATOM_BYTES, &mapK, &k_full[ks],
+                                    head * DH + t * C::ATOM_COLS, j * 128);
+                    ++kcount;
+                    const int vs = vcount % C::VST;
+                    if (!mbar_wait(&v_empty[vs], ((vcount / C::VST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(&v_full[vs], C::TILE_BYTES);
+                    for (int t = 0; t < C::NATOM; ++t)
+                        tma_load_2d(smem + C::OFF_V + vs * C::TILE_BYTES + t * C::ATOM_BYTES, &mapV, &v_full[vs],
+                                    head * DH + t * C::ATOM_COLS, j * 128);
+                    ++vcount;
+                }
+            }
+            // Drain: every issued load has landed before exit.
+            for (int s = 0; s < C::KST; ++s)
+                if (kcount > s) {
+                    const int last = kcount - 1 - ((kcount - 1 - s) % C::KST);
+                    long long t0 = clock64();
+                    while (!mbar_try_wait(&k_full[s], (last / C::KST) & 1) && clock64() - t0 < err.wait_limit) {}
+                }
+            for (int s = 0; s < C::VST; ++s)
+                if (vcount > s) {
+                    const int last = vcount - 1 - ((vcount - 1 - s) % C::VST);
+                    long long t0 = clock64();
+                    while (!mbar_try_wait(&v_full[s], (last / C::VST) & 1) && clock64() - t0 < err.wait_limit) {}
+                }
+            if (item_iter > 0) {
+                long long t0 = clock64();
+                while (!mbar_try_wait(q_full, (item_iter - 1) & 1) && clock64() - t0 < err.wait_limit) {}
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
+            const uint32_t qbase = smem_u32(smem + C::OFF_Q);
+            const uint32_t pbase = smem_u32(smem + C::OFF_P);
+            int kcount = 0, vcount = 0, tcount = 0, item_iter = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < a.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int nkv = a.order[2 * it + 1];
+                if (!mbar_wait(q_full, item_iter & 1, abort_flag, err)) break;
+                tc_fence_after();
+                // prologue: S_w for key tile 0
+                {
+                    const int ks = kcount % C::KST;
+                    if (!mbar_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) break;
+                    tc_fence_after();
+                    const uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
+                    for (int w = 0; w < 2; ++w) {
+                        for (int kk = 0; kk < DH / 16; ++kk)
+                            umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
+                                      kmajor_desc<DH>(kb, kk), idS, kk > 0);
+                        umma_commit(&s_full[w]);
+                    }
+                    umma_commit(&k_empty[ks]);
+                    ++kcount;
+                }
+                for (int j = 0; j < nkv && ok; ++j, ++tcount) {
+                    const int vs = vcount % C::VST;
+                    if (!mbar_wait(&v_full[vs], (vcount / C::VST) & 1, abort_flag, err)) { ok = false; break; }
+                    const uint32_t vb = smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES);
+                    int ks = kcount % C::KST;
+                    uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
+                    for (int w = 0; w < 2; ++w) {
+                        if (!mbar_wait(&p_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_bf16(tmem + 256 + w * 128, p_desc(pbase + w * C::P_BYTES, kk), mnmajor_desc<DH>(vb, kk),
+                                      idO, (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&o_done[w]);
+                        if (j + 1 < nkv) {
+                            if (w == 0) {
+                                if (!mbar_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) { ok = false; break; }
+                                tc_fence_after();
+                            }
+                            for (int kk = 0; kk < DH / 16; ++kk)
+                                umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
+                                          kmajor_desc<DH>(kb, kk), idS, kk > 0);
+                            umma_commit(&s_full[w]);
+                            if (w == 1) {
+                                umma_commit(&k_empty[ks]);
+                                ++kcount;
+                            }
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(&v_empty[vs]);
+                    ++vcount;
+                }
+                umma_commit(q_empty);
+            }
+            if (!ok || *abort_flag) {
+                umma_commit(drain);
+                long long t0 = clock64();
+                while (!mbar_try_wait(drain, 0) && clock64() - t0 < err.wait_limit) {}
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax groups
+        const int w = (warp - 2) / 4;
+        const int quarter = warp & 3;
+        const int trow = quarter * 32 + lane;  // row within the 128-row tile = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + w * 128;
+        const uint32_t o_addr = tmem + lane_off + 256 + w * 128;
+        uint8_t *prow = smem + C::OFF_P + w * C::P_BYTES + trow * 128;
+        int tcount = 0;
+        for (int it = blockIdx.x; it < a.num_items; it += gridDim.x) {
+            const int qb = a.order[2 * it] / a.H, head = a.order[2 * it] % a.H, nkv = a.order[2 * it + 1];
+            const int lrow = qb * 256 + w * 128 + trow;
+            const int pos = zig_pos(lrow, a.L, a.D, a.chunk);
+            float m = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nkv; ++j, ++tcount) {
+                if (!mbar_wait(&s_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                float s[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float t[32];
+                    tmem_ld32(s_addr + c * 32, t);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = t[e];
+                }
+                tmem_ld_wait();
+                const int kv0 = j * 128;
+                float mt = -INFINITY;
+                if (kv0 + 127 <= pos) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        s[c] *= sl2;
+                        mt = fmaxf(mt, s[c]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        s[c] = (kv0 + c <= pos) ? s[c] * sl2 : -INFINITY;
+                        mt = fmaxf(mt, s[c]);
+                    }
+                }
+                const float m_new = fmaxf(m, mt);
+                if (j > 0) {
+                    if (!mbar_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    if (m_new > m) {
+                        const float alpha = ex2(m - m_new);
+                        l *= alpha;
+#pragma unroll 1
+                        for (int c = 0; c < DH / 32; ++c) {
+                            float o[32];
+                            tmem_ld32(o_addr + c * 32, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                            tmem_st32(o_addr + c * 32, o);
+                        }
+                        tmem_st_wait();
+                    }
+                }
+                m = m_new;
+                float ls = 0.f;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    float p[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        p[e] = ex2(s[q * 8 + e] - m);
+                        ls += p[e];
+                    }
+                    uint4 v;
+                    v.x = pack_bf16(p[0], p[1]);
+                    v.y = pack_bf16(p[2], p[3]);
+                    v.z = pack_bf16(p[4], p[5]);
+                    v.w = pack_bf16(p[6], p[7]);
+                    const int atom = q >> 3, chunk = (q & 7) ^ (trow & 7);
+                    *reinterpret_cast<uint4 *>(prow + atom * 16384 + chunk * 16) = v;
+                }
+                l += ls;
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(&p_full[w]);
+            }
+            if (!ok) break;
+            // epilogue: wait for the last P V of this tile
+            if (!mbar_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            const float inv = 1.0f / l;
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.o) + static_cast<int64_t>(lrow) * h + head * DH;
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+                float o[32];
+                tmem_ld32(o_addr + c * 32, o);
+                tmem_ld_wait();
+                uint4 *d = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 v;
+                    v.x = pack_bf16(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+                    v.y = pack_bf16(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+                    v.z = pack_bf16(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+                    v.w = pack_bf16(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+                    d[q] = v;
+                }
+            }
+            a.lse[static_cast<int64_t>(head) * a.S + lrow] = m + __log2f(l);
+            tc_fence_before();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int DH>
+cudaError_t launch_fwd_impl(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st) {
+    using C = FwdCfg<DH>;
+    const int h = a.H * DH;
+    const CUtensorMapSwizzle swz = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : C::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUtensorMap mq, mk, mv;
+    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2,
+                                   C::ATOM_COLS, 128, swz);
+    ok = ok && encode_tensor_map_2d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2,
+                                    C::ATOM_COLS, 128, swz);
+    ok = ok && encode_tensor_map_2d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2,
+                                    C::ATOM_COLS, 128, swz);
+    if (!ok) return cudaErrorInvalidValue;
+    auto kern = attn_fwd_kernel<DH>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int grid = a.num_items < num_sms ? a.num_items : num_sms;
+    kern<<<grid, kFwdThreads, C::SMEM, st>>>(mq, mk, mv, a, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st) {
+    switch (a.dh) {
+        case 32: return launch_fwd_impl<32>(a, err, num_sms, st);
+        case 64: return launch_fwd_impl<64>(a, err, num_sms, st);
+        case 128: return launch_fwd_impl<128>(a, err, num_sms, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace tsp

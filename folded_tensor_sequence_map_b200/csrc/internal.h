@@ -1,0 +1,105 @@
+// Internal (not exported) interfaces between the host plan and the kernel
+// translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tsp {
+
+struct DevErr;
+
+// Epilogues of the GEMM (row = thread's output row, acc = fp32 accumulator):
+enum GemmEpilogue : int {
+    EPI_F32 = 0,        // out  f32[row][col] = acc
+    EPI_BF16 = 1,       // out bf16[row][col] = acc
+    EPI_QKV = 2,        // col < h: out (Q) at local row; h..2h: out_k at rowmap[row]; 2h..3h: out_v likewise
+    EPI_RESID_F32 = 3,  // out  f32 = acc + aux bf16 (residual)
+    EPI_GELU = 4,       // out bf16 = acc (pre-activation U), out2 bf16 = gelu_tanh(acc)
+    EPI_RESID_BF16 = 5, // out bf16 = acc + aux f32 (residual)
+    EPI_DGELU = 6,      // out bf16 = acc * gelu_tanh'(aux bf16)
+};
+
+// C[M][N] = sum_k A[m][k] B[n][k].
+//   a_mn == false: A is [M][K] with row stride lda;  true: A is stored [K][M] (row stride lda).
+//   b_mn == false: B is [N][K] with row stride ldb;  true: B is stored [K][N] (row stride ldb).
+// M % 128 == 0, K % 64 == 0, N % 128 == 0, pointers 16-byte aligned.
+struct GemmDesc {
+    const void *A;
+    int64_t lda;
+    bool a_mn;
+    const void *B;
+    int64_t ldb;
+    bool b_mn;
+    int M, N, K;
+    int epi;
+    void *out;
+    int64_t ldo;
+    void *out2;
+    int64_t ldo2;
+    const void *aux;
+    int64_t ldaux;
+    // ring K order: rows of rank m / ring_rows start at K block rank * ring_kblocks
+    int ring_rows;
+    int ring_kblocks;
+    // EPI_QKV only
+    const int *rowmap;
+    int hsplit;
+    void *out_k;
+    void *out_v;
+    bool force_bn128;
+};
+
+cudaError_t launch_gemm(const GemmDesc &g, const DevErr &err, int num_sms, cudaStream_t st);
+
+// Tensor-map encoding through the driver entry point (no libcuda link).
+bool encode_tensor_map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                          int64_t inner, int64_t outer, int64_t outer_stride_bytes, int box_inner, int box_outer,
+                          CUtensorMapSwizzle swz);
+
+// RMSNorm forward: out bf16 = x * rstd * g, rstd = 1/sqrt(mean(x^2)+eps).
+// x is bf16 (x_f32 == nullptr) or f32.
+cudaError_t launch_rmsnorm_fwd(const void *x_bf16, const float *x_f32, const float *g, void *out, float *rstd,
+                               int rows, int h, cudaStream_t st);
+
+// RMSNorm backward plus residual:
+//   n = x*rstd, dn = dout*g, dx = resid + rstd*(dn - n*mean(dn*n)).
+// dout f32; x bf16 or f32; resid bf16 or f32; outputs dx_f32 and/or dx_bf16;
+// per-block partial sums of dout*n go to dg_partial[nblocks][h], and are
+// reduced (in block order) into dg.
+cudaError_t launch_rmsnorm_bwd(const float *dout, const void *x_bf16, const float *x_f32, const float *rstd,
+                               const float *g, const void *resid_bf16, const float *resid_f32, float *dx_f32,
+                               void *dx_bf16, float *dg_partial, float *dg, int rows, int h, cudaStream_t st);
+int rmsnorm_bwd_partial_blocks(int rows);
+
+// Attention.
+struct AttnDesc {
+    int S, L, D, H, dh, chunk;  // tokens, tokens per rank, ranks, heads, head dim, zigzag chunk
+    const void *q;              // bf16 [S][h] rank-major (local) rows
+    const void *k, *v;          // bf16 [S][h] global rows
+    void *o;                    // bf16 [S][h] local rows
+    float *lse;                 // f32 [H][S] local rows, log2 domain (scores pre-multiplied by log2 e / sqrt(dh))
+    const int *order;           // pairs (qblock * H + head, number of 128-key tiles), longest first
+    int num_items;
+};
+cudaError_t launch_attn_fwd(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st);
+
+struct AttnBwdDesc {
+    int S, L, D, H, dh, chunk;
+    const void *q, *k, *v, *o, *dout;  // q, o, dout local rows; k, v global rows
+    const float *lse;                  // as written by the forward
+    float *delta;                      // f32 [H][S] scratch: rowsum(dO * O) per head, local rows
+    void *dq;                          // bf16, row stride ldd, local rows
+    void *dk, *dv;                     // bf16, row stride ldd, local rows of the key's owner
+    int64_t ldd;
+    const int *inv_map;                // global position -> local row
+    const int *kv_order;               // work order of (head, 128-key block), longest first
+    const int *q_order;                // work order of (head, 128-row query block), longest first
+};
+// zig: local row -> global position; qtile_maxpos: largest position of each
+// 128-row local query tile.  Launches the Delta, dK/dV and dQ kernels.
+cudaError_t launch_attn_bwd_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
+                                 const int *zig, const int *qtile_maxpos);
+
+}  // namespace tsp

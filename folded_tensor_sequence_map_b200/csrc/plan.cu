@@ -1,0 +1,517 @@
+// Host side of the C ABI: the plan (shape checks, zigzag map, shard schedules,
+// workspace layout, device tables, work orders) and the forward / backward
+// launch sequences.  Every step of the layer runs in the kernels of this
+// library; this file only validates arguments and enqueues launches.
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/tsp.h"
+#include "../../include/tsp_testing.h"
+#include "common.cuh"
+#include "internal.h"
+
+#define TSP_API extern "C" __attribute__((visibility("default")))
+
+struct tsp_plan_s {
+    int h, H, F, D, dh;
+    int64_t S, L, c;
+    std::vector<int32_t> zig;  // local row -> global position
+    // device state, created on first use on the then-current device
+    bool dev_ready = false;
+    int device = -1;
+    int num_sms = 0;
+    int32_t *d_zig = nullptr, *d_inv = nullptr, *d_qmax = nullptr;
+    int32_t *d_fwd_order = nullptr, *d_kv_order = nullptr, *d_q_order = nullptr;
+    unsigned int *d_err = nullptr;
+    int fwd_items = 0;
+    long long wait_limit = 0;
+    std::mutex mu;
+};
+
+namespace {
+
+using namespace tsp;
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// Byte layout of the saved-activation buffer and of the backward scratch.
+struct Layout {
+    size_t rstd1, a, q, k, v, o, lse, y, rstd2, b, u, g, saved_total;
+    size_t du, db, dy, dyb, dO, delta, dqkv, da, dgp, bwd_total;
+};
+
+Layout layout_of(const tsp_plan_s *p) {
+    Layout l{};
+    const size_t S = p->S, h = p->h, F = p->F, H = p->H;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += up(bytes);
+        return o;
+    };
+    l.rstd1 = take(S * 4);
+    l.a = take(S * h * 2);
+    l.q = take(S * h * 2);
+    l.k = take(S * h * 2);
+    l.v = take(S * h * 2);
+    l.o = take(S * h * 2);
+    l.lse = take(H * S * 4);
+    l.y = take(S * h * 4);
+    l.rstd2 = take(S * 4);
+    l.b = take(S * h * 2);
+    l.u = take(S * F * 2);
+    l.g = take(S * F * 2);
+    l.saved_total = off;
+    off = 0;
+    l.du = take(S * F * 2);
+    l.db = take(S * h * 4);
+    l.dy = take(S * h * 4);
+    l.dyb = take(S * h * 2);
+    l.dO = take(S * h * 2);
+    l.delta = take(H * S * 4);
+    l.dqkv = take(S * 3 * h * 2);
+    l.da = take(S * h * 4);
+    l.dgp = take(static_cast<size_t>(rmsnorm_bwd_partial_blocks(static_cast<int>(S))) * h * 4);
+    l.bwd_total = off;
+    return l;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                              const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(f);
+    });
+    return fn;
+}
+
+tsp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA; }
+
+// Device tables: map, inverse map, per-query-tile max position and the work
+// orders of the attention kernels (longest item first).
+tsp_status ensure_device(tsp_plan_s *p) {
+    std::lock_guard<std::mutex> g(p->mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TSP_ERR_CUDA;
+    if (p->dev_ready) return dev == p->device ? TSP_OK : TSP_ERR_INVALID_ARG;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return TSP_ERR_CUDA;
+    if (prop.major != 10) return TSP_ERR_UNSUPPORTED;
+    if (!get_encode()) return TSP_ERR_CUDA;
+    const int64_t S = p->S;
+    const int H = p->H;
+    std::vector<int32_t> inv(S), qmax(S / 128);
+    for (int64_t i = 0; i < S; ++i) inv[p->zig[i]] = static_cast<int32_t>(i);
+    for (int64_t t = 0; t < S / 128; ++t) {
+        int32_t m = 0;
+        for (int64_t i = t * 128; i < t * 128 + 128; ++i) m = std::max(m, p->zig[i]);
+        qmax[t] = m;
+    }
+    // forward items: (256-row query block, head), cost = key tiles
+    std::vector<std::pair<int, int>> fitems;
+    for (int64_t qb = 0; qb < S / 256; ++qb) {
+        int32_t m = std::max(qmax[2 * qb], qmax[2 * qb + 1]);
+        for (int hd = 0; hd < H; ++hd) fitems.push_back({static_cast<int>(qb * H + hd), m / 128 + 1});
+    }
+    std::stable_sort(fitems.begin(), fitems.end(), [](auto &x, auto &y) { return x.second > y.second; });
+    std::vector<int32_t> forder;
+    for (auto &it : fitems) {
+        forder.push_back(it.first);
+        forder.push_back(it.second);
+    }
+    // backward items: key tiles (cost = query tiles that see them) and query tiles (cost = key tiles)
+    std::vector<std::pair<int, int64_t>> kitems, qitems;
+    for (int64_t kt = 0; kt < S / 128; ++kt) {
+        int64_t cost = 0;
+        for (int64_t t = 0; t < S / 128; ++t) cost += qmax[t] >= kt * 128;
+        for (int hd = 0; hd < H; ++hd) kitems.push_back({static_cast<int>(kt * H + hd), cost});
+    }
+    for (int64_t qt = 0; qt < S / 128; ++qt)
+        for (int hd = 0; hd < H; ++hd) qitems.push_back({static_cast<int>(qt * H + hd), qmax[qt] / 128 + 1});
+    auto by_cost = [](auto &x, auto &y) { return x.second > y.second; };
+    std::stable_sort(kitems.begin(), kitems.end(), by_cost);
+    std::stable_sort(qitems.begin(), qitems.end(), by_cost);
+    std::vector<int32_t> korder, qorder;
+    for (auto &it : kitems) korder.push_back(it.first);
+    for (auto &it : qitems) qorder.push_back(it.first);
+
+    auto upload = [](int32_t **dst, const std::vector<int32_t> &v) {
+        if (cudaMalloc(dst, v.size() * 4) != cudaSuccess) return false;
+        return cudaMemcpy(*dst, v.data(), v.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess;
+    };
+    if (!upload(&p->d_zig, p->zig) || !upload(&p->d_inv, inv) || !upload(&p->d_qmax, qmax) ||
+        !upload(&p->d_fwd_order, forder) || !upload(&p->d_kv_order, korder) || !upload(&p->d_q_order, qorder))
+        return TSP_ERR_CUDA;
+    if (cudaMalloc(&p->d_err, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
+    if (cudaMemset(p->d_err, 0, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
+    p->fwd_items = static_cast<int>(fitems.size());
+    p->num_sms = prop.multiProcessorCount;
+    // A single wait may spin for about 2 s at the boost clock; the test hook
+    // can lower it.
+    long long limit = 4000000000LL;
+    if (const char *env = std::getenv("TSP_WAIT_LIMIT_CYCLES")) limit = std::atoll(env);
+    p->wait_limit = limit;
+    p->device = dev;
+    p->dev_ready = true;
+    return TSP_OK;
+}
+
+tsp_status check_pending_error(tsp_plan_s *p) {
+    unsigned int e = 0;
+    if (cudaMemcpy(&e, p->d_err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return TSP_ERR_CUDA;
+    if (e) {
+        cudaMemset(p->d_err, 0, sizeof(unsigned int));
+        return TSP_ERR_TIMEOUT;
+    }
+    return TSP_OK;
+}
+
+DevErr dev_err(const tsp_plan_s *p) { return DevErr{p->d_err, p->wait_limit}; }
+
+GemmDesc gemm(const void *A, int64_t lda, bool a_mn, const void *B, int64_t ldb, bool b_mn, int M, int N, int K,
+              int epi, void *out, int64_t ldo) {
+    GemmDesc g{};
+    g.A = A;
+    g.lda = lda;
+    g.a_mn = a_mn;
+    g.B = B;
+    g.ldb = ldb;
+    g.b_mn = b_mn;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.epi = epi;
+    g.out = out;
+    g.ldo = ldo;
+    return g;
+}
+
+}  // namespace
+
+namespace tsp {
+bool encode_tensor_map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dtype, int elem_bytes, int64_t inner,
+                          int64_t outer, int64_t outer_stride_bytes, int box_inner, int box_outer,
+                          CUtensorMapSwizzle swz) {
+    EncodeFn fn = get_encode();
+    if (!fn) return false;
+    (void)elem_bytes;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(outer_stride_bytes)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+}  // namespace tsp
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+
+TSP_API tsp_status tsp_plan(int h, int heads, int ffn, int64_t S, int D, tsp_plan_t *out) {
+    if (!out) return TSP_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (h <= 0 || heads <= 0 || ffn <= 0 || S <= 0 || D <= 0) return TSP_ERR_INVALID_ARG;
+    if (S % (2 * D) || heads % D || ffn % D || h % heads) return TSP_ERR_INDIVISIBLE;
+    const int dh = h / heads;
+    if (dh != 32 && dh != 64 && dh != 128) return TSP_ERR_UNSUPPORTED;
+    if (h % 128 || S % 256 || (S / D) % 128 || ffn % 128 || (ffn / D) % 64) return TSP_ERR_UNSUPPORTED;
+    if (S > (int64_t(1) << 30) / 4 || static_cast<int64_t>(heads) * S > (int64_t(1) << 31) - 1)
+        return TSP_ERR_UNSUPPORTED;
+    tsp_plan_s *p = new (std::nothrow) tsp_plan_s();
+    if (!p) return TSP_ERR_INVALID_ARG;
+    p->h = h;
+    p->H = heads;
+    p->F = ffn;
+    p->D = D;
+    p->dh = dh;
+    p->S = S;
+    p->L = S / D;
+    p->c = S / (2 * D);
+    p->zig.resize(S);
+    for (int r = 0; r < D; ++r)
+        for (int64_t i = 0; i < p->L; ++i)
+            p->zig[r * p->L + i] = static_cast<int32_t>(i < p->c ? r * p->c + i : (2 * D - 1 - r) * p->c + (i - p->c));
+    *out = p;
+    return TSP_OK;
+}
+
+TSP_API void tsp_plan_destroy(tsp_plan_t p) {
+    if (!p) return;
+    if (p->dev_ready) {
+        int cur = 0;
+        cudaGetDevice(&cur);
+        cudaSetDevice(p->device);
+        cudaFree(p->d_zig);
+        cudaFree(p->d_inv);
+        cudaFree(p->d_qmax);
+        cudaFree(p->d_fwd_order);
+        cudaFree(p->d_kv_order);
+        cudaFree(p->d_q_order);
+        cudaFree(p->d_err);
+        cudaSetDevice(cur);
+    }
+    delete p;
+}
+
+TSP_API tsp_status tsp_zigzag_map(tsp_plan_t p, int32_t *map_host) {
+    if (!p || !map_host) return TSP_ERR_INVALID_ARG;
+    std::memcpy(map_host, p->zig.data(), p->zig.size() * sizeof(int32_t));
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_shard_schedule(tsp_plan_t p, int phase, int32_t *sched) {
+    if (!p || !sched || (phase != 0 && phase != 1)) return TSP_ERR_INVALID_ARG;
+    const int D = p->D;
+    for (int t = 0; t < D; ++t)
+        for (int r = 0; r < D; ++r) sched[t * D + r] = phase == 0 ? t : (r + t) % D;
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_workspace_size(tsp_plan_t p, int training, size_t *ws, size_t *saved) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    Layout l = layout_of(p);
+    if (training) {
+        if (saved) *saved = l.saved_total;
+        if (ws) *ws = l.bwd_total;
+    } else {
+        if (saved) *saved = 0;
+        if (ws) *ws = l.saved_total;
+    }
+    return TSP_OK;
+}
+
+TSP_API double tsp_layer_flops(tsp_plan_t p, int backward) {
+    if (!p) return 0.0;
+    const double S = static_cast<double>(p->S), h = p->h, F = p->F;
+    const double fwd = 2.0 * S * (4.0 * h * h + 2.0 * h * F) + 2.0 * h * S * (S + 1.0);
+    return backward ? 2.0 * fwd : fwd;
+}
+
+TSP_API const char *tsp_status_string(tsp_status s) {
+    switch (s) {
+        case TSP_OK: return "TSP_OK";
+        case TSP_ERR_INVALID_ARG: return "TSP_ERR_INVALID_ARG";
+        case TSP_ERR_INDIVISIBLE: return "TSP_ERR_INDIVISIBLE";
+        case TSP_ERR_UNSUPPORTED: return "TSP_ERR_UNSUPPORTED";
+        case TSP_ERR_ALIGNMENT: return "TSP_ERR_ALIGNMENT";
+        case TSP_ERR_CUDA: return "TSP_ERR_CUDA";
+        case TSP_ERR_TIMEOUT: return "TSP_ERR_TIMEOUT";
+    }
+    return "TSP_ERR_UNKNOWN";
+}
+
+TSP_API tsp_status tsp_sync_status(tsp_plan_t p, void *stream) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TSP_ERR_CUDA;
+    if (!p->dev_ready) return TSP_OK;
+    return check_pending_error(p);
+}
+
+TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g1, const void *wqkv, const void *wo,
+                                     const float *g2, const void *w1, const void *w2, void *y, void *saved, void *ws,
+                                     void *stream) {
+    if (!p || !x || !g1 || !wqkv || !wo || !g2 || !w1 || !w2 || !y || !ws) return TSP_ERR_INVALID_ARG;
+    for (const void *q : {x, (const void *)g1, wqkv, wo, (const void *)g2, w1, w2, (const void *)y, (const void *)ws})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    if (saved && !aligned16(saved)) return TSP_ERR_ALIGNMENT;
+    tsp_status st = ensure_device(p);
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Layout l = layout_of(p);
+    uint8_t *base = static_cast<uint8_t *>(saved ? saved : ws);
+    const int S = static_cast<int>(p->S), h = p->h, F = p->F, L = static_cast<int>(p->L);
+    const DevErr err = dev_err(p);
+    auto *rstd1 = reinterpret_cast<float *>(base + l.rstd1);
+    void *a = base + l.a, *q = base + l.q, *k = base + l.k, *v = base + l.v, *o = base + l.o;
+    auto *lse = reinterpret_cast<float *>(base + l.lse);
+    auto *yres = reinterpret_cast<float *>(base + l.y);
+    auto *rstd2 = reinterpret_cast<float *>(base + l.rstd2);
+    void *b = base + l.b, *u = base + l.u, *g = base + l.g;
+
+    cudaError_t e = launch_rmsnorm_fwd(x, nullptr, g1, a, rstd1, S, h, s);
+    if (e != cudaSuccess) return TSP_ERR_CUDA;
+    // QKV projection over the broadcast attention shards; K/V land at global rows.
+    GemmDesc gq = gemm(a, h, false, wqkv, h, false, S, 3 * h, h, EPI_QKV, q, h);
+    gq.rowmap = p->d_zig;
+    gq.hsplit = h;
+    gq.out_k = k;
+    gq.out_v = v;
+    if ((e = launch_gemm(gq, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    AttnDesc ad{};
+    ad.S = S;
+    ad.L = L;
+    ad.D = p->D;
+    ad.H = p->H;
+    ad.dh = p->dh;
+    ad.chunk = static_cast<int>(p->c);
+    ad.q = q;
+    ad.k = k;
+    ad.v = v;
+    ad.o = o;
+    ad.lse = lse;
+    ad.order = p->d_fwd_order;
+    ad.num_items = p->fwd_items;
+    if ((e = launch_attn_fwd(ad, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    // out-projection (head-group partial sums in broadcast order) + residual, fp32 residual stream
+    GemmDesc go = gemm(o, h, false, wo, h, false, S, h, h, EPI_RESID_F32, yres, h);
+    go.aux = x;
+    go.ldaux = h;
+    if ((e = launch_gemm(go, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    if ((e = launch_rmsnorm_fwd(nullptr, yres, g2, b, rstd2, S, h, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    GemmDesc g1d = gemm(b, h, false, w1, h, false, S, F, h, EPI_GELU, u, F);
+    g1d.out2 = g;
+    g1d.ldo2 = F;
+    if ((e = launch_gemm(g1d, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    // W2 with the K loop over FFN shards in ring order (r + t) mod D, + residual
+    GemmDesc g2d = gemm(g, F, false, w2, F, false, S, h, F, EPI_RESID_BF16, y, h);
+    g2d.aux = yres;
+    g2d.ldaux = h;
+    g2d.ring_rows = L;
+    g2d.ring_kblocks = (F / p->D) / 64;
+    if ((e = launch_gemm(g2d, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *x, const float *g1, const void *wqkv,
+                                      const void *wo, const float *g2, const void *w1, const void *w2,
+                                      const void *saved, void *ws, void *dx, float *dg1, float *dwqkv, float *dwo,
+                                      float *dg2, float *dw1, float *dw2, void *stream) {
+    if (!p || !dy || !x || !g1 || !wqkv || !wo || !g2 || !w1 || !w2 || !saved || !ws || !dx || !dg1 || !dwqkv ||
+        !dwo || !dg2 || !dw1 || !dw2)
+        return TSP_ERR_INVALID_ARG;
+    for (const void *q : {dy, x, (const void *)g1, wqkv, wo, (const void *)g2, w1, w2, saved, (const void *)ws,
+                          (const void *)dx, (const void *)dg1, (const void *)dwqkv, (const void *)dwo,
+                          (const void *)dg2, (const void *)dw1, (const void *)dw2})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    tsp_status st = ensure_device(p);
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Layout l = layout_of(p);
+    const uint8_t *sv = static_cast<const uint8_t *>(saved);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const int S = static_cast<int>(p->S), h = p->h, F = p->F, L = static_cast<int>(p->L);
+    const DevErr err = dev_err(p);
+    const float *rstd1 = reinterpret_cast<const float *>(sv + l.rstd1);
+    const void *a = sv + l.a, *q = sv + l.q, *k = sv + l.k, *v = sv + l.v, *o = sv + l.o;
+    const float *lse = reinterpret_cast<const float *>(sv + l.lse);
+    const float *yres = reinterpret_cast<const float *>(sv + l.y);
+    const float *rstd2 = reinterpret_cast<const float *>(sv + l.rstd2);
+    const void *b = sv + l.b, *u = sv + l.u, *g = sv + l.g;
+    void *du = w + l.du;
+    float *db = reinterpret_cast<float *>(w + l.db);
+    float *dyf = reinterpret_cast<float *>(w + l.dy);
+    void *dyb = w + l.dyb, *dO = w + l.dO, *dqkv = w + l.dqkv;
+    float *delta = reinterpret_cast<float *>(w + l.delta);
+    float *da = reinterpret_cast<float *>(w + l.da);
+    float *dgp = reinterpret_cast<float *>(w + l.dgp);
+    cudaError_t e;
+#define TSP_LAUNCH(call)                          \
+    do {                                          \
+        if ((e = (call)) != cudaSuccess) return TSP_ERR_CUDA; \
+    } while (0)
+
+    // MLP ring backward: dU = (dY W2) * GELU'(U); dW2 = dY^T G; dW1 = dU^T b; db = dU W1 (ring K order)
+    GemmDesc gdu = gemm(dy, h, false, w2, F, true, S, F, h, EPI_DGELU, du, F);
+    gdu.aux = u;
+    gdu.ldaux = F;
+    TSP_LAUNCH(launch_gemm(gdu, err, p->num_sms, s));
+    TSP_LAUNCH(launch_gemm(gemm(dy, h, true, g, F, true, h, F, S, EPI_F32, dw2, F), err, p->num_sms, s));
+    TSP_LAUNCH(launch_gemm(gemm(du, F, true, b, h, true, F, h, S, EPI_F32, dw1, h), err, p->num_sms, s));
+    GemmDesc gdb = gemm(du, F, false, w1, h, true, S, h, F, EPI_F32, db, h);
+    gdb.ring_rows = L;
+    gdb.ring_kblocks = (F / p->D) / 64;
+    TSP_LAUNCH(launch_gemm(gdb, err, p->num_sms, s));
+    // RMSNorm2 backward + residual: dy = dY + RMSNorm2^T(db)
+    TSP_LAUNCH(launch_rmsnorm_bwd(db, nullptr, yres, rstd2, g2, dy, nullptr, dyf, dyb, dgp, dg2, S, h, s));
+    // out-projection backward: dO = dy Wo, dWo = dy^T O
+    TSP_LAUNCH(launch_gemm(gemm(dyb, h, false, wo, h, true, S, h, h, EPI_BF16, dO, h), err, p->num_sms, s));
+    TSP_LAUNCH(launch_gemm(gemm(dyb, h, true, o, h, true, h, h, S, EPI_F32, dwo, h), err, p->num_sms, s));
+    // attention backward; dK/dV reduced to the keys' owners
+    AttnBwdDesc ab{};
+    ab.S = S;
+    ab.L = L;
+    ab.D = p->D;
+    ab.H = p->H;
+    ab.dh = p->dh;
+    ab.chunk = static_cast<int>(p->c);
+    ab.q = q;
+    ab.k = k;
+    ab.v = v;
+    ab.o = o;
+    ab.dout = dO;
+    ab.lse = lse;
+    ab.delta = delta;
+    ab.dq = dqkv;
+    ab.dk = static_cast<uint8_t *>(dqkv) + static_cast<size_t>(h) * 2;
+    ab.dv = static_cast<uint8_t *>(dqkv) + static_cast<size_t>(2 * h) * 2;
+    ab.ldd = 3 * h;
+    ab.inv_map = p->d_inv;
+    ab.kv_order = p->d_kv_order;
+    ab.q_order = p->d_q_order;
+    TSP_LAUNCH(launch_attn_bwd_impl(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
+    // projection backward: dWqkv = [dQ|dK|dV]^T a, da = [dQ|dK|dV] Wqkv
+    TSP_LAUNCH(launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h), err, p->num_sms, s));
+    TSP_LAUNCH(launch_gemm(gemm(dqkv, 3 * h, false, wqkv, h, true, S, h, 3 * h, EPI_F32, da, h), err, p->num_sms, s));
+    // RMSNorm1 backward + residual: dx = dy + RMSNorm1^T(da)
+    TSP_LAUNCH(launch_rmsnorm_bwd(da, x, nullptr, rstd1, g1, nullptr, dyf, nullptr, dx, dgp, dg1, S, h, s));
+#undef TSP_LAUNCH
+    return TSP_OK;
+}
+
+// ===========================================================================
+// Test hooks (tsp_testing.h)
+// ===========================================================================
+
+TSP_API tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A, int64_t lda, const void *B,
+                                 int64_t ldb, float *C, int64_t ldc, int force_bn128, void *stream) {
+    if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0) return TSP_ERR_INVALID_ARG;
+    if (M % 128 || N % 128 || K % 64) return TSP_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return TSP_ERR_ALIGNMENT;
+    static unsigned int *d_err = nullptr;
+    static int sms = 0;
+    if (!d_err) {
+        if (cudaMalloc(&d_err, 4) != cudaSuccess || cudaMemset(d_err, 0, 4) != cudaSuccess) return TSP_ERR_CUDA;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    GemmDesc g = gemm(A, lda, a_mn != 0, B, ldb, b_mn != 0, M, N, K, EPI_F32, C, ldc);
+    g.force_bn128 = force_bn128 != 0;
+    return cuda_status(launch_gemm(g, DevErr{d_err, 4000000000LL}, sms, static_cast<cudaStream_t>(stream)));
+}
+
+TSP_API tsp_status tsp_test_buffer_offset(tsp_plan_t p, const char *name, size_t *offset) {
+    if (!p || !name || !offset) return TSP_ERR_INVALID_ARG;
+    const Layout l = layout_of(p);
+    struct {
+        const char *n;
+        size_t o;
+    } tab[] = {{"rstd1", l.rstd1}, {"a", l.a},   {"q", l.q},         {"k", l.k},     {"v", l.v},
+               {"o", l.o},         {"lse", l.lse}, {"y", l.y},       {"rstd2", l.rstd2}, {"b", l.b},
+               {"u", l.u},         {"g", l.g},   {"ws.du", l.du},    {"ws.db", l.db}, {"ws.dy", l.dy},
+               {"ws.dO", l.dO},    {"ws.delta", l.delta}, {"ws.dqkv", l.dqkv}, {"ws.da", l.da}};
+    for (auto &t : tab)
+        if (std::strcmp(t.n, name) == 0) {
+            *offset = t.o;
+            return TSP_OK;
+        }
+    return TSP_ERR_INVALID_ARG;
+}

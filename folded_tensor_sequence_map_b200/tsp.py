@@ -1,0 +1,235 @@
+"""Thin Python binding of the C ABI in ``include/tsp.h`` (and the test hooks
+of ``include/tsp_testing.h``).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity and passed as raw pointers; every step of the layer runs in the
+CUDA kernels of ``libtsp.so``.  There is no fallback: if the library is
+missing or fails to load, importing this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtsp.so")
+
+TSP_OK = 0
+STATUS_NAMES = {
+    0: "TSP_OK",
+    1: "TSP_ERR_INVALID_ARG",
+    2: "TSP_ERR_INDIVISIBLE",
+    3: "TSP_ERR_UNSUPPORTED",
+    4: "TSP_ERR_ALIGNMENT",
+    5: "TSP_ERR_CUDA",
+    6: "TSP_ERR_TIMEOUT",
+}
+
+EXPORTED = (
+    "tsp_plan",
+    "tsp_plan_destroy",
+    "tsp_zigzag_map",
+    "tsp_shard_schedule",
+    "tsp_workspace_size",
+    "tsp_layer_forward",
+    "tsp_layer_backward",
+    "tsp_sync_status",
+    "tsp_status_string",
+    "tsp_layer_flops",
+    "tsp_test_gemm",
+    "tsp_test_buffer_offset",
+)
+
+
+class TSPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libtsp.so is not built ({LIB_PATH}); run python -m folded_tensor_sequence_map_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, SZ, V = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+    lib.tsp_plan.argtypes = [I, I, I, I64, I, ctypes.POINTER(P)]
+    lib.tsp_plan.restype = I
+    lib.tsp_plan_destroy.argtypes = [P]
+    lib.tsp_plan_destroy.restype = None
+    lib.tsp_zigzag_map.argtypes = [P, P]
+    lib.tsp_zigzag_map.restype = I
+    lib.tsp_shard_schedule.argtypes = [P, I, P]
+    lib.tsp_shard_schedule.restype = I
+    lib.tsp_workspace_size.argtypes = [P, I, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]
+    lib.tsp_workspace_size.restype = I
+    lib.tsp_layer_forward.argtypes = [P] + [V] * 11
+    lib.tsp_layer_forward.restype = I
+    lib.tsp_layer_backward.argtypes = [P] + [V] * 18
+    lib.tsp_layer_backward.restype = I
+    lib.tsp_sync_status.argtypes = [P, V]
+    lib.tsp_sync_status.restype = I
+    lib.tsp_status_string.argtypes = [I]
+    lib.tsp_status_string.restype = ctypes.c_char_p
+    lib.tsp_layer_flops.argtypes = [P, I]
+    lib.tsp_layer_flops.restype = ctypes.c_double
+    lib.tsp_test_gemm.argtypes = [I, I, I, I, I, V, I64, V, I64, V, I64, I, V]
+    lib.tsp_test_gemm.restype = I
+    lib.tsp_test_buffer_offset.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(SZ)]
+    lib.tsp_test_buffer_offset.restype = I
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != TSP_OK:
+        raise TSPError(status, where)
+
+
+class Plan:
+    """Owner of a ``tsp_plan_t``; freed with the object."""
+
+    def __init__(self, handle: int, h: int, heads: int, ffn: int, S: int, D: int):
+        self.handle = ctypes.c_void_p(handle)
+        self.h, self.heads, self.ffn, self.S, self.D = h, heads, ffn, S, D
+
+    def __del__(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            _lib.tsp_plan_destroy(self.handle)
+            self.handle = None
+
+
+def _ptr(t, name, dtype=None, shape=None):
+    """Device pointer of a contiguous CUDA tensor (or a raw int address)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch tensor or an address")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def tsp_plan(h: int, heads: int, ffn: int, S: int, D: int) -> Plan:
+    out = ctypes.c_void_p()
+    _check(_lib.tsp_plan(h, heads, ffn, S, D, ctypes.byref(out)), "tsp_plan")
+    return Plan(out.value, h, heads, ffn, S, D)
+
+
+def tsp_zigzag_map(plan: Plan) -> np.ndarray:
+    m = np.empty(plan.S, dtype=np.int32)
+    _check(_lib.tsp_zigzag_map(plan.handle, m.ctypes.data), "tsp_zigzag_map")
+    return m
+
+
+def tsp_shard_schedule(plan: Plan, phase: int) -> np.ndarray:
+    s = np.empty((plan.D, plan.D), dtype=np.int32)
+    _check(_lib.tsp_shard_schedule(plan.handle, phase, s.ctypes.data), "tsp_shard_schedule")
+    return s
+
+
+def tsp_workspace_size(plan: Plan, training: bool):
+    ws, saved = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.tsp_workspace_size(plan.handle, int(bool(training)), ctypes.byref(ws), ctypes.byref(saved)),
+           "tsp_workspace_size")
+    return ws.value, saved.value
+
+
+def tsp_layer_flops(plan: Plan, backward: bool) -> float:
+    return _lib.tsp_layer_flops(plan.handle, int(bool(backward)))
+
+
+def tsp_status_string(status: int) -> str:
+    return _lib.tsp_status_string(status).decode()
+
+
+def tsp_layer_forward(plan: Plan, x, g1, wqkv, wo, g2, w1, w2, y, saved, ws, stream=None) -> None:
+    import torch
+
+    h, F, S = plan.h, plan.ffn, plan.S
+    bf, f32, u8 = torch.bfloat16, torch.float32, None
+    args = [
+        _ptr(x, "x", bf, (S, h)),
+        _ptr(g1, "g1", f32, (h,)),
+        _ptr(wqkv, "wqkv", bf, (3 * h, h)),
+        _ptr(wo, "wo", bf, (h, h)),
+        _ptr(g2, "g2", f32, (h,)),
+        _ptr(w1, "w1", bf, (F, h)),
+        _ptr(w2, "w2", bf, (h, F)),
+        _ptr(y, "y", bf, (S, h)),
+        _ptr(saved, "saved", u8),
+        _ptr(ws, "ws", u8),
+        _stream(stream),
+    ]
+    _check(_lib.tsp_layer_forward(plan.handle, *args), "tsp_layer_forward")
+
+
+def tsp_layer_backward(plan: Plan, dy, x, g1, wqkv, wo, g2, w1, w2, saved, ws, dx, dg1, dwqkv, dwo, dg2, dw1, dw2,
+                       stream=None) -> None:
+    import torch
+
+    h, F, S = plan.h, plan.ffn, plan.S
+    bf, f32 = torch.bfloat16, torch.float32
+    args = [
+        _ptr(dy, "dy", bf, (S, h)),
+        _ptr(x, "x", bf, (S, h)),
+        _ptr(g1, "g1", f32, (h,)),
+        _ptr(wqkv, "wqkv", bf, (3 * h, h)),
+        _ptr(wo, "wo", bf, (h, h)),
+        _ptr(g2, "g2", f32, (h,)),
+        _ptr(w1, "w1", bf, (F, h)),
+        _ptr(w2, "w2", bf, (h, F)),
+        _ptr(saved, "saved"),
+        _ptr(ws, "ws"),
+        _ptr(dx, "dx", bf, (S, h)),
+        _ptr(dg1, "dg1", f32, (h,)),
+        _ptr(dwqkv, "dwqkv", f32, (3 * h, h)),
+        _ptr(dwo, "dwo", f32, (h, h)),
+        _ptr(dg2, "dg2", f32, (h,)),
+        _ptr(dw1, "dw1", f32, (F, h)),
+        _ptr(dw2, "dw2", f32, (h, F)),
+        _stream(stream),
+    ]
+    _check(_lib.tsp_layer_backward(plan.handle, *args), "tsp_layer_backward")
+
+
+def tsp_sync_status(plan: Plan, stream=None) -> None:
+    _check(_lib.tsp_sync_status(plan.handle, _stream(stream)), "tsp_sync_status")
+
+
+# ---- test hooks --------------------------------------------------------------
+
+def tsp_test_gemm(a_mn: bool, b_mn: bool, M: int, N: int, K: int, A, lda: int, B, ldb: int, C, ldc: int,
+                  force_bn128: bool = False, stream=None) -> None:
+    _check(_lib.tsp_test_gemm(int(a_mn), int(b_mn), M, N, K, _ptr(A, "A"), lda, _ptr(B, "B"), ldb, _ptr(C, "C"),
+                              ldc, int(force_bn128), _stream(stream)), "tsp_test_gemm")
+
+
+def tsp_test_buffer_offset(plan: Plan, name: str) -> int:
+    off = ctypes.c_size_t()
+    _check(_lib.tsp_test_buffer_offset(plan.handle, name.encode(), ctypes.byref(off)), "tsp_test_buffer_offset")
+    return off.value

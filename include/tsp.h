@@ -1,0 +1,156 @@
+/*
+ * tsp.h - C ABI of the folded Tensor-Sequence-Parallel (TSP) decoder layer on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  "Zyphra TSP folds TP+SP onto one GPU axis, 2.6x throughput
+ * on 1,024 MI300Xs" (zubnet.ai), paragraph 1: tensor parallelism (weights) and
+ * sequence parallelism (tokens) share one mesh axis of size D, so each of the D
+ * ranks holds 1/D of the layer's weights and 1/D of the sequence.  Paragraph 2
+ * of the same page gives the schedule: attention weight shards are broadcast
+ * one after another and applied by every rank to its own tokens, K/V are then
+ * all-gathered under a zigzag token partition, and the MLP weight shards travel
+ * a ring so that partial sums stay on their rank (no all-reduce).  Here the D
+ * ranks are virtual ranks of one GPU: a broadcast, an all-gather or a ring step
+ * becomes the choice of which shard, or which K/V rows, a tile reads.
+ *
+ * The layer (one dense pre-norm decoder layer, batch 1, no bias, no positional
+ * encoding):
+ *     a = RMSNorm(x; g1)            eps = 1e-5 inside the square root
+ *     [Q|K|V] = a Wqkv^T            Wqkv rows: Q heads 0..H-1, then K, then V
+ *     O = causal softmax(Q K^T / sqrt(dh)) V     per head, key <= query
+ *     y = x + O Wo^T
+ *     b = RMSNorm(y; g2)
+ *     z = y + GELU_tanh(b W1^T) W2^T
+ *
+ * Conventions shared by every call.
+ *   - Weights use the [out, in] row-major layout of a linear layer, bf16:
+ *     wqkv [3h][h], wo [h][h], w1 [F][h], w2 [h][F].  Gains g1, g2: float32 [h].
+ *   - Activations are row-major [tokens][features] in RANK-MAJOR ZIGZAG order:
+ *     rank 0's L = S/D tokens, then rank 1's, ...  Row r*L+i holds global token
+ *     tsp_zigzag_map()[r*L+i].  The caller permutes with that map.
+ *   - The caller owns and allocates every buffer; the library never allocates
+ *     or frees caller memory.  The plan owns its host metadata and a few small
+ *     device tables, created on first use and freed by tsp_plan_destroy.
+ *   - Device pointers must be 16-byte aligned (TSP_ERR_ALIGNMENT otherwise).
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Layer calls are asynchronous on `stream` (a cudaStream_t, may be 0).
+ *     Argument errors are reported synchronously and enqueue nothing.
+ *   - A bounded device-side wait that ran out sets a flag in the plan; it is
+ *     reported as TSP_ERR_TIMEOUT by tsp_sync_status() and by the next layer
+ *     call.  Kernels never spin without a limit.
+ */
+#ifndef TSP_H
+#define TSP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tsp_plan_s *tsp_plan_t; /* opaque, host-owned */
+
+typedef enum {
+    TSP_OK = 0,
+    TSP_ERR_INVALID_ARG = 1, /* NULL pointer, non-positive size, bad phase */
+    TSP_ERR_INDIVISIBLE = 2, /* S % 2D, heads % D, ffn % D or h % heads != 0 */
+    TSP_ERR_UNSUPPORTED = 3, /* shape outside the kernels' tiling, or device is not sm_100 */
+    TSP_ERR_ALIGNMENT = 4,   /* a device pointer is not 16-byte aligned */
+    TSP_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+    TSP_ERR_TIMEOUT = 6      /* a bounded device-side wait expired */
+} tsp_status;
+
+/* Build a plan for one layer: hidden size h, `heads` attention heads (head size
+ * dh = h/heads, Q and K/V heads equal), FFN width `ffn`, S tokens, D virtual
+ * ranks.  Divisibility follows from the partition (2D zigzag chunks, heads and
+ * FFN units split D ways): TSP_ERR_INDIVISIBLE if S % (2D), heads % D,
+ * ffn % D or h % heads is non-zero.  TSP_ERR_UNSUPPORTED when the shape is
+ * outside what the kernels tile: dh not in {32, 64, 128}, h % 128, S % 256,
+ * (S/D) % 128, ffn % 128 or (ffn/D) % 64 non-zero.  Needs no GPU.
+ * On success *out receives a new plan. */
+tsp_status tsp_plan(int h, int heads, int ffn, int64_t S, int D, tsp_plan_t *out);
+
+/* Free a plan and its device tables.  NULL is ignored.  Not while a layer call
+ * that uses the plan is still running on the GPU. */
+void tsp_plan_destroy(tsp_plan_t plan);
+
+/* Zigzag token partition ("Zyphra TSP folds TP+SP onto one GPU axis",
+ * zubnet.ai, paragraph 2: zigzag partition of K/V for load balance).  The
+ * sequence is cut into 2D chunks of c = S/(2D) tokens and rank r owns chunks r
+ * and 2D-1-r, in ascending order, so every rank sees the same number of causal
+ * (query, key) pairs.  Writes S int32 values to host memory:
+ * map_host[r*L + i] = global position of rank r's i-th token.  Needs no GPU. */
+tsp_status tsp_zigzag_map(tsp_plan_t plan, int32_t *map_host);
+
+/* Shard schedule of one phase (same page, paragraph 2), D x D int32 to host
+ * memory, sched_host[t*D + r] = shard that rank r applies at step t.
+ * phase 0: attention broadcast, shard t at step t on every rank.
+ * phase 1: MLP ring, rank r holds shard (r + t) mod D (it starts with its own
+ * shard and receives rank r+1's after each step).  Attention shard t is heads
+ * [t*H/D, (t+1)*H/D); MLP shard s is FFN units [s*F/D, (s+1)*F/D).
+ * TSP_ERR_INVALID_ARG for another phase.  Needs no GPU. */
+tsp_status tsp_shard_schedule(tsp_plan_t plan, int phase, int32_t *sched_host);
+
+/* Bytes of device memory the layer calls need.
+ *   training != 0: *saved_bytes = activations kept from forward to backward,
+ *                  *ws_bytes = scratch of either call.
+ *   training == 0: *saved_bytes = 0, *ws_bytes = scratch of an inference
+ *                  forward (pass saved = NULL).
+ * Either output pointer may be NULL.  Needs no GPU. */
+tsp_status tsp_workspace_size(tsp_plan_t plan, int training, size_t *ws_bytes, size_t *saved_bytes);
+
+/* Forward of the folded layer.  Device pointers:
+ *   x    bf16 [S][h] rank-major zigzag order (input)
+ *   g1, g2 float32 [h]; wqkv, wo, w1, w2 bf16 as above (inputs)
+ *   y    bf16 [S][h] rank-major zigzag order (output z of the layer)
+ *   saved  NULL for inference, else saved_bytes for tsp_layer_backward
+ *   ws     ws_bytes of scratch (its contents are not kept)
+ * Steps on the GPU: RMSNorm1; QKV projection over the attention shards in
+ * broadcast order, whose epilogue writes K and V at their global rows (the
+ * all-gather); causal attention of local queries over the gathered K/V;
+ * out-projection with head-group partial sums in broadcast order plus the
+ * residual; RMSNorm2; W1 with GELU; W2 with its K loop over FFN shards in ring
+ * order (r+t) mod D, partial sums in the rank's fp32 accumulator, plus the
+ * residual.  bf16 tensor-core operands, fp32 accumulation, fp32 residual
+ * stream. */
+tsp_status tsp_layer_forward(tsp_plan_t plan, const void *x, const float *g1, const void *wqkv,
+                             const void *wo, const float *g2, const void *w1, const void *w2,
+                             void *y, void *saved, void *ws, void *stream);
+
+/* Backward of the folded layer (exact gradient of the forward; the pages give
+ * no backward schedule, so it runs the forward's collectives in reverse:
+ * weight-gradient pieces are summed over ranks in rank order, and key/value
+ * gradients are summed over every rank's queries and written back at the
+ * owning rank's rows).  Device pointers:
+ *   dy   bf16 [S][h] upstream gradient of the layer output, rank-major order
+ *   x, g1, wqkv, wo, g2, w1, w2  the forward's inputs
+ *   saved  the buffer filled by tsp_layer_forward with the same inputs
+ *   ws     ws_bytes of scratch
+ * Outputs: dx bf16 [S][h] rank-major order; dg1, dg2 float32 [h];
+ *   dwqkv float32 [3h][h], dwo float32 [h][h], dw1 float32 [F][h],
+ *   dw2 float32 [h][F]. */
+tsp_status tsp_layer_backward(tsp_plan_t plan, const void *dy, const void *x, const float *g1,
+                              const void *wqkv, const void *wo, const float *g2, const void *w1,
+                              const void *w2, const void *saved, void *ws, void *dx, float *dg1,
+                              float *dwqkv, float *dwo, float *dg2, float *dw1, float *dw2,
+                              void *stream);
+
+/* Wait for `stream`, then report TSP_ERR_CUDA for an asynchronous CUDA error
+ * or TSP_ERR_TIMEOUT if a device-side wait of this plan ran out (the flag is
+ * cleared by the report). */
+tsp_status tsp_sync_status(tsp_plan_t plan, void *stream);
+
+/* Static, human-readable name of a status. */
+const char *tsp_status_string(tsp_status status);
+
+/* Algorithmic floating-point work of one call, counting causal attention
+ * pairs only and no recompute: forward = 2S(4h^2 + 2hF) + 2hS(S+1);
+ * backward = 2 x forward.  Needs no GPU. */
+double tsp_layer_flops(tsp_plan_t plan, int backward);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSP_H */

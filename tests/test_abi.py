@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol the headers declare, and its integer outputs (zigzag map, shard
+schedules) match the oracle bit for bit; argument errors are reported."""
+
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import folded_tensor_sequence_map_b200 as T
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for hdr in ("tsp.h", "tsp_testing.h"):
+        src = open(os.path.join(ROOT, "include", hdr)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(tsp_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    import ctypes
+
+    declared = _declared_functions()
+    assert {"tsp_plan", "tsp_zigzag_map", "tsp_layer_forward", "tsp_layer_backward"} <= declared
+    lib = ctypes.CDLL(T.LIB_PATH)
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    assert declared == set(T.EXPORTED)
+
+
+@pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8),
+                                       (4096, 32, 16384, 131072, 8), (4096, 32, 16384, 131072, 16),
+                                       (4096, 32, 16384, 131072, 1), (256, 4, 1024, 2048, 4)])
+def test_zigzag_and_schedules_match_oracle(h, H, F, S, D):
+    p = T.tsp_plan(h, H, F, S, D)
+    assert np.array_equal(T.tsp_zigzag_map(p), O.zigzag_map(S, D).ravel())
+    for phase in (0, 1):
+        assert np.array_equal(T.tsp_shard_schedule(p, phase), O.shard_schedule(D, phase))
+
+
+def test_flops_formula_matches_workload_figures():
+    # algorithmic FLOPs of the forward: 24 S h^2 + 2 h S (S+1) for the 7B shape
+    for S, expect in ((256, None), (8192, 3.848e12), (32768, 2.199e13), (131072, 1.935e14)):
+        if expect is None:
+            p = T.tsp_plan(128, 4, 512, S, 2)
+            assert T.tsp_layer_flops(p, False) == 2 * S * (4 * 128**2 + 2 * 128 * 512) + 2 * 128 * S * (S + 1)
+            continue
+        p = T.tsp_plan(4096, 32, 16384, S, 8)
+        assert abs(T.tsp_layer_flops(p, False) / expect - 1) < 1e-3
+        assert T.tsp_layer_flops(p, True) == 2 * T.tsp_layer_flops(p, False)
+
+
+def test_workspace_sizes_cover_the_layout():
+    p = T.tsp_plan(128, 4, 512, 256, 2)
+    ws_t, saved_t = T.tsp_workspace_size(p, True)
+    ws_i, saved_i = T.tsp_workspace_size(p, False)
+    S, h, F, H = 256, 128, 512, 4
+    assert saved_i == 0 and ws_i == saved_t
+    assert saved_t >= S * h * 2 * 6 + S * h * 4 + S * F * 2 * 2 + H * S * 4 + 2 * S * 4
+    assert ws_t >= S * F * 2 + S * h * (4 + 4 + 2 + 2 + 4) + S * 3 * h * 2
+    names = ["rstd1", "a", "q", "k", "v", "o", "lse", "y", "rstd2", "b", "u", "g"]
+    offs = [T.tsp_test_buffer_offset(p, n) for n in names]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and offs[-1] < saved_t
+    with pytest.raises(T.TSPError):
+        T.tsp_test_buffer_offset(p, "nope")
+
+
+@pytest.mark.parametrize("args,status", [
+    ((128, 4, 512, 250, 2), "TSP_ERR_INDIVISIBLE"),
+    ((128, 3, 512, 256, 2), "TSP_ERR_INDIVISIBLE"),
+    ((128, 4, 511, 256, 2), "TSP_ERR_INDIVISIBLE"),
+    ((96, 4, 512, 256, 2), "TSP_ERR_UNSUPPORTED"),      # dh = 24
+    ((128, 4, 512, 128, 1), "TSP_ERR_UNSUPPORTED"),     # S % 256
+    ((128, 4, 512, 256, 4), "TSP_ERR_UNSUPPORTED"),     # S/D = 64 tokens per rank
+    ((0, 4, 512, 256, 2), "TSP_ERR_INVALID_ARG"),
+])
+def test_plan_rejects_bad_shapes(args, status):
+    with pytest.raises(T.TSPError) as e:
+        T.tsp_plan(*args)
+    assert T.STATUS_NAMES[e.value.status] == status
+    assert T.tsp_status_string(e.value.status) == status
+
+
+def test_bad_phase_is_rejected():
+    p = T.tsp_plan(128, 4, 512, 256, 2)
+    with pytest.raises(T.TSPError):
+        T.tsp_shard_schedule(p, 2)
