@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the folded TSP decoder layer on B200.
+
+One step = one pass of the whole hot path: the layer forward (RMSNorm1, QKV
+projection over the broadcast attention shards with the K/V all-gather in its
+epilogue, causal attention over the zigzag layout, out-projection + residual,
+RMSNorm2, W1 + GELU, ring-ordered W2 + residual) and its backward, over one
+batch of seeded synthetic inputs (7B-shaped layer: h=4096, 32 heads x 128,
+FFN 16384, S=131072 tokens, D=8 virtual ranks, bf16, weights N(0, 0.02),
+x and dY N(0, 1), seed 4).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tsp|reference]
+
+Prints one JSON line on rank 0.  With N > 1 (launched by torch.distributed.run)
+every rank runs an independent replica of the same layer ("replicas only": the
+folded layer's ranks are virtual ranks of one GPU), timed on the device and
+reduced with MAX over ranks.  ``--impl reference`` times the fp64 CPU oracle on
+the host cores instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth_inputs import WORKLOADS, LayerShape, make_layer_inputs  # noqa: E402
+
+METRIC = "TSP layer tokens/s (fwd, fwd+bwd) at S=128K, D=8; % bf16 tensor-core peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "7b_s128k"
+CPU_SAMPLE_S = 2048  # oracle sample: the same 7B layer at this many tokens
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def layer_flops(s: LayerShape, backward: bool) -> float:
+    fwd = 2.0 * s.S * (4.0 * s.h * s.h + 2.0 * s.h * s.ffn) + 2.0 * s.h * s.S * (s.S + 1.0)
+    return 2.0 * fwd if backward else fwd
+
+
+def stage_flops(s: LayerShape) -> dict:
+    """Algorithmic FLOPs of one launch of each stage (causal pairs only, no recompute)."""
+    S, h, F = float(s.S), float(s.h), float(s.ffn)
+    att = h * S * (S + 1.0)
+    return {
+        "fwd_qkv_gemm": 6 * S * h * h, "fwd_attention": 2 * att, "fwd_out_proj_gemm": 2 * S * h * h,
+        "fwd_w1_gelu_gemm": 2 * S * h * F, "fwd_w2_ring_gemm": 2 * S * h * F,
+        "bwd_dgelu_gemm": 2 * S * h * F, "bwd_dw2_gemm": 2 * S * h * F, "bwd_dw1_gemm": 2 * S * h * F,
+        "bwd_db_ring_gemm": 2 * S * h * F, "bwd_do_gemm": 2 * S * h * h, "bwd_dwo_gemm": 2 * S * h * h,
+        "bwd_attn_dkdv": 3 * att, "bwd_attn_dq": att, "bwd_dwqkv_gemm": 6 * S * h * h, "bwd_da_gemm": 6 * S * h * h,
+    }
+
+
+# ---------------------------------------------------------------------------
+# multi-process plumbing (N > 1: independent replicas)
+# ---------------------------------------------------------------------------
+
+def dist_setup(backend: str):
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return int(os.environ.get("RANK", "0")), world
+
+
+def reduce_max(value: float, device=None) -> float:
+    """MAX of a per-rank float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, flag in zip(self.NAMES, parts[3:7]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_seconds(shape: LayerShape, seed: int) -> tuple:
+    """Time the fp64 oracle's folded forward + backward of the same layer at
+    CPU_SAMPLE_S tokens.  Returns (seconds, sample_shape)."""
+    import oracle as O
+    from synth_inputs import bits_to_f32
+
+    s = LayerShape(h=shape.h, heads=shape.heads, ffn=shape.ffn, S=CPU_SAMPLE_S, D=shape.D)
+    inp = make_layer_inputs(s, seed)
+    zig = O.zigzag_map(s.S, s.D).ravel()
+    w = {k: bits_to_f32(inp[k]).astype(np.float64) for k in ("wqkv", "wo", "w1", "w2")}
+    w["g1"] = inp["g1"].astype(np.float64)
+    w["g2"] = inp["g2"].astype(np.float64)
+    x = bits_to_f32(inp["x"][zig]).astype(np.float64)
+    dy = bits_to_f32(inp["dy"][zig]).astype(np.float64)
+    t0 = time.perf_counter()
+    _, cache = O.tsp_layer_forward(x, w, s.heads, s.D)
+    O.tsp_layer_backward(dy, w, cache)
+    return time.perf_counter() - t0, s
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:  # noqa: BLE001
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(shape: LayerShape, seed: int, steps: int = 1) -> dict:
+    secs = []
+    for _ in range(steps):
+        t, s = oracle_sample_seconds(shape, seed)
+        secs.append(t)
+    t = statistics.median(secs)
+    full = layer_flops(shape, True)
+    samp = layer_flops(s, True)
+    projected = t * full / samp
+    return {
+        "value": shape.S / projected,
+        "unit": UNIT,
+        "cores": cpu_threads(),
+        "kind": "oracle",
+        "sample": (f"fp64 NumPy oracle, folded forward+backward of the same 7B layer at S={s.S}, D={s.D} "
+                   f"({t:.2f} s median of {len(secs)}), projected to S={shape.S} by algorithmic FLOPs "
+                   f"({full:.3e} / {samp:.3e})"),
+        "sample_seconds": t,
+    }
+
+
+def run_reference(args, shape: LayerShape, seed: int):
+    rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample_seconds(shape, seed)
+    base = cpu_baseline(shape, seed, steps=args.steps)
+    per_step = shape.S / base["value"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "h": shape.h, "heads": shape.heads, "ffn": shape.ffn, "seq_len": shape.S,
+                   "D": shape.D, "global_batch": 1, "parallelism": "virtual ranks on one device",
+                   "l2": "inputs larger than L2"},
+        "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU run
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    args = ap.parse_args()
+    shape, seed = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, shape, seed)
+        return
+
+    import torch
+
+    import folded_tensor_sequence_map_b200 as T
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    rank, world = dist_setup("nccl")
+    bf = torch.bfloat16
+
+    plan = T.tsp_plan(shape.h, shape.heads, shape.ffn, shape.S, shape.D)
+    zig = T.tsp_zigzag_map(plan)
+    inp = make_layer_inputs(shape, seed)
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(bf).to(dev)
+    x_host = torch.from_numpy(np.ascontiguousarray(inp["x"][zig]).view(np.int16)).view(bf).pin_memory()
+    dy_host = torch.from_numpy(np.ascontiguousarray(inp["dy"][zig]).view(np.int16)).view(bf).pin_memory()
+    W = {k: to_dev(inp[k]) for k in ("wqkv", "wo", "w1", "w2")}
+    g1 = torch.from_numpy(inp["g1"]).to(dev)
+    g2 = torch.from_numpy(inp["g2"]).to(dev)
+    del inp
+    x = x_host.to(dev)
+    dy = dy_host.to(dev)
+    S, h, F = shape.S, shape.h, shape.ffn
+    ws_n, saved_n = T.tsp_workspace_size(plan, True)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+    saved = torch.empty(saved_n, dtype=torch.uint8, device=dev)
+    y = torch.empty(S, h, dtype=bf, device=dev)
+    grads = dict(dx=torch.empty(S, h, dtype=bf, device=dev), dg1=torch.empty(h, device=dev),
+                 dwqkv=torch.empty(3 * h, h, device=dev), dwo=torch.empty(h, h, device=dev),
+                 dg2=torch.empty(h, device=dev), dw1=torch.empty(F, h, device=dev), dw2=torch.empty(h, F, device=dev))
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        T.tsp_layer_forward(plan, x, g1, W["wqkv"], W["wo"], g2, W["w1"], W["w2"], y, saved, ws, stream)
+
+    def bwd():
+        g = grads
+        T.tsp_layer_backward(plan, dy, x, g1, W["wqkv"], W["wo"], g2, W["w1"], W["w2"], saved, ws, g["dx"],
+                             g["dg1"], g["dwqkv"], g["dwo"], g["dg2"], g["dw1"], g["dw2"], stream)
+
+    def timed(fn, steps):
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        T.tsp_sync_status(plan, stream)
+        return reduce_max(a.elapsed_time(b) / 1e3, dev)
+
+    step = lambda: (fwd(), bwd())
+    for _ in range(args.warmup):
+        step()
+    T.tsp_sync_status(plan, stream)
+
+    # fwd+bwd: the headline, with per-stage events and clocks
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    launches0 = T.tsp_kernel_launches(plan)
+    T.tsp_profile_enable(plan, True)
+    with ClockSampler(gpu_id) as clk:
+        t_step = timed(step, args.steps)
+    launches = T.tsp_kernel_launches(plan) - launches0
+    stages = {}
+    for i in range(T.TSP_NUM_STAGES):
+        name, ms, calls, nk = T.tsp_profile_read(plan, i)
+        stages[name] = (ms, calls, nk)
+    T.tsp_profile_enable(plan, False)
+    for _ in range(2):
+        fwd()
+    t_fwd = timed(fwd, args.steps)
+
+    # end to end: pinned host inputs in, results out, inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        y_host = torch.empty(S, h, dtype=bf).pin_memory()
+        dx_host = torch.empty(S, h, dtype=bf).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_host, non_blocking=True)
+            dy.copy_(dy_host, non_blocking=True)
+            fwd()
+            bwd()
+            y_host.copy_(y, non_blocking=True)
+            dx_host.copy_(grads["dx"], non_blocking=True)
+
+        e2e_step()
+        t_e2e = timed(e2e_step, args.steps)
+        e2e = {"value": world * S * args.steps / t_e2e, "unit": UNIT,
+               "h2d_bytes_per_step": 2 * S * h * 2, "d2h_bytes_per_step": 2 * S * h * 2}
+
+    burst, sustained, hbm, src = peaks()
+    flops = stage_flops(shape)
+    total_ms = sum(v[0] for v in stages.values())
+    dom = max((k for k in flops), key=lambda k: stages[k][0])
+    dom_ms = stages[dom][0] / max(stages[dom][1], 1)
+    achieved = flops[dom] / (dom_ms / 1e3) / 1e12
+    value = world * S * args.steps / t_step
+    fwd_value = world * S * args.steps / t_fwd
+    frac_step = layer_flops(shape, True) * args.steps / t_step / 1e12 / sustained
+    frac_fwd = layer_flops(shape, False) * args.steps / t_fwd / 1e12 / sustained
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_step / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "h": h, "heads": shape.heads, "ffn": F, "seq_len": S, "D": shape.D,
+                   "global_batch": 1, "parallelism": "virtual ranks on one device; replicas across GPUs",
+                   "l2": "inputs larger than L2 (1 GiB activations per tensor)"},
+        "fwd": {"value": fwd_value, "unit": UNIT, "ms": t_fwd / args.steps * 1e3,
+                "frac_of_bf16_peak": frac_fwd},
+        "fwd_bwd_frac_of_bf16_peak": frac_step,
+        "peak_source": f"{src} (sustained {sustained} TFLOP/s for the step fractions)",
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                     "frac": achieved / sustained, "traffic": None,
+                     "peak_note": f"{src} sustained bf16 (kernel timed inside a long step)"},
+        "stage_ms_per_step": {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()},
+        "stage_share": {k: round(v[0] / total_ms, 4) for k, v in stages.items()},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        base = cpu_baseline(shape, seed)
+        line["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    T.tsp_plan_destroy  # noqa: B018  (plan freed with the object)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

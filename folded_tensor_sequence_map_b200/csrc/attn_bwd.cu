@@ -251,10 +251,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int qt = 0; qt < nqt; ++qt) {
                 if (bp.qtile_maxpos[qt] < kt * 128) continue;
                 any = true;
-                if (!mbar_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
+                if (!warp_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
                 // previous step's MMAs must be done reading P^T / dS^T
-                if (step > 0 && !mbar_wait(step_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
+                if (step > 0 && !warp_wait(step_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float s[32], dp[32];
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             if (!ok) break;
             if (!any) continue;
-            if (!mbar_wait(step_done, (step - 1) & 1, abort_flag, err)) break;
+            if (!warp_wait(step_done, (step - 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             const int lrow = a.inv_map[key];
             __nv_bfloat16 *dvrow = static_cast<__nv_bfloat16 *>(a.dv) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
@@ -459,9 +459,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int nkv = item_nkv(qt);
             bool ok = true;
             for (int j = 0; j < nkv; ++j, ++step) {
-                if (!mbar_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
+                if (!warp_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
-                if (step > 0 && !mbar_wait(ds_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
+                if (step > 0 && !warp_wait(ds_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float s[32], dp[32], dsv[32];
@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mbar_arrive(p_full);
             }
             if (!ok) break;
-            if (!mbar_wait(ds_done, (step - 1) & 1, abort_flag, err)) break;
+            if (!warp_wait(ds_done, (step - 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             __nv_bfloat16 *dqrow = static_cast<__nv_bfloat16 *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
 #pragma unroll 1
@@ -507,55 +507,85 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 template <int DH>
-cudaError_t launch_bwd_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
-                            const int *zig, const int *qtile_maxpos) {
-    using C = BCfg<DH>;
-    const int h = a.H * DH;
-    CUtensorMap mq, mk, mv, mdo;
-    const auto swz = swz_of<DH>();
-    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-    ok = ok && encode_tensor_map_2d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-    ok = ok && encode_tensor_map_2d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-    ok = ok && encode_tensor_map_2d(&mdo, a.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-    if (!ok) return cudaErrorInvalidValue;
+struct BwdMaps {
+    CUtensorMap q, k, v, dout;
+    bool make(const AttnBwdDesc &a) {
+        using C = BCfg<DH>;
+        const int h = a.H * DH;
+        const auto swz = swz_of<DH>();
+        bool ok = encode_tensor_map_2d(&q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        return ok;
+    }
+};
 
-    const int warps = a.S * a.H;
-    attn_delta_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.o),
-                                                                 static_cast<const __nv_bfloat16 *>(a.dout), a.delta,
-                                                                 a.S, a.H, DH);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-
+BwdParams make_params(const AttnBwdDesc &a, const int *zig, const int *qtile_maxpos) {
     BwdParams bp;
     bp.d = a;
     bp.zig = zig;
     bp.qtile_maxpos = qtile_maxpos;
     bp.num_items = (a.S / 128) * a.H;
+    return bp;
+}
+
+template <int DH>
+cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
+                             const int *qtile_maxpos) {
+    using C = BCfg<DH>;
+    BwdMaps<DH> m;
+    if (!m.make(a)) return cudaErrorInvalidValue;
+    const BwdParams bp = make_params(a, zig, qtile_maxpos);
     const int grid = bp.num_items < num_sms ? bp.num_items : num_sms;
-
-    const int smem_kv = 4 * C::TILE_BYTES + 2 * C::SQ_BYTES + 3 * 512 + 128 + 1024;
+    const int smem = 4 * C::TILE_BYTES + 2 * C::SQ_BYTES + 3 * 512 + 128 + 1024;
     auto k1 = attn_dkdv_kernel<DH>;
-    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k1<<<grid, kBwdThreads, smem_kv, st>>>(mq, mk, mv, mdo, bp, err);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    k1<<<grid, kBwdThreads, smem, st>>>(m.q, m.k, m.v, m.dout, bp, err);
+    return cudaGetLastError();
+}
 
+template <int DH>
+cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
+                           const int *qtile_maxpos) {
+    BwdMaps<DH> m;
+    if (!m.make(a)) return cudaErrorInvalidValue;
+    const BwdParams bp = make_params(a, zig, qtile_maxpos);
+    const int grid = bp.num_items < num_sms ? bp.num_items : num_sms;
     auto k2 = attn_dq_kernel<DH>;
-    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<DH>::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
-    k2<<<grid, kBwdThreads, DqCfg<DH>::SMEM, st>>>(mq, mk, mv, mdo, bp, err);
+    k2<<<grid, kBwdThreads, DqCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, bp, err);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attn_bwd_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
-                                 const int *zig, const int *qtile_maxpos) {
+cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st) {
+    const int warps = a.S * a.H;
+    attn_delta_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.o),
+                                                                 static_cast<const __nv_bfloat16 *>(a.dout), a.delta,
+                                                                 a.S, a.H, a.dh);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
+                             const int *qtile_maxpos) {
     switch (a.dh) {
-        case 32: return launch_bwd_impl<32>(a, err, num_sms, st, zig, qtile_maxpos);
-        case 64: return launch_bwd_impl<64>(a, err, num_sms, st, zig, qtile_maxpos);
-        case 128: return launch_bwd_impl<128>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 32: return launch_dkdv_impl<32>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 64: return launch_dkdv_impl<64>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 128: return launch_dkdv_impl<128>(a, err, num_sms, st, zig, qtile_maxpos);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_attn_dq(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
+                           const int *qtile_maxpos) {
+    switch (a.dh) {
+        case 32: return launch_dq_impl<32>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 64: return launch_dq_impl<64>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 128: return launch_dq_impl<128>(a, err, num_sms, st, zig, qtile_maxpos);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             float m = -INFINITY, l = 0.f;
             bool ok = true;
             for (int j = 0; j < nkv; ++j, ++tcount) {
-                if (!mbar_wait(&s_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
+                if (!warp_wait(&s_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
                 float s[128];
 #pragma unroll
@@ -299,9 +299,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 const float m_new = fmaxf(m, mt);
                 if (j > 0) {
-                    if (!mbar_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) { ok = false; break; }
+                    if (!warp_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
-                    if (m_new > m) {
+                    // TMEM loads/stores are warp-collective: rescale the whole
+                    // warp's rows when any row's max grew (alpha = 1 elsewhere).
+                    if (__any_sync(0xffffffffu, m_new > m)) {
                         const float alpha = ex2(m - m_new);
                         l *= alpha;
 #pragma unroll 1
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             if (!ok) break;
             // epilogue: wait for the last P V of this tile
-            if (!mbar_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) break;
+            if (!warp_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             const float inv = 1.0f / l;
             __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.o) + static_cast<int64_t>(lrow) * h + head * DH;

@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <cstdio>
 
 namespace tsp {
 
@@ -63,9 +64,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (clock64() - t0 > e.wait_limit) {
             *abort = 1;
             atomicOr(e.word, 1u);
+            printf("tsp: bounded wait gave up (block %d thread %d smem bar 0x%x parity %u)\n", blockIdx.x,
+                   threadIdx.x, smem_u32(bar), parity);
             return false;
         }
     }
+}
+
+// Warp-uniform wait for code that goes on to issue warp-collective
+// (.sync.aligned) tcgen05 instructions: all 32 lanes wait, and the warp
+// proceeds only if every lane saw the phase complete, so an abort can never
+// leave part of a warp inside a collective instruction.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, const DevErr &e) {
+    const bool ok = mbar_wait(bar, parity, abort, e);
+    return __all_sync(0xffffffffu, ok);
 }
 
 // ---- TMA --------------------------------------------------------------------

@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int mb, nb;
             tile_coords(t, mt, nt, mb, nb);
             const int m0 = mb * BM, n0 = nb * BN;
-            if (!mbar_wait(&acc_full[buf], acc_phase[buf], abort_flag, p.err)) break;
+            if (!warp_wait(&acc_full[buf], acc_phase[buf], abort_flag, p.err)) break;
             acc_phase[buf] ^= 1u;
             tc_fence_after();
             const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);

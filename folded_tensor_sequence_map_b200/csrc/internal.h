@@ -97,9 +97,13 @@ struct AttnBwdDesc {
     const int *kv_order;               // work order of (head, 128-key block), longest first
     const int *q_order;                // work order of (head, 128-row query block), longest first
 };
-// zig: local row -> global position; qtile_maxpos: largest position of each
-// 128-row local query tile.  Launches the Delta, dK/dV and dQ kernels.
-cudaError_t launch_attn_bwd_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
-                                 const int *zig, const int *qtile_maxpos);
+// Delta = rowsum(dO * O) per head; then dK/dV (key-tile items) and dQ
+// (query-tile items).  zig: local row -> global position; qtile_maxpos:
+// largest position of each 128-row local query tile.
+cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st);
+cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
+                             const int *qtile_maxpos);
+cudaError_t launch_attn_dq(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
+                           const int *qtile_maxpos);
 
 }  // namespace tsp

@@ -3,6 +3,9 @@
 // launch sequences.  Every step of the layer runs in the kernels of this
 // library; this file only validates arguments and enqueues launches.
 #include <algorithm>
+#include <chrono>
+#include <cstdio>
+#include <thread>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -31,6 +34,11 @@ struct tsp_plan_s {
     int fwd_items = 0;
     long long wait_limit = 0;
     std::mutex mu;
+    // profiling: per stage, the (start, stop) events recorded since enable
+    bool profiling = false;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof[TSP_NUM_STAGES];
+    int64_t prof_launches[TSP_NUM_STAGES] = {};
+    int64_t launches = 0;
 };
 
 namespace {
@@ -162,11 +170,8 @@ tsp_status ensure_device(tsp_plan_s *p) {
     if (cudaMemset(p->d_err, 0, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
     p->fwd_items = static_cast<int>(fitems.size());
     p->num_sms = prop.multiProcessorCount;
-    // A single wait may spin for about 2 s at the boost clock; the test hook
-    // can lower it.
-    long long limit = 4000000000LL;
-    if (const char *env = std::getenv("TSP_WAIT_LIMIT_CYCLES")) limit = std::atoll(env);
-    p->wait_limit = limit;
+    // A single device-side wait may spin for about 2 s at the boost clock.
+    p->wait_limit = 4000000000LL;
     p->device = dev;
     p->dev_ready = true;
     return TSP_OK;
@@ -183,6 +188,78 @@ tsp_status check_pending_error(tsp_plan_s *p) {
 }
 
 DevErr dev_err(const tsp_plan_s *p) { return DevErr{p->d_err, p->wait_limit}; }
+
+// Enqueue one stage (nk kernel launches); with profiling on, bracket it with
+// a pair of CUDA events on the same stream.
+extern const char *kStageNames[TSP_NUM_STAGES];
+
+// TSP_DEBUG_SYNC=1: after every stage, poll the stream for up to 30 s and log
+// the stage's completion (or that it is still running) to stderr.  For
+// localising a stuck or faulting kernel; off by default.
+bool debug_sync() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("TSP_DEBUG_SYNC");
+        v = (e && e[0] == '1') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+cudaError_t debug_wait(int id, cudaStream_t s) {
+    const auto t0 = std::chrono::steady_clock::now();
+    while (true) {
+        cudaError_t q = cudaStreamQuery(s);
+        double ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
+        if (q == cudaSuccess) {
+            std::fprintf(stderr, "[tsp] stage %-20s done (%.3f ms after launch)\n", kStageNames[id], ms);
+            return cudaSuccess;
+        }
+        if (q != cudaErrorNotReady) {
+            std::fprintf(stderr, "[tsp] stage %-20s failed: %s\n", kStageNames[id], cudaGetErrorString(q));
+            return q;
+        }
+        if (ms > 30000.0) {
+            std::fprintf(stderr, "[tsp] stage %-20s still running after 30 s\n", kStageNames[id]);
+            return cudaErrorLaunchTimeout;
+        }
+        std::this_thread::sleep_for(std::chrono::milliseconds(1));
+    }
+}
+
+template <class F>
+cudaError_t stage(tsp_plan_s *p, int id, int nk, cudaStream_t s, F &&launch) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (p->profiling) {
+        if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return cudaErrorUnknown;
+        cudaEventRecord(a, s);
+    }
+    cudaError_t e = launch();
+    if (p->profiling) {
+        cudaEventRecord(b, s);
+        p->prof[id].push_back({a, b});
+        p->prof_launches[id] += nk;
+    }
+    if (e == cudaSuccess) p->launches += nk;
+    if (e == cudaSuccess && debug_sync()) e = debug_wait(id, s);
+    return e;
+}
+
+void profile_clear(tsp_plan_s *p) {
+    for (auto &v : p->prof) {
+        for (auto &ev : v) {
+            cudaEventDestroy(ev.first);
+            cudaEventDestroy(ev.second);
+        }
+        v.clear();
+    }
+    for (auto &n : p->prof_launches) n = 0;
+}
+
+const char *kStageNames[TSP_NUM_STAGES] = {
+    "fwd_rmsnorm1", "fwd_qkv_gemm", "fwd_attention", "fwd_out_proj_gemm", "fwd_rmsnorm2", "fwd_w1_gelu_gemm",
+    "fwd_w2_ring_gemm", "bwd_dgelu_gemm", "bwd_dw2_gemm", "bwd_dw1_gemm", "bwd_db_ring_gemm", "bwd_rmsnorm2",
+    "bwd_do_gemm", "bwd_dwo_gemm", "bwd_attn_delta", "bwd_attn_dkdv", "bwd_attn_dq", "bwd_dwqkv_gemm",
+    "bwd_da_gemm", "bwd_rmsnorm1"};
 
 GemmDesc gemm(const void *A, int64_t lda, bool a_mn, const void *B, int64_t ldb, bool b_mn, int M, int N, int K,
               int epi, void *out, int64_t ldo) {
@@ -346,15 +423,20 @@ TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g
     auto *rstd2 = reinterpret_cast<float *>(base + l.rstd2);
     void *b = base + l.b, *u = base + l.u, *g = base + l.g;
 
-    cudaError_t e = launch_rmsnorm_fwd(x, nullptr, g1, a, rstd1, S, h, s);
-    if (e != cudaSuccess) return TSP_ERR_CUDA;
+    cudaError_t e;
+#define TSP_STAGE(id, nk, call)                                                  \
+    do {                                                                         \
+        if ((e = stage(p, id, nk, s, [&] { return (call); })) != cudaSuccess) \
+            return TSP_ERR_CUDA;                                                 \
+    } while (0)
+    TSP_STAGE(0, 1, launch_rmsnorm_fwd(x, nullptr, g1, a, rstd1, S, h, s));
     // QKV projection over the broadcast attention shards; K/V land at global rows.
     GemmDesc gq = gemm(a, h, false, wqkv, h, false, S, 3 * h, h, EPI_QKV, q, h);
     gq.rowmap = p->d_zig;
     gq.hsplit = h;
     gq.out_k = k;
     gq.out_v = v;
-    if ((e = launch_gemm(gq, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    TSP_STAGE(1, 1, launch_gemm(gq, err, p->num_sms, s));
     AttnDesc ad{};
     ad.S = S;
     ad.L = L;
@@ -369,24 +451,25 @@ TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g
     ad.lse = lse;
     ad.order = p->d_fwd_order;
     ad.num_items = p->fwd_items;
-    if ((e = launch_attn_fwd(ad, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    TSP_STAGE(2, 1, launch_attn_fwd(ad, err, p->num_sms, s));
     // out-projection (head-group partial sums in broadcast order) + residual, fp32 residual stream
     GemmDesc go = gemm(o, h, false, wo, h, false, S, h, h, EPI_RESID_F32, yres, h);
     go.aux = x;
     go.ldaux = h;
-    if ((e = launch_gemm(go, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
-    if ((e = launch_rmsnorm_fwd(nullptr, yres, g2, b, rstd2, S, h, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    TSP_STAGE(3, 1, launch_gemm(go, err, p->num_sms, s));
+    TSP_STAGE(4, 1, launch_rmsnorm_fwd(nullptr, yres, g2, b, rstd2, S, h, s));
     GemmDesc g1d = gemm(b, h, false, w1, h, false, S, F, h, EPI_GELU, u, F);
     g1d.out2 = g;
     g1d.ldo2 = F;
-    if ((e = launch_gemm(g1d, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    TSP_STAGE(5, 1, launch_gemm(g1d, err, p->num_sms, s));
     // W2 with the K loop over FFN shards in ring order (r + t) mod D, + residual
     GemmDesc g2d = gemm(g, F, false, w2, F, false, S, h, F, EPI_RESID_BF16, y, h);
     g2d.aux = yres;
     g2d.ldaux = h;
     g2d.ring_rows = L;
     g2d.ring_kblocks = (F / p->D) / 64;
-    if ((e = launch_gemm(g2d, err, p->num_sms, s)) != cudaSuccess) return TSP_ERR_CUDA;
+    TSP_STAGE(6, 1, launch_gemm(g2d, err, p->num_sms, s));
+#undef TSP_STAGE
     return TSP_OK;
 }
 
@@ -423,27 +506,27 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     float *da = reinterpret_cast<float *>(w + l.da);
     float *dgp = reinterpret_cast<float *>(w + l.dgp);
     cudaError_t e;
-#define TSP_LAUNCH(call)                          \
-    do {                                          \
-        if ((e = (call)) != cudaSuccess) return TSP_ERR_CUDA; \
+#define TSP_STAGE(id, nk, call)                                                  \
+    do {                                                                         \
+        if ((e = stage(p, id, nk, s, [&] { return (call); })) != cudaSuccess) \
+            return TSP_ERR_CUDA;                                                 \
     } while (0)
-
     // MLP ring backward: dU = (dY W2) * GELU'(U); dW2 = dY^T G; dW1 = dU^T b; db = dU W1 (ring K order)
     GemmDesc gdu = gemm(dy, h, false, w2, F, true, S, F, h, EPI_DGELU, du, F);
     gdu.aux = u;
     gdu.ldaux = F;
-    TSP_LAUNCH(launch_gemm(gdu, err, p->num_sms, s));
-    TSP_LAUNCH(launch_gemm(gemm(dy, h, true, g, F, true, h, F, S, EPI_F32, dw2, F), err, p->num_sms, s));
-    TSP_LAUNCH(launch_gemm(gemm(du, F, true, b, h, true, F, h, S, EPI_F32, dw1, h), err, p->num_sms, s));
+    TSP_STAGE(7, 1, launch_gemm(gdu, err, p->num_sms, s));
+    TSP_STAGE(8, 1, launch_gemm(gemm(dy, h, true, g, F, true, h, F, S, EPI_F32, dw2, F), err, p->num_sms, s));
+    TSP_STAGE(9, 1, launch_gemm(gemm(du, F, true, b, h, true, F, h, S, EPI_F32, dw1, h), err, p->num_sms, s));
     GemmDesc gdb = gemm(du, F, false, w1, h, true, S, h, F, EPI_F32, db, h);
     gdb.ring_rows = L;
     gdb.ring_kblocks = (F / p->D) / 64;
-    TSP_LAUNCH(launch_gemm(gdb, err, p->num_sms, s));
+    TSP_STAGE(10, 1, launch_gemm(gdb, err, p->num_sms, s));
     // RMSNorm2 backward + residual: dy = dY + RMSNorm2^T(db)
-    TSP_LAUNCH(launch_rmsnorm_bwd(db, nullptr, yres, rstd2, g2, dy, nullptr, dyf, dyb, dgp, dg2, S, h, s));
+    TSP_STAGE(11, 2, launch_rmsnorm_bwd(db, nullptr, yres, rstd2, g2, dy, nullptr, dyf, dyb, dgp, dg2, S, h, s));
     // out-projection backward: dO = dy Wo, dWo = dy^T O
-    TSP_LAUNCH(launch_gemm(gemm(dyb, h, false, wo, h, true, S, h, h, EPI_BF16, dO, h), err, p->num_sms, s));
-    TSP_LAUNCH(launch_gemm(gemm(dyb, h, true, o, h, true, h, h, S, EPI_F32, dwo, h), err, p->num_sms, s));
+    TSP_STAGE(12, 1, launch_gemm(gemm(dyb, h, false, wo, h, true, S, h, h, EPI_BF16, dO, h), err, p->num_sms, s));
+    TSP_STAGE(13, 1, launch_gemm(gemm(dyb, h, true, o, h, true, h, h, S, EPI_F32, dwo, h), err, p->num_sms, s));
     // attention backward; dK/dV reduced to the keys' owners
     AttnBwdDesc ab{};
     ab.S = S;
@@ -466,13 +549,15 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     ab.inv_map = p->d_inv;
     ab.kv_order = p->d_kv_order;
     ab.q_order = p->d_q_order;
-    TSP_LAUNCH(launch_attn_bwd_impl(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
+    TSP_STAGE(14, 1, launch_attn_delta(ab, s));
+    TSP_STAGE(15, 1, launch_attn_dkdv(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
+    TSP_STAGE(16, 1, launch_attn_dq(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
     // projection backward: dWqkv = [dQ|dK|dV]^T a, da = [dQ|dK|dV] Wqkv
-    TSP_LAUNCH(launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h), err, p->num_sms, s));
-    TSP_LAUNCH(launch_gemm(gemm(dqkv, 3 * h, false, wqkv, h, true, S, h, 3 * h, EPI_F32, da, h), err, p->num_sms, s));
+    TSP_STAGE(17, 1, launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h), err, p->num_sms, s));
+    TSP_STAGE(18, 1, launch_gemm(gemm(dqkv, 3 * h, false, wqkv, h, true, S, h, 3 * h, EPI_F32, da, h), err, p->num_sms, s));
     // RMSNorm1 backward + residual: dx = dy + RMSNorm1^T(da)
-    TSP_LAUNCH(launch_rmsnorm_bwd(da, x, nullptr, rstd1, g1, nullptr, dyf, nullptr, dx, dgp, dg1, S, h, s));
-#undef TSP_LAUNCH
+    TSP_STAGE(19, 2, launch_rmsnorm_bwd(da, x, nullptr, rstd1, g1, nullptr, dyf, nullptr, dx, dgp, dg1, S, h, s));
+#undef TSP_STAGE
     return TSP_OK;
 }
 
@@ -514,4 +599,64 @@ TSP_API tsp_status tsp_test_buffer_offset(tsp_plan_t p, const char *name, size_t
             return TSP_OK;
         }
     return TSP_ERR_INVALID_ARG;
+}
+
+// ===========================================================================
+// Profiling (tsp.h)
+// ===========================================================================
+
+TSP_API tsp_status tsp_profile_enable(tsp_plan_t p, int enable) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(p->mu);
+    profile_clear(p);
+    p->profiling = enable != 0;
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_profile_read(tsp_plan_t p, int stage_id, const char **name, double *total_ms,
+                                    int64_t *calls, int64_t *kernel_launches) {
+    if (!p || stage_id < 0 || stage_id >= TSP_NUM_STAGES) return TSP_ERR_INVALID_ARG;
+    double ms = 0.0;
+    for (auto &ev : p->prof[stage_id]) {
+        if (cudaEventSynchronize(ev.second) != cudaSuccess) return TSP_ERR_CUDA;
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, ev.first, ev.second) != cudaSuccess) return TSP_ERR_CUDA;
+        ms += t;
+    }
+    if (name) *name = kStageNames[stage_id];
+    if (total_ms) *total_ms = ms;
+    if (calls) *calls = static_cast<int64_t>(p->prof[stage_id].size());
+    if (kernel_launches) *kernel_launches = p->prof_launches[stage_id];
+    return TSP_OK;
+}
+
+TSP_API int64_t tsp_kernel_launches(tsp_plan_t p) { return p ? p->launches : 0; }
+
+// ===========================================================================
+// Bounded-wait self test (tsp_testing.h)
+// ===========================================================================
+
+namespace {
+__global__ void wait_timeout_kernel(DevErr err, int *result) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);  // nothing ever arrives on it
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    bool ok = mbar_wait(&bar, 0, &abort_flag, err);
+    __syncthreads();
+    if (threadIdx.x == 0) result[blockIdx.x] = ok ? 1 : 0;
+}
+}  // namespace
+
+TSP_API tsp_status tsp_test_wait_timeout(tsp_plan_t p, long long limit_cycles, int *result_dev, void *stream) {
+    if (!p || !result_dev || limit_cycles <= 0) return TSP_ERR_INVALID_ARG;
+    tsp_status st = ensure_device(p);
+    if (st != TSP_OK) return st;
+    DevErr e{p->d_err, limit_cycles};
+    wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(e, result_dev);
+    return cuda_status(cudaGetLastError());
 }

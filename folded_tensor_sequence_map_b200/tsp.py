@@ -39,9 +39,14 @@ EXPORTED = (
     "tsp_sync_status",
     "tsp_status_string",
     "tsp_layer_flops",
+    "tsp_profile_enable",
+    "tsp_profile_read",
+    "tsp_kernel_launches",
     "tsp_test_gemm",
     "tsp_test_buffer_offset",
+    "tsp_test_wait_timeout",
 )
+TSP_NUM_STAGES = 20
 
 
 class TSPError(RuntimeError):
@@ -79,6 +84,15 @@ def _load() -> ctypes.CDLL:
     lib.tsp_test_gemm.restype = I
     lib.tsp_test_buffer_offset.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(SZ)]
     lib.tsp_test_buffer_offset.restype = I
+    lib.tsp_profile_enable.argtypes = [P, I]
+    lib.tsp_profile_enable.restype = I
+    lib.tsp_profile_read.argtypes = [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(I64), ctypes.POINTER(I64)]
+    lib.tsp_profile_read.restype = I
+    lib.tsp_kernel_launches.argtypes = [P]
+    lib.tsp_kernel_launches.restype = I64
+    lib.tsp_test_wait_timeout.argtypes = [P, ctypes.c_longlong, V, V]
+    lib.tsp_test_wait_timeout.restype = I
     return lib
 
 
@@ -221,6 +235,24 @@ def tsp_sync_status(plan: Plan, stream=None) -> None:
     _check(_lib.tsp_sync_status(plan.handle, _stream(stream)), "tsp_sync_status")
 
 
+def tsp_profile_enable(plan: Plan, enable: bool) -> None:
+    _check(_lib.tsp_profile_enable(plan.handle, int(bool(enable))), "tsp_profile_enable")
+
+
+def tsp_profile_read(plan: Plan, stage: int):
+    """(name, total_ms, calls, kernel_launches) of one stage."""
+    name = ctypes.c_char_p()
+    ms = ctypes.c_double()
+    calls, launches = ctypes.c_int64(), ctypes.c_int64()
+    _check(_lib.tsp_profile_read(plan.handle, stage, ctypes.byref(name), ctypes.byref(ms), ctypes.byref(calls),
+                                 ctypes.byref(launches)), "tsp_profile_read")
+    return name.value.decode(), ms.value, calls.value, launches.value
+
+
+def tsp_kernel_launches(plan: Plan) -> int:
+    return _lib.tsp_kernel_launches(plan.handle)
+
+
 # ---- test hooks --------------------------------------------------------------
 
 def tsp_test_gemm(a_mn: bool, b_mn: bool, M: int, N: int, K: int, A, lda: int, B, ldb: int, C, ldc: int,
@@ -233,3 +265,8 @@ def tsp_test_buffer_offset(plan: Plan, name: str) -> int:
     off = ctypes.c_size_t()
     _check(_lib.tsp_test_buffer_offset(plan.handle, name.encode(), ctypes.byref(off)), "tsp_test_buffer_offset")
     return off.value
+
+
+def tsp_test_wait_timeout(plan: Plan, limit_cycles: int, result, stream=None) -> None:
+    _check(_lib.tsp_test_wait_timeout(plan.handle, limit_cycles, _ptr(result, "result"), _stream(stream)),
+           "tsp_test_wait_timeout")

@@ -144,6 +144,23 @@ tsp_status tsp_sync_status(tsp_plan_t plan, void *stream);
 /* Static, human-readable name of a status. */
 const char *tsp_status_string(tsp_status status);
 
+/* Kernel stages of one forward + backward, in launch order (profiling ids). */
+#define TSP_NUM_STAGES 20
+
+/* Per-stage timing with CUDA events.  tsp_profile_enable(plan, 1) clears the
+ * record and starts bracketing every stage of later layer calls with a pair of
+ * events on the call's stream; 0 stops.  tsp_profile_read waits for the
+ * recorded events of one stage (0 <= stage < TSP_NUM_STAGES) and returns its
+ * static name, the summed elapsed milliseconds, the number of calls recorded
+ * and the kernel launches they made.  Any output pointer may be NULL. */
+tsp_status tsp_profile_enable(tsp_plan_t plan, int enable);
+tsp_status tsp_profile_read(tsp_plan_t plan, int stage, const char **name, double *total_ms, int64_t *calls,
+                            int64_t *kernel_launches);
+
+/* Kernels this plan has launched since it was created (every layer call adds
+ * 7 for a forward and 15 for a backward). */
+int64_t tsp_kernel_launches(tsp_plan_t plan);
+
 /* Algorithmic floating-point work of one call, counting causal attention
  * pairs only and no recompute: forward = 2S(4h^2 + 2hF) + 2hS(S+1);
  * backward = 2 x forward.  Needs no GPU. */

@@ -36,6 +36,14 @@ tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A,
  * log2(e)/sqrt(dh)); rstd f32 [S].  TSP_ERR_INVALID_ARG for an unknown name. */
 tsp_status tsp_test_buffer_offset(tsp_plan_t plan, const char *name, size_t *offset);
 
+/* Self-test of the bounded device-side wait used by every kernel: launches one
+ * CTA that waits on an mbarrier nothing ever completes, with a limit of
+ * `limit_cycles` SM cycles.  The wait gives up, the kernel writes 0 to
+ * result_dev[0] (1 would mean the wait completed) and sets the plan's error
+ * flag, so the next tsp_sync_status() reports TSP_ERR_TIMEOUT.  No memory
+ * copy or tensor-core work is in flight, so giving up is safe. */
+tsp_status tsp_test_wait_timeout(tsp_plan_t plan, long long limit_cycles, int *result_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
