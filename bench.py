@@ -53,8 +53,14 @@ def peaks():
 
 
 def layer_flops(s: LayerShape, backward: bool) -> float:
+    """Algorithmic FLOPs of the forward (backward=False) or of the backward
+    alone (backward=True, twice the forward); a step is their sum."""
     fwd = 2.0 * s.S * (4.0 * s.h * s.h + 2.0 * s.h * s.ffn) + 2.0 * s.h * s.S * (s.S + 1.0)
     return 2.0 * fwd if backward else fwd
+
+
+def step_flops(s: LayerShape) -> float:
+    return layer_flops(s, False) + layer_flops(s, True)
 
 
 def stage_flops(s: LayerShape) -> dict:
@@ -208,8 +214,8 @@ def cpu_baseline(shape: LayerShape, seed: int, steps: int = 1) -> dict:
         t, s = oracle_sample_seconds(shape, seed)
         secs.append(t)
     t = statistics.median(secs)
-    full = layer_flops(shape, True)
-    samp = layer_flops(s, True)
+    full = step_flops(shape)
+    samp = step_flops(s)
     projected = t * full / samp
     return {
         "value": shape.S / projected,
@@ -257,8 +263,13 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--seq", type=int, default=0, help="override S of the workload (profiling runs)")
+    ap.add_argument("--ranks", type=int, default=0, help="override D of the workload (D sweep)")
     args = ap.parse_args()
     shape, seed = WORKLOADS[args.workload]
+    if args.seq or args.ranks:
+        shape = LayerShape(h=shape.h, heads=shape.heads, ffn=shape.ffn, S=args.seq or shape.S,
+                           D=args.ranks or shape.D)
     if args.impl == "reference":
         run_reference(args, shape, seed)
         return
@@ -365,7 +376,7 @@ def main():
     achieved = flops[dom] / (dom_ms / 1e3) / 1e12
     value = world * S * args.steps / t_step
     fwd_value = world * S * args.steps / t_fwd
-    frac_step = layer_flops(shape, True) * args.steps / t_step / 1e12 / sustained
+    frac_step = step_flops(shape) * args.steps / t_step / 1e12 / sustained
     frac_fwd = layer_flops(shape, False) * args.steps / t_fwd / 1e12 / sustained
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -377,6 +388,7 @@ def main():
         "fwd": {"value": fwd_value, "unit": UNIT, "ms": t_fwd / args.steps * 1e3,
                 "frac_of_bf16_peak": frac_fwd},
         "fwd_bwd_frac_of_bf16_peak": frac_step,
+        "fwd_bwd_frac_of_bf16_burst_peak": frac_step * sustained / burst,
         "peak_source": f"{src} (sustained {sustained} TFLOP/s for the step fractions)",
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
                      "frac": achieved / sustained, "traffic": None,
@@ -392,7 +404,7 @@ def main():
         line["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    T.tsp_plan_destroy  # noqa: B018  (plan freed with the object)
+    del plan
     import torch.distributed as dist
 
     if dist.is_available() and dist.is_initialized():

@@ -312,6 +312,284 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Pipelined dK/dV kernel: steps of 64 query rows.
+//   TMEM: S^T buffers [2] at columns 0 / 64, dP^T buffers [2] at 128 / 192,
+//         dV at 256, dK at 384 (128 key lanes each).
+//   The MMA warp issues S^T/dP^T of step g+1 before dV/dK of step g, so the
+//   tensor core works on the next step while the element-wise warps (two
+//   groups of four, 32 query columns each) turn step g into P^T and dS^T.
+template <int DH>
+struct KvCfg {
+    using C = BCfg<DH>;
+    static constexpr int BQ = 64;
+    static constexpr int QST = 3;
+    static constexpr int QTILE = BQ * DH * 2;
+    static constexpr int QATOM = BQ * C::SWB;
+    static constexpr int PT_BYTES = 128 * BQ * 2;
+    static constexpr int VEC_BYTES = 3 * BQ * 4;  // lse, delta, pos of one step
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + C::TILE_BYTES;
+    static constexpr int OFF_Q = OFF_V + C::TILE_BYTES;
+    static constexpr int OFF_DO = OFF_Q + QST * QTILE;
+    static constexpr int OFF_PT = OFF_DO + QST * QTILE;
+    static constexpr int OFF_DST = OFF_PT + PT_BYTES;
+    static constexpr int OFF_VEC = OFF_DST + PT_BYTES;
+    static constexpr int OFF_BAR = OFF_VEC + QST * VEC_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+};
+
+// K-major descriptor of a [64 rows][DH] sub-tile for K step kk (16 columns of DH).
+template <int DH>
+__device__ __forceinline__ uint64_t kdesc64(uint32_t base, int kk) {
+    using C = BCfg<DH>;
+    using K = KvCfg<DH>;
+    const int col = kk * 16;
+    return sdesc(base + (col / C::ATOM_COLS) * K::QATOM + (col % C::ATOM_COLS) * 2, 16, 8 * C::SWB, C::LAYOUT);
+}
+// MN-major descriptor of a [64 rows (K)][DH (N)] sub-tile for K step kk (16 rows).
+template <int DH>
+__device__ __forceinline__ uint64_t mndesc64(uint32_t base, int kk) {
+    using C = BCfg<DH>;
+    using K = KvCfg<DH>;
+    return sdesc(base + kk * 16 * C::SWB, K::QATOM, 8 * C::SWB, C::LAYOUT);
+}
+// K-major descriptor of a [128 rows][64 cols] bf16 operand (P^T, dS^T).
+__device__ __forceinline__ uint64_t pt_desc(uint32_t base, int kk) {
+    return sdesc(base + kk * 32, 16, 1024, kSwizzle128);
+}
+__device__ __forceinline__ int next_visible(const int *qmax64, int nq64, int from, int kv0) {
+    while (from < nq64 && qmax64[from] < kv0) ++from;
+    return from;
+}
+
+struct KvParams {
+    AttnBwdDesc d;
+    const int *zig;
+    const int *qmax64;  // per 64-row local query tile, largest global position
+    int num_items;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(320, 1)
+    attn_dkdv2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                      const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
+                      const KvParams kp, const DevErr err) {
+    using C = BCfg<DH>;
+    using K = KvCfg<DH>;
+    const AttnBwdDesc &a = kp.d;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+    uint64_t *kv_full = bars + 0, *kv_empty = bars + 1;
+    uint64_t *q_full = bars + 2;                 // [QST]
+    uint64_t *q_empty = q_full + K::QST;         // [QST]
+    uint64_t *s_full = q_empty + K::QST;         // [2]
+    uint64_t *p_full = s_full + 2;
+    uint64_t *pd_free = p_full + 1;
+    uint64_t *drain = pd_free + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nq64 = a.S / 64;
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
+    const float scale = rsqrtf(static_cast<float>(DH));
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        mbar_init(kv_empty, 1);
+        for (int s = 0; s < K::QST; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+        }
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(p_full, 256);
+        mbar_init(pd_free, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int item_iter = 0, g = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < kp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
+                if (!mbar_wait(kv_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
+                mbar_arrive_tx(kv_full, 2 * C::TILE_BYTES);
+                for (int t = 0; t < C::NATOM; ++t) {
+                    tma_load_2d(smem + K::OFF_K + t * C::ATOM_BYTES, &mK, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
+                    tma_load_2d(smem + K::OFF_V + t * C::ATOM_BYTES, &mV, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
+                }
+                for (int q = next_visible(kp.qmax64, nq64, 0, kt * 128); q < nq64;
+                     q = next_visible(kp.qmax64, nq64, q + 1, kt * 128), ++g) {
+                    const int s = g % K::QST;
+                    if (!mbar_wait(&q_empty[s], ((g / K::QST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(&q_full[s], 2 * K::QTILE + K::VEC_BYTES);
+                    for (int t = 0; t < C::NATOM; ++t) {
+                        tma_load_2d(smem + K::OFF_Q + s * K::QTILE + t * K::QATOM, &mQ, &q_full[s],
+                                    head * DH + t * C::ATOM_COLS, q * 64);
+                        tma_load_2d(smem + K::OFF_DO + s * K::QTILE + t * K::QATOM, &mdO, &q_full[s],
+                                    head * DH + t * C::ATOM_COLS, q * 64);
+                    }
+                    float *vec = reinterpret_cast<float *>(smem + K::OFF_VEC + s * K::VEC_BYTES);
+                    bulk_load(vec, a.lse + static_cast<int64_t>(head) * a.S + q * 64, 256, &q_full[s]);
+                    bulk_load(vec + 64, a.delta + static_cast<int64_t>(head) * a.S + q * 64, 256, &q_full[s]);
+                    bulk_load(vec + 128, kp.zig + q * 64, 256, &q_full[s]);
+                }
+            }
+            if (item_iter > 0) spin_drain(kv_full, (item_iter - 1) & 1, err.wait_limit);
+            for (int s = 0; s < K::QST; ++s)
+                if (g > s) {
+                    const int last = g - 1 - ((g - 1 - s) % K::QST);
+                    spin_drain(&q_full[s], (last / K::QST) & 1, err.wait_limit);
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
+            const uint32_t k_b = smem_u32(smem + K::OFF_K), v_b = smem_u32(smem + K::OFF_V);
+            const uint32_t pt_b = smem_u32(smem + K::OFF_PT), dst_b = smem_u32(smem + K::OFF_DST);
+            int item_iter = 0, g = 0;
+            bool ok = true;
+            auto issue_sdp = [&](int gi) -> bool {
+                const int s = gi % K::QST, b = gi & 1;
+                if (!mbar_wait(&q_full[s], (gi / K::QST) & 1, abort_flag, err)) return false;
+                tc_fence_after();
+                const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
+                const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    umma_bf16(tmem + 64 * b, kdesc<DH>(k_b, kk), kdesc64<DH>(q_b, kk), idS, kk > 0);
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(v_b, kk), kdesc64<DH>(do_b, kk), idS, kk > 0);
+                umma_commit(&s_full[b]);
+                return true;
+            };
+            for (int it = blockIdx.x; it < kp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kt = a.kv_order[it] / a.H;
+                const int kv0 = kt * 128;
+                if (!mbar_wait(kv_full, item_iter & 1, abort_flag, err)) break;
+                tc_fence_after();
+                int q = next_visible(kp.qmax64, nq64, 0, kv0);
+                if (q < nq64 && !issue_sdp(g)) break;
+                bool first = true;
+                while (q < nq64) {
+                    const int qn = next_visible(kp.qmax64, nq64, q + 1, kv0);
+                    if (qn < nq64 && !issue_sdp(g + 1)) { ok = false; break; }
+                    if (!mbar_wait(p_full, g & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    const int s = g % K::QST;
+                    const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
+                    const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
+                    for (int kk = 0; kk < K::BQ / 16; ++kk)
+                        umma_bf16(tmem + 256, pt_desc(pt_b, kk), mndesc64<DH>(do_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < K::BQ / 16; ++kk)
+                        umma_bf16(tmem + 384, pt_desc(dst_b, kk), mndesc64<DH>(q_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
+                    umma_commit(&q_empty[s]);
+                    umma_commit(pd_free);
+                    first = false;
+                    ++g;
+                    q = qn;
+                }
+                umma_commit(kv_empty);
+            }
+            if (!ok || *abort_flag) {
+                umma_commit(drain);
+                spin_drain(drain, 0, err.wait_limit);
+            }
+        }
+    } else {
+        const int wg = (warp - 2) / 4;          // query columns [32 wg, 32 wg + 32) of a step
+        const int quarter = warp & 3;
+        const int trow = quarter * 32 + lane;   // key row of the tile = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        uint8_t *sPt = smem + K::OFF_PT;
+        uint8_t *sdSt = smem + K::OFF_DST;
+        int g = 0;
+        for (int it = blockIdx.x; it < kp.num_items; it += gridDim.x) {
+            const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
+            const int kv0 = kt * 128;
+            const int key = kv0 + trow;
+            bool ok = true, any = false;
+            for (int q = next_visible(kp.qmax64, nq64, 0, kv0); q < nq64;
+                 q = next_visible(kp.qmax64, nq64, q + 1, kv0), ++g) {
+                any = true;
+                const int b = g & 1, s = g % K::QST;
+                if (!warp_wait(&s_full[b], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                float sv[32], dp[32];
+                tmem_ld32(tmem + lane_off + 64 * b + 32 * wg, sv);
+                tmem_ld32(tmem + lane_off + 128 + 64 * b + 32 * wg, dp);
+                tmem_ld_wait();
+                const float *vec = reinterpret_cast<const float *>(smem + K::OFF_VEC + s * K::VEC_BYTES);
+                const int *pos = reinterpret_cast<const int *>(vec + 128);
+                float pv[32], dsv[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = 32 * wg + e;
+                    const float p = (key <= pos[c]) ? ex2b(sv[e] * sl2 - vec[c]) : 0.f;
+                    pv[e] = p;
+                    dsv[e] = p * (dp[e] - vec[64 + c]);
+                }
+                // the previous step's dV/dK MMAs must be done reading P^T / dS^T
+                if (g > 0 && !warp_wait(pd_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int col = 32 * wg + qq * 8;
+                    const int chunk = (col >> 3) ^ (trow & 7);
+                    *reinterpret_cast<uint4 *>(sPt + trow * 128 + chunk * 16) =
+                        make_uint4(pack_bf16(pv[8 * qq], pv[8 * qq + 1]), pack_bf16(pv[8 * qq + 2], pv[8 * qq + 3]),
+                                   pack_bf16(pv[8 * qq + 4], pv[8 * qq + 5]), pack_bf16(pv[8 * qq + 6], pv[8 * qq + 7]));
+                    *reinterpret_cast<uint4 *>(sdSt + trow * 128 + chunk * 16) =
+                        make_uint4(pack_bf16(dsv[8 * qq], dsv[8 * qq + 1]), pack_bf16(dsv[8 * qq + 2], dsv[8 * qq + 3]),
+                                   pack_bf16(dsv[8 * qq + 4], dsv[8 * qq + 5]), pack_bf16(dsv[8 * qq + 6], dsv[8 * qq + 7]));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            if (!any) continue;
+            if (!warp_wait(pd_free, (g - 1) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            // group 0 writes dV, group 1 writes dK (scaled), at the key owner's local row
+            const int lrow = a.inv_map[key];
+            void *dst = wg == 0 ? a.dv : a.dk;
+            const float f = wg == 0 ? 1.0f : scale;
+            __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(dst) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + 256 + 128 * wg + c * 32, v);
+                tmem_ld_wait();
+                uint4 *d4 = reinterpret_cast<uint4 *>(row + c * 32);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+                    d4[qq] = make_uint4(pack_bf16(v[8 * qq] * f, v[8 * qq + 1] * f), pack_bf16(v[8 * qq + 2] * f, v[8 * qq + 3] * f),
+                                        pack_bf16(v[8 * qq + 4] * f, v[8 * qq + 5] * f), pack_bf16(v[8 * qq + 6] * f, v[8 * qq + 7] * f));
+            }
+            tc_fence_before();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
 template <int DH>
 struct DqCfg {
     using C = BCfg<DH>;
@@ -532,17 +810,26 @@ BwdParams make_params(const AttnBwdDesc &a, const int *zig, const int *qtile_max
 
 template <int DH>
 cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
-                             const int *qtile_maxpos) {
+                             const int *qmax64) {
     using C = BCfg<DH>;
     BwdMaps<DH> m;
     if (!m.make(a)) return cudaErrorInvalidValue;
-    const BwdParams bp = make_params(a, zig, qtile_maxpos);
-    const int grid = bp.num_items < num_sms ? bp.num_items : num_sms;
-    const int smem = 4 * C::TILE_BYTES + 2 * C::SQ_BYTES + 3 * 512 + 128 + 1024;
-    auto k1 = attn_dkdv_kernel<DH>;
-    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // Q and dO sub-tiles of 64 rows
+    const int h = a.H * DH;
+    const auto swz = swz_of<DH>();
+    bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    if (!ok) return cudaErrorInvalidValue;
+    KvParams kp;
+    kp.d = a;
+    kp.zig = zig;
+    kp.qmax64 = qmax64;
+    kp.num_items = (a.S / 128) * a.H;
+    const int grid = kp.num_items < num_sms ? kp.num_items : num_sms;
+    auto k1 = attn_dkdv2_kernel<DH>;
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, KvCfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
-    k1<<<grid, kBwdThreads, smem, st>>>(m.q, m.k, m.v, m.dout, bp, err);
+    k1<<<grid, 320, KvCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, kp, err);
     return cudaGetLastError();
 }
 

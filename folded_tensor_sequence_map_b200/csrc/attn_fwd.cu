@@ -16,7 +16,7 @@
 //   warps 2-5  softmax group 0 (query tile 0), warps 6-9 group 1: thread =
 //              query row; online softmax in the log2 domain, P written to
 //              shared memory as bf16 in the MMA's 128B-swizzled K-major
-//              layout; O rescaled in TMEM when the running max grows; final
+//              layout; O rescaled in TMEM when the running max grows by more than 2^8; final
 //              O / l written as bf16 and LSE (log2 domain) as fp32.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+dh), O1 [384,384+dh).
 #include "common.cuh"
@@ -297,14 +297,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         mt = fmaxf(mt, s[c]);
                     }
                 }
+                // Lazy rescaling: keep the running max unless a row's max grew
+                // by more than 8 (log2 units), so P stays below 2^8 in bf16 and
+                // O is rescaled in TMEM only rarely.
                 const float m_new = fmaxf(m, mt);
+                const float m_use = (j == 0 || m_new - m > 8.0f) ? m_new : m;
                 if (j > 0) {
                     if (!warp_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
                     // TMEM loads/stores are warp-collective: rescale the whole
-                    // warp's rows when any row's max grew (alpha = 1 elsewhere).
-                    if (__any_sync(0xffffffffu, m_new > m)) {
-                        const float alpha = ex2(m - m_new);
+                    // warp's rows when any row's max moved (alpha = 1 elsewhere).
+                    if (__any_sync(0xffffffffu, m_use != m)) {
+                        const float alpha = ex2(m - m_use);
                         l *= alpha;
 #pragma unroll 1
                         for (int c = 0; c < DH / 32; ++c) {
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         tmem_st_wait();
                     }
                 }
-                m = m_new;
+                m = m_use;
                 float ls = 0.f;
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {

@@ -97,12 +97,12 @@ struct AttnBwdDesc {
     const int *kv_order;               // work order of (head, 128-key block), longest first
     const int *q_order;                // work order of (head, 128-row query block), longest first
 };
-// Delta = rowsum(dO * O) per head; then dK/dV (key-tile items) and dQ
-// (query-tile items).  zig: local row -> global position; qtile_maxpos:
-// largest position of each 128-row local query tile.
+// Delta = rowsum(dO * O) per head; then dK/dV (key-tile items, 64-row query
+// steps) and dQ (query-tile items).  zig: local row -> global position;
+// qmax64 / qtile_maxpos: largest position of each 64- / 128-row local query tile.
 cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st);
 cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
-                             const int *qtile_maxpos);
+                             const int *qmax64);
 cudaError_t launch_attn_dq(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
                            const int *qtile_maxpos);
 

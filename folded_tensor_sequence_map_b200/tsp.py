@@ -112,8 +112,9 @@ class Plan:
         self.h, self.heads, self.ffn, self.S, self.D = h, heads, ffn, S, D
 
     def __del__(self):
-        if getattr(self, "handle", None) is not None and self.handle.value:
-            _lib.tsp_plan_destroy(self.handle)
+        lib = globals().get("_lib")
+        if lib is not None and getattr(self, "handle", None) is not None and self.handle.value:
+            lib.tsp_plan_destroy(self.handle)
             self.handle = None
 
 
