@@ -42,6 +42,7 @@ EXPORTED = (
     "tsp_profile_enable",
     "tsp_profile_read",
     "tsp_kernel_launches",
+    "tsp_rmsnorm_backward_noalloc",
     "tsp_test_gemm",
     "tsp_test_buffer_offset",
     "tsp_test_wait_timeout",
@@ -91,6 +92,8 @@ def _load() -> ctypes.CDLL:
     lib.tsp_profile_read.restype = I
     lib.tsp_kernel_launches.argtypes = [P]
     lib.tsp_kernel_launches.restype = I64
+    lib.tsp_rmsnorm_backward_noalloc.argtypes = [V, V, V, V, V, V, V, I, I, V]
+    lib.tsp_rmsnorm_backward_noalloc.restype = I
     lib.tsp_test_wait_timeout.argtypes = [P, ctypes.c_longlong, V, V]
     lib.tsp_test_wait_timeout.restype = I
     return lib
@@ -252,6 +255,18 @@ def tsp_profile_read(plan: Plan, stage: int):
 
 def tsp_kernel_launches(plan: Plan) -> int:
     return _lib.tsp_kernel_launches(plan.handle)
+
+
+def tsp_rmsnorm_backward_noalloc(dout, x, rstd, g, resid, dx, dg, rows: int, h: int, stream=None) -> None:
+    """RMSNorm backward + residual with library-owned scratch (no allocation);
+    see include/tsp.h for the contract."""
+    import torch
+
+    f32, bf = torch.float32, torch.bfloat16
+    _check(_lib.tsp_rmsnorm_backward_noalloc(
+        _ptr(dout, "dout", f32, (rows, h)), _ptr(x, "x", bf, (rows, h)), _ptr(rstd, "rstd", f32, (rows,)),
+        _ptr(g, "g", f32, (h,)), _ptr(resid, "resid", f32, (rows, h)), _ptr(dx, "dx", bf, (rows, h)),
+        _ptr(dg, "dg", f32, (h,)), rows, h, _stream(stream)), "tsp_rmsnorm_backward_noalloc")
 
 
 # ---- test hooks --------------------------------------------------------------

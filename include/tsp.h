@@ -161,6 +161,35 @@ tsp_status tsp_profile_read(tsp_plan_t plan, int stage, const char **name, doubl
  * 7 for a forward and 15 for a backward). */
 int64_t tsp_kernel_launches(tsp_plan_t plan);
 
+/* RMSNorm backward plus residual that allocates nothing.  The TSP pages have
+ * no counterpart: this is a library convenience.  It computes what the last
+ * stage of tsp_layer_backward computes for RMSNorm1:
+ *     n = x * rstd,   dn = dout * g,
+ *     dx = resid + rstd * (dn - n * mean(dn * n))      (bf16 out)
+ *     dg = sum over rows of dout * n                    (float32 out)
+ * for callers that cannot allocate device memory (no cudaMalloc allowed in
+ * their context, or no memory pool to draw scratch from).  The per-block
+ * partial sums of dg live in a 16 MiB device array owned by the library, which
+ * every GPU that loads the library holds until the process exits; the call
+ * needs only its inputs and outputs.  Device pointers, 16-byte aligned:
+ *   dout  float32 [rows][h]  gradient reaching the normalised output
+ *   x     bf16    [rows][h]  the normalised input
+ *   rstd  float32 [rows]     1/sqrt(mean(x^2) + eps) from the forward
+ *   g     float32 [h]        gain
+ *   resid float32 [rows][h]  gradient reaching x through the residual branch
+ *   dx    bf16    [rows][h]  output
+ *   dg    float32 [h]        output
+ * Limits: h % 128 == 0 and ceil(rows / 64) * h <= 4,194,304; beyond them the
+ * call returns TSP_ERR_UNSUPPORTED and enqueues nothing.  The first call on a
+ * device looks up the array's device address with that device current; make
+ * that first call before any stream capture.  All calls share the one array:
+ * calls that overlap on the GPU (on different streams or from different host
+ * threads) race, so the caller must order them.  Nothing in the array needs
+ * clearing between calls, since each call writes every slot it reads.
+ * Asynchronous on `stream`. */
+tsp_status tsp_rmsnorm_backward_noalloc(const float *dout, const void *x, const float *rstd, const float *g,
+                                        const float *resid, void *dx, float *dg, int rows, int h, void *stream);
+
 /* Algorithmic floating-point work of one call, counting causal attention
  * pairs only and no recompute: forward = 2S(4h^2 + 2hF) + 2hS(S+1);
  * backward = 2 x forward.  Needs no GPU. */
