@@ -539,7 +539,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int c = 32 * wg + e;
-                    const float p = (key <= pos[c]) ? ex2b(sv[e] * sl2 - vec[c]) : 0.f;
+                    const float pe = ex2b(fmaf(sv[e], sl2, -vec[c]));
+                    const float p = (key <= pos[c]) ? pe : 0.f;
                     pv[e] = p;
                     dsv[e] = p * (dp[e] - vec[64 + c]);
                 }
@@ -579,6 +580,229 @@ __global__ void __launch_bounds__(320, 1)
                 for (int qq = 0; qq < 4; ++qq)
                     d4[qq] = make_uint4(pack_bf16(v[8 * qq] * f, v[8 * qq + 1] * f), pack_bf16(v[8 * qq + 2] * f, v[8 * qq + 3] * f),
                                         pack_bf16(v[8 * qq + 4] * f, v[8 * qq + 5] * f), pack_bf16(v[8 * qq + 6] * f, v[8 * qq + 7] * f));
+            }
+            tc_fence_before();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// Pipelined dQ kernel: one item = (head, 128-row query tile); steps of 64 keys.
+//   TMEM: S buffers [2] at columns 0 / 64, dP buffers [2] at 128 / 192, dQ at
+//   256 (128 query lanes).  The MMA warp issues S/dP of step j+1 before dQ of
+//   step j, so the tensor core works while the element-wise warps (two groups
+//   of four, 32 key columns each) turn step j into dS.
+template <int DH>
+struct Dq2Cfg {
+    using C = BCfg<DH>;
+    static constexpr int BK = 64;
+    static constexpr int KST = 3;
+    static constexpr int KTILE = BK * DH * 2;   // one K or V sub-tile of 64 keys
+    static constexpr int KATOM = BK * C::SWB;
+    static constexpr int DS_BYTES = 128 * BK * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_DO = OFF_Q + C::TILE_BYTES;
+    static constexpr int OFF_K = OFF_DO + C::TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + KST * KTILE;
+    static constexpr int OFF_DS = OFF_V + KST * KTILE;
+    static constexpr int OFF_BAR = OFF_DS + DS_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(320, 1)
+    attn_dq2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                    const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
+                    const BwdParams bp, const DevErr err) {
+    using C = BCfg<DH>;
+    using Q = Dq2Cfg<DH>;
+    const AttnBwdDesc &a = bp.d;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Q::OFF_BAR);
+    uint64_t *q_full = bars + 0, *q_empty = bars + 1;
+    uint64_t *k_full = bars + 2;            // [KST]
+    uint64_t *k_empty = k_full + Q::KST;    // [KST]
+    uint64_t *s_full = k_empty + Q::KST;    // [2]
+    uint64_t *p_full = s_full + 2;
+    uint64_t *ds_free = p_full + 1;
+    uint64_t *drain = ds_free + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
+    const float scale = rsqrtf(static_cast<float>(DH));
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < Q::KST; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(p_full, 256);
+        mbar_init(ds_free, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto nkv64 = [&](int qt) { return bp.qtile_maxpos[qt] / 64 + 1; };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int item_iter = 0, g = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
+                if (!mbar_wait(q_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
+                mbar_arrive_tx(q_full, 2 * C::TILE_BYTES);
+                for (int t = 0; t < C::NATOM; ++t) {
+                    tma_load_2d(smem + Q::OFF_Q + t * C::ATOM_BYTES, &mQ, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
+                    tma_load_2d(smem + Q::OFF_DO + t * C::ATOM_BYTES, &mdO, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
+                }
+                const int n = nkv64(qt);
+                for (int j = 0; j < n; ++j, ++g) {
+                    const int s = g % Q::KST;
+                    if (!mbar_wait(&k_empty[s], ((g / Q::KST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(&k_full[s], 2 * Q::KTILE);
+                    for (int t = 0; t < C::NATOM; ++t) {
+                        tma_load_2d(smem + Q::OFF_K + s * Q::KTILE + t * Q::KATOM, &mK, &k_full[s],
+                                    head * DH + t * C::ATOM_COLS, j * 64);
+                        tma_load_2d(smem + Q::OFF_V + s * Q::KTILE + t * Q::KATOM, &mV, &k_full[s],
+                                    head * DH + t * C::ATOM_COLS, j * 64);
+                    }
+                }
+            }
+            if (item_iter > 0) spin_drain(q_full, (item_iter - 1) & 1, err.wait_limit);
+            for (int s = 0; s < Q::KST; ++s)
+                if (g > s) {
+                    const int last = g - 1 - ((g - 1 - s) % Q::KST);
+                    spin_drain(&k_full[s], (last / Q::KST) & 1, err.wait_limit);
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
+            const uint32_t q_b = smem_u32(smem + Q::OFF_Q), do_b = smem_u32(smem + Q::OFF_DO);
+            const uint32_t ds_b = smem_u32(smem + Q::OFF_DS);
+            int item_iter = 0, g = 0;
+            bool ok = true;
+            auto issue_sdp = [&](int gi) -> bool {
+                const int s = gi % Q::KST, b = gi & 1;
+                if (!mbar_wait(&k_full[s], (gi / Q::KST) & 1, abort_flag, err)) return false;
+                tc_fence_after();
+                const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
+                const uint32_t v_b = smem_u32(smem + Q::OFF_V + s * Q::KTILE);
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    umma_bf16(tmem + 64 * b, kdesc<DH>(q_b, kk), kdesc64<DH>(k_b, kk), idS, kk > 0);
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(do_b, kk), kdesc64<DH>(v_b, kk), idS, kk > 0);
+                umma_commit(&s_full[b]);
+                return true;
+            };
+            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int qt = a.q_order[it] / a.H;
+                if (!mbar_wait(q_full, item_iter & 1, abort_flag, err)) break;
+                tc_fence_after();
+                const int n = nkv64(qt);
+                if (!issue_sdp(g)) break;
+                for (int j = 0; j < n; ++j, ++g) {
+                    if (j + 1 < n && !issue_sdp(g + 1)) { ok = false; break; }
+                    if (!mbar_wait(p_full, g & 1, abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    const int s = g % Q::KST;
+                    const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
+                    for (int kk = 0; kk < Q::BK / 16; ++kk)
+                        umma_bf16(tmem + 256, pt_desc(ds_b, kk), mndesc64<DH>(k_b, kk), idG, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&k_empty[s]);
+                    umma_commit(ds_free);
+                }
+                umma_commit(q_empty);
+            }
+            if (!ok || *abort_flag) {
+                umma_commit(drain);
+                spin_drain(drain, 0, err.wait_limit);
+            }
+        }
+    } else {
+        const int wg = (warp - 2) / 4;          // key columns [32 wg, 32 wg + 32) of a step
+        const int quarter = warp & 3;
+        const int trow = quarter * 32 + lane;   // query row of the tile = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        uint8_t *sDS = smem + Q::OFF_DS;
+        int g = 0;
+        for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
+            const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
+            const int lrow = qt * 128 + trow;
+            const int pos = bp.zig[lrow];
+            const float lse = a.lse[static_cast<int64_t>(head) * a.S + lrow];
+            const float dl = a.delta[static_cast<int64_t>(head) * a.S + lrow];
+            const int n = nkv64(qt);
+            bool ok = true;
+            for (int j = 0; j < n; ++j, ++g) {
+                const int b = g & 1;
+                if (!warp_wait(&s_full[b], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                float sv[32], dp[32], dsv[32];
+                tmem_ld32(tmem + lane_off + 64 * b + 32 * wg, sv);
+                tmem_ld32(tmem + lane_off + 128 + 64 * b + 32 * wg, dp);
+                tmem_ld_wait();
+                const int k0 = j * 64 + 32 * wg;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float pe = ex2b(fmaf(sv[e], sl2, -lse));
+                    const float p = (k0 + e <= pos) ? pe : 0.f;
+                    dsv[e] = p * (dp[e] - dl);
+                }
+                if (g > 0 && !warp_wait(ds_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int col = 32 * wg + qq * 8;
+                    const int chunk = (col >> 3) ^ (trow & 7);
+                    *reinterpret_cast<uint4 *>(sDS + trow * 128 + chunk * 16) =
+                        make_uint4(pack_bf16(dsv[8 * qq], dsv[8 * qq + 1]), pack_bf16(dsv[8 * qq + 2], dsv[8 * qq + 3]),
+                                   pack_bf16(dsv[8 * qq + 4], dsv[8 * qq + 5]), pack_bf16(dsv[8 * qq + 6], dsv[8 * qq + 7]));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            if (!warp_wait(ds_free, (g - 1) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            if (wg == 0) {
+                __nv_bfloat16 *dqrow = static_cast<__nv_bfloat16 *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+#pragma unroll 1
+                for (int c = 0; c < DH / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_off + 256 + c * 32, v);
+                    tmem_ld_wait();
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dqrow + c * 32);
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq)
+                        d4[qq] = make_uint4(pack_bf16(v[8 * qq] * scale, v[8 * qq + 1] * scale),
+                                            pack_bf16(v[8 * qq + 2] * scale, v[8 * qq + 3] * scale),
+                                            pack_bf16(v[8 * qq + 4] * scale, v[8 * qq + 5] * scale),
+                                            pack_bf16(v[8 * qq + 6] * scale, v[8 * qq + 7] * scale));
+                }
             }
             tc_fence_before();
         }
@@ -836,14 +1060,21 @@ cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sm
 template <int DH>
 cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
                            const int *qtile_maxpos) {
+    using C = BCfg<DH>;
     BwdMaps<DH> m;
     if (!m.make(a)) return cudaErrorInvalidValue;
+    // K and V sub-tiles of 64 keys
+    const int h = a.H * DH;
+    const auto swz = swz_of<DH>();
+    bool ok = encode_tensor_map_2d(&m.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    ok = ok && encode_tensor_map_2d(&m.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    if (!ok) return cudaErrorInvalidValue;
     const BwdParams bp = make_params(a, zig, qtile_maxpos);
     const int grid = bp.num_items < num_sms ? bp.num_items : num_sms;
-    auto k2 = attn_dq_kernel<DH>;
-    cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<DH>::SMEM);
+    auto k2 = attn_dq2_kernel<DH>;
+    cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, Dq2Cfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
-    k2<<<grid, kBwdThreads, DqCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, bp, err);
+    k2<<<grid, 320, Dq2Cfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, bp, err);
     return cudaGetLastError();
 }
 

@@ -8,7 +8,7 @@
 // Work item = (head, block of 256 local query rows) = two 128-row query tiles.
 // CTA layout (10 warps, persistent, one CTA per SM):
 //   warp 0     TMA producer: the two Q tiles of the item, then K_j / V_j tiles
-//              of 128 keys (K ring of 2, V ring of 1 or 2 slots).
+//              of 128 keys (K ring of 1 or 2 slots, V ring of 2).
 //   warp 1     TMEM owner and MMA issuer: S_w = Q_w K_j^T (128x128, fp32 in
 //              TMEM) and O_w += P_w V_j (128 x dh, fp32 in TMEM) for w = 0, 1,
 //              ordered so that S of the next tile overlaps the softmax of the
@@ -48,8 +48,10 @@ struct FwdCfg {
     static constexpr int TILE_BYTES = 128 * DH * 2;           // one 128-row tile of Q, K or V
     static constexpr int ATOM_BYTES = 128 * SWB;
     static constexpr uint32_t LAYOUT = SWB == 128 ? kSwizzle128 : (SWB == 64 ? kSwizzle64 : kSwizzle32);
-    static constexpr int KST = 2;
-    static constexpr int VST = DH == 128 ? 1 : 2;
+    // K_j is read by both S MMAs long before P V needs V_j, so a single K slot
+    // is enough; V gets two so its next tile loads during the softmax.
+    static constexpr int KST = DH == 128 ? 1 : 2;
+    static constexpr int VST = 2;
     static constexpr int P_BYTES = 128 * 128 * 2;
     // smem map (1024-aligned pieces)
     static constexpr int OFF_Q = 0;
@@ -283,23 +285,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 tmem_ld_wait();
                 const int kv0 = j * 128;
-                float mt = -INFINITY;
-                if (kv0 + 127 <= pos) {
+                // Row max on the raw scores (the scale is positive), masking
+                // only on tiles that reach past this row's position.
+                const bool full = kv0 + 127 <= pos;
+                // eight independent partial maxima: no 128-long dependency chain
+                float mx[8];
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        s[c] *= sl2;
-                        mt = fmaxf(mt, s[c]);
-                    }
+                for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+                if (full) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
                 } else {
 #pragma unroll
                     for (int c = 0; c < 128; ++c) {
-                        s[c] = (kv0 + c <= pos) ? s[c] * sl2 : -INFINITY;
-                        mt = fmaxf(mt, s[c]);
+                        if (kv0 + c > pos) s[c] = -INFINITY;
+                        mx[c & 7] = fmaxf(mx[c & 7], s[c]);
                     }
                 }
-                // Lazy rescaling: keep the running max unless a row's max grew
-                // by more than 8 (log2 units), so P stays below 2^8 in bf16 and
-                // O is rescaled in TMEM only rarely.
+                float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                mt *= sl2;
                 const float m_new = fmaxf(m, mt);
                 const float m_use = (j == 0 || m_new - m > 8.0f) ? m_new : m;
                 if (j > 0) {
@@ -323,14 +328,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     }
                 }
                 m = m_use;
-                float ls = 0.f;
+                // eight independent partial sums
+                float ls[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ls[e] = 0.f;
+                const float neg_m = -m;
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     float p[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        p[e] = ex2(s[q * 8 + e] - m);
-                        ls += p[e];
+                        p[e] = ex2(fmaf(s[q * 8 + e], sl2, neg_m));
+                        ls[e] += p[e];
                     }
                     uint4 v;
                     v.x = pack_bf16(p[0], p[1]);
@@ -340,7 +349,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const int atom = q >> 3, chunk = (q & 7) ^ (trow & 7);
                     *reinterpret_cast<uint4 *>(prow + atom * 16384 + chunk * 16) = v;
                 }
-                l += ls;
+                l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(&p_full[w]);

@@ -112,7 +112,7 @@ EncodeFn get_encode() {
 tsp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA; }
 
 // Device tables: map, inverse map, per-query-tile max position and the work
-// orders of the attention kernels (longest item first).
+// orders of the attention kernels (head-major, longest item first per head).
 tsp_status ensure_device(tsp_plan_s *p) {
     std::lock_guard<std::mutex> g(p->mu);
     int dev = 0;
@@ -142,7 +142,13 @@ tsp_status ensure_device(tsp_plan_s *p) {
         int32_t m = std::max(qmax[2 * qb], qmax[2 * qb + 1]);
         for (int hd = 0; hd < H; ++hd) fitems.push_back({static_cast<int>(qb * H + hd), m / 128 + 1});
     }
-    std::stable_sort(fitems.begin(), fitems.end(), [](auto &x, auto &y) { return x.second > y.second; });
+    // Head-major, longest first within a head: the CTAs running at the same
+    // time then share one head's K/V (64 MiB at S = 128K) in L2 instead of
+    // streaming every head's K/V from HBM.
+    std::stable_sort(fitems.begin(), fitems.end(), [H](auto &x, auto &y) {
+        const int hx = x.first % H, hy = y.first % H;
+        return hx != hy ? hx < hy : x.second > y.second;
+    });
     std::vector<int32_t> forder;
     for (auto &it : fitems) {
         forder.push_back(it.first);
@@ -157,7 +163,10 @@ tsp_status ensure_device(tsp_plan_s *p) {
     }
     for (int64_t qt = 0; qt < S / 128; ++qt)
         for (int hd = 0; hd < H; ++hd) qitems.push_back({static_cast<int>(qt * H + hd), qmax[qt] / 128 + 1});
-    auto by_cost = [](auto &x, auto &y) { return x.second > y.second; };
+    auto by_cost = [H](auto &x, auto &y) {
+        const int hx = x.first % H, hy = y.first % H;
+        return hx != hy ? hx < hy : x.second > y.second;
+    };
     std::stable_sort(kitems.begin(), kitems.end(), by_cost);
     std::stable_sort(qitems.begin(), qitems.end(), by_cost);
     std::vector<int32_t> korder, qorder;
@@ -666,3 +675,4 @@ TSP_API tsp_status tsp_test_wait_timeout(tsp_plan_t p, long long limit_cycles, i
     wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(e, result_dev);
     return cuda_status(cudaGetLastError());
 }
+

@@ -286,3 +286,4 @@ def tsp_test_buffer_offset(plan: Plan, name: str) -> int:
 def tsp_test_wait_timeout(plan: Plan, limit_cycles: int, result, stream=None) -> None:
     _check(_lib.tsp_test_wait_timeout(plan.handle, limit_cycles, _ptr(result, "result"), _stream(stream)),
            "tsp_test_wait_timeout")
+
