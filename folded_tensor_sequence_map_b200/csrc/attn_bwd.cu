@@ -11,14 +11,14 @@
 //
 // Three kernels, no atomics (deterministic):
 //   attn_delta   Delta[h][row] = sum_d dO * O (bf16 inputs, fp32 sum).
-//   attn_dkdv    one item = (head, 128-key tile); loops over the 128-row query
-//                tiles that see any of its keys.  S^T = K Q^T and dP^T = V dO^T
-//                in TMEM; P^T, dS^T written to smem as bf16; dV += P^T dO and
-//                dK += dS^T Q accumulate in TMEM for the whole item.
-//   attn_dq      one item = (head, 128-row query tile); loops over key tiles.
+//   attn_dkdv2   one item = (head, 128-key tile); steps of 64 query rows over
+//                the query tiles that see any of its keys.  S^T = K Q^T and
+//                dP^T = V dO^T in TMEM; P^T, dS^T written to smem as bf16;
+//                dV += P^T dO and dK += dS^T Q accumulate in TMEM.
+//   attn_dq2     one item = (head, 128-row query tile); steps of 64 keys.
 //                S = Q K^T, dP = dO V^T in TMEM; dS to smem; dQ += dS K.
-// Warp roles as in the forward: warp 0 TMA, warp 1 TMEM + MMA, warps 2-5
-// element-wise (thread = TMEM lane = row of the 128-row tile).
+// Warp roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2-9 element-wise (two
+// groups of four; thread = TMEM lane = row of the 128-row tile).
 #include "common.cuh"
 #include "internal.h"
 
@@ -121,196 +121,6 @@ struct BwdParams {
     int num_items;
 };
 
-template <int DH>
-__global__ void __launch_bounds__(kBwdThreads, 1)
-    attn_dkdv_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
-                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
-                     const BwdParams bp, const DevErr err) {
-    using C = BCfg<DH>;
-    const AttnBwdDesc &a = bp.d;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t *sK = smem;
-    uint8_t *sV = sK + C::TILE_BYTES;
-    uint8_t *sQ = sV + C::TILE_BYTES;
-    uint8_t *sdO = sQ + C::TILE_BYTES;
-    uint8_t *sPt = sdO + C::TILE_BYTES;
-    uint8_t *sdSt = sPt + C::SQ_BYTES;
-    float *sLse = reinterpret_cast<float *>(sdSt + C::SQ_BYTES);
-    float *sDelta = sLse + 128;
-    int *sPos = reinterpret_cast<int *>(sDelta + 128);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sPos + 128);
-    uint64_t *kv_full = bars + 0, *kv_empty = bars + 1, *q_full = bars + 2, *step_done = bars + 3,
-             *s_full = bars + 4, *p_full = bars + 5, *drain = bars + 6;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int h = a.H * DH;
-    const int nqt = a.S / 128;
-    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
-    const float scale = rsqrtf(static_cast<float>(DH));
-
-    if (threadIdx.x == 0) {
-        mbar_init(kv_full, 1);
-        mbar_init(kv_empty, 1);
-        mbar_init(q_full, 1);
-        mbar_init(step_done, 1);
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            int item_iter = 0, step = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
-                const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
-                if (!mbar_wait(kv_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
-                mbar_arrive_tx(kv_full, 2 * C::TILE_BYTES);
-                for (int t = 0; t < C::NATOM; ++t) {
-                    tma_load_2d(sK + t * C::ATOM_BYTES, &mK, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
-                    tma_load_2d(sV + t * C::ATOM_BYTES, &mV, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
-                }
-                for (int qt = 0; qt < nqt; ++qt) {
-                    if (bp.qtile_maxpos[qt] < kt * 128) continue;
-                    if (!mbar_wait(step_done, (step & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-                    mbar_arrive_tx(q_full, 2 * C::TILE_BYTES + 3 * 512);
-                    for (int t = 0; t < C::NATOM; ++t) {
-                        tma_load_2d(sQ + t * C::ATOM_BYTES, &mQ, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
-                        tma_load_2d(sdO + t * C::ATOM_BYTES, &mdO, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
-                    }
-                    bulk_load(sLse, a.lse + static_cast<int64_t>(head) * a.S + qt * 128, 512, q_full);
-                    bulk_load(sDelta, a.delta + static_cast<int64_t>(head) * a.S + qt * 128, 512, q_full);
-                    bulk_load(sPos, bp.zig + qt * 128, 512, q_full);
-                    ++step;
-                }
-            }
-            if (item_iter > 0) spin_drain(kv_full, (item_iter - 1) & 1, err.wait_limit);
-            if (step > 0) spin_drain(q_full, (step - 1) & 1, err.wait_limit);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
-            const uint32_t k_b = smem_u32(sK), v_b = smem_u32(sV), q_b = smem_u32(sQ), do_b = smem_u32(sdO);
-            const uint32_t pt_b = smem_u32(sPt), dst_b = smem_u32(sdSt);
-            int item_iter = 0, step = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
-                const int kt = a.kv_order[it] / a.H;
-                if (!mbar_wait(kv_full, item_iter & 1, abort_flag, err)) break;
-                bool first = true;
-                for (int qt = 0; qt < nqt; ++qt) {
-                    if (bp.qtile_maxpos[qt] < kt * 128) continue;
-                    if (!mbar_wait(q_full, step & 1, abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 0, kdesc<DH>(k_b, kk), kdesc<DH>(q_b, kk), idS, kk > 0);
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 128, kdesc<DH>(v_b, kk), kdesc<DH>(do_b, kk), idS, kk > 0);
-                    umma_commit(s_full);
-                    if (!mbar_wait(p_full, step & 1, abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(tmem + 256, sq_desc(pt_b, kk), mndesc<DH>(do_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(tmem + 384, sq_desc(dst_b, kk), mndesc<DH>(q_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
-                    umma_commit(step_done);
-                    first = false;
-                    ++step;
-                }
-                umma_commit(kv_empty);
-            }
-            if (!ok || *abort_flag) {
-                umma_commit(drain);
-                spin_drain(drain, 0, err.wait_limit);
-            }
-        }
-    } else {
-        const int quarter = warp & 3;
-        const int trow = quarter * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        int step = 0;
-        for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
-            const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
-            const int key = kt * 128 + trow;
-            bool ok = true, any = false;
-            for (int qt = 0; qt < nqt; ++qt) {
-                if (bp.qtile_maxpos[qt] < kt * 128) continue;
-                any = true;
-                if (!warp_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
-                tc_fence_after();
-                // previous step's MMAs must be done reading P^T / dS^T
-                if (step > 0 && !warp_wait(step_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float s[32], dp[32];
-                    tmem_ld32(tmem + lane_off + c * 32, s);
-                    tmem_ld32(tmem + lane_off + 128 + c * 32, dp);
-                    tmem_ld_wait();
-                    float pv[32], dsv[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int q = c * 32 + e;
-                        const float p = (key <= sPos[q]) ? ex2b(s[e] * sl2 - sLse[q]) : 0.f;
-                        pv[e] = p;
-                        dsv[e] = p * (dp[e] - sDelta[q]);
-                    }
-                    store_row32(sPt, trow, c * 32, pv);
-                    store_row32(sdSt, trow, c * 32, dsv);
-                }
-                fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(p_full);
-                ++step;
-            }
-            if (!ok) break;
-            if (!any) continue;
-            if (!warp_wait(step_done, (step - 1) & 1, abort_flag, err)) break;
-            tc_fence_after();
-            const int lrow = a.inv_map[key];
-            __nv_bfloat16 *dvrow = static_cast<__nv_bfloat16 *>(a.dv) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
-            __nv_bfloat16 *dkrow = static_cast<__nv_bfloat16 *>(a.dk) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
-#pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
-                float v[32], k[32];
-                tmem_ld32(tmem + lane_off + 256 + c * 32, v);
-                tmem_ld32(tmem + lane_off + 384 + c * 32, k);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) k[e] *= scale;
-                uint4 *dv4 = reinterpret_cast<uint4 *>(dvrow + c * 32);
-                uint4 *dk4 = reinterpret_cast<uint4 *>(dkrow + c * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    dv4[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                        pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
-                    dk4[q] = make_uint4(pack_bf16(k[8 * q], k[8 * q + 1]), pack_bf16(k[8 * q + 2], k[8 * q + 3]),
-                                        pack_bf16(k[8 * q + 4], k[8 * q + 5]), pack_bf16(k[8 * q + 6], k[8 * q + 7]));
-                }
-            }
-            tc_fence_before();
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
 // ---------------------------------------------------------------------------
 // Pipelined dK/dV kernel: steps of 64 query rows.
 //   TMEM: S^T buffers [2] at columns 0 / 64, dP^T buffers [2] at 128 / 192,
@@ -318,6 +128,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 //   The MMA warp issues S^T/dP^T of step g+1 before dV/dK of step g, so the
 //   tensor core works on the next step while the element-wise warps (two
 //   groups of four, 32 query columns each) turn step g into P^T and dS^T.
+//   P^T and dS^T go back into TMEM as packed bf16 (two queries per column) in
+//   the columns their S^T / dP^T values came from, where the dV / dK MMAs
+//   read them as the A operand.
 template <int DH>
 struct KvCfg {
     using C = BCfg<DH>;
@@ -325,15 +138,12 @@ struct KvCfg {
     static constexpr int QST = 3;
     static constexpr int QTILE = BQ * DH * 2;
     static constexpr int QATOM = BQ * C::SWB;
-    static constexpr int PT_BYTES = 128 * BQ * 2;
     static constexpr int VEC_BYTES = 3 * BQ * 4;  // lse, delta, pos of one step
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + C::TILE_BYTES;
     static constexpr int OFF_Q = OFF_V + C::TILE_BYTES;
     static constexpr int OFF_DO = OFF_Q + QST * QTILE;
-    static constexpr int OFF_PT = OFF_DO + QST * QTILE;
-    static constexpr int OFF_DST = OFF_PT + PT_BYTES;
-    static constexpr int OFF_VEC = OFF_DST + PT_BYTES;
+    static constexpr int OFF_VEC = OFF_DO + QST * QTILE;
     static constexpr int OFF_BAR = OFF_VEC + QST * VEC_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
 };
@@ -352,10 +162,6 @@ __device__ __forceinline__ uint64_t mndesc64(uint32_t base, int kk) {
     using C = BCfg<DH>;
     using K = KvCfg<DH>;
     return sdesc(base + kk * 16 * C::SWB, K::QATOM, 8 * C::SWB, C::LAYOUT);
-}
-// K-major descriptor of a [128 rows][64 cols] bf16 operand (P^T, dS^T).
-__device__ __forceinline__ uint64_t pt_desc(uint32_t base, int kk) {
-    return sdesc(base + kk * 32, 16, 1024, kSwizzle128);
 }
 __device__ __forceinline__ int next_visible(const int *qmax64, int nq64, int from, int kv0) {
     while (from < nq64 && qmax64[from] < kv0) ++from;
@@ -461,7 +267,6 @@ __global__ void __launch_bounds__(320, 1)
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
             const uint32_t k_b = smem_u32(smem + K::OFF_K), v_b = smem_u32(smem + K::OFF_V);
-            const uint32_t pt_b = smem_u32(smem + K::OFF_PT), dst_b = smem_u32(smem + K::OFF_DST);
             int item_iter = 0, g = 0;
             bool ok = true;
             auto issue_sdp = [&](int gi) -> bool {
@@ -493,10 +298,14 @@ __global__ void __launch_bounds__(320, 1)
                     const int s = g % K::QST;
                     const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
                     const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
+                    const int b = g & 1;
+                    // A operands from TMEM: queries 16 kk.. at column 32 (kk / 2) + 8 (kk % 2)
                     for (int kk = 0; kk < K::BQ / 16; ++kk)
-                        umma_bf16(tmem + 256, pt_desc(pt_b, kk), mndesc64<DH>(do_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(tmem + 256, tmem + 64 * b + (kk >> 1) * 32 + (kk & 1) * 8, mndesc64<DH>(do_b, kk),
+                                     idG, (!first || kk > 0) ? 1u : 0u);
                     for (int kk = 0; kk < K::BQ / 16; ++kk)
-                        umma_bf16(tmem + 384, pt_desc(dst_b, kk), mndesc64<DH>(q_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(tmem + 384, tmem + 128 + 64 * b + (kk >> 1) * 32 + (kk & 1) * 8,
+                                     mndesc64<DH>(q_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
                     umma_commit(&q_empty[s]);
                     umma_commit(pd_free);
                     first = false;
@@ -515,8 +324,6 @@ __global__ void __launch_bounds__(320, 1)
         const int quarter = warp & 3;
         const int trow = quarter * 32 + lane;   // key row of the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        uint8_t *sPt = smem + K::OFF_PT;
-        uint8_t *sdSt = smem + K::OFF_DST;
         int g = 0;
         for (int it = blockIdx.x; it < kp.num_items; it += gridDim.x) {
             const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
@@ -535,29 +342,36 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_ld_wait();
                 const float *vec = reinterpret_cast<const float *>(smem + K::OFF_VEC + s * K::VEC_BYTES);
                 const int *pos = reinterpret_cast<const int *>(vec + 128);
-                float pv[32], dsv[32];
+                // the 64 query rows of a step lie in one zigzag chunk (chunks are
+                // multiples of 64 rows), so their positions are consecutive: this
+                // key is visible to column e of the group iff e >= key - pos0
+                const int first_vis = key - pos[32 * wg];
+                const float4 *lse4 = reinterpret_cast<const float4 *>(vec + 32 * wg);
+                const float4 *dl4 = reinterpret_cast<const float4 *>(vec + 64 + 32 * wg);
+                uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = 32 * wg + e;
-                    const float pe = ex2b(fmaf(sv[e], sl2, -vec[c]));
-                    const float p = (key <= pos[c]) ? pe : 0.f;
-                    pv[e] = p;
-                    dsv[e] = p * (dp[e] - vec[64 + c]);
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 l = lse4[e4], d = dl4[e4];
+                    const int e = 4 * e4;
+                    float p0 = ex2b(fmaf(sv[e], sl2, -l.x)), p1 = ex2b(fmaf(sv[e + 1], sl2, -l.y));
+                    float p2 = ex2b(fmaf(sv[e + 2], sl2, -l.z)), p3 = ex2b(fmaf(sv[e + 3], sl2, -l.w));
+                    if (first_vis > 0) {
+                        p0 = e >= first_vis ? p0 : 0.f;
+                        p1 = e + 1 >= first_vis ? p1 : 0.f;
+                        p2 = e + 2 >= first_vis ? p2 : 0.f;
+                        p3 = e + 3 >= first_vis ? p3 : 0.f;
+                    }
+                    pk[2 * e4] = pack_bf16(p0, p1);
+                    pk[2 * e4 + 1] = pack_bf16(p2, p3);
+                    dk[2 * e4] = pack_bf16(p0 * (dp[e] - d.x), p1 * (dp[e + 1] - d.y));
+                    dk[2 * e4 + 1] = pack_bf16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
                 }
-                // the previous step's dV/dK MMAs must be done reading P^T / dS^T
-                if (g > 0 && !warp_wait(pd_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int col = 32 * wg + qq * 8;
-                    const int chunk = (col >> 3) ^ (trow & 7);
-                    *reinterpret_cast<uint4 *>(sPt + trow * 128 + chunk * 16) =
-                        make_uint4(pack_bf16(pv[8 * qq], pv[8 * qq + 1]), pack_bf16(pv[8 * qq + 2], pv[8 * qq + 3]),
-                                   pack_bf16(pv[8 * qq + 4], pv[8 * qq + 5]), pack_bf16(pv[8 * qq + 6], pv[8 * qq + 7]));
-                    *reinterpret_cast<uint4 *>(sdSt + trow * 128 + chunk * 16) =
-                        make_uint4(pack_bf16(dsv[8 * qq], dsv[8 * qq + 1]), pack_bf16(dsv[8 * qq + 2], dsv[8 * qq + 3]),
-                                   pack_bf16(dsv[8 * qq + 4], dsv[8 * qq + 5]), pack_bf16(dsv[8 * qq + 6], dsv[8 * qq + 7]));
-                }
-                fence_async_smem();
+                // each group packs its 32 queries into the first 16 of the 32
+                // columns it has just read, so no group writes what the other
+                // still has to read
+                tmem_st16(tmem + lane_off + 64 * b + 32 * wg, pk);
+                tmem_st16(tmem + lane_off + 128 + 64 * b + 32 * wg, dk);
+                tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(p_full);
             }
@@ -595,7 +409,8 @@ __global__ void __launch_bounds__(320, 1)
 //   TMEM: S buffers [2] at columns 0 / 64, dP buffers [2] at 128 / 192, dQ at
 //   256 (128 query lanes).  The MMA warp issues S/dP of step j+1 before dQ of
 //   step j, so the tensor core works while the element-wise warps (two groups
-//   of four, 32 key columns each) turn step j into dS.
+//   of four, 32 key columns each) turn step j into dS, which goes back into
+//   TMEM as packed bf16 in the S columns it came from (the dQ MMA's A).
 template <int DH>
 struct Dq2Cfg {
     using C = BCfg<DH>;
@@ -603,13 +418,11 @@ struct Dq2Cfg {
     static constexpr int KST = 3;
     static constexpr int KTILE = BK * DH * 2;   // one K or V sub-tile of 64 keys
     static constexpr int KATOM = BK * C::SWB;
-    static constexpr int DS_BYTES = 128 * BK * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_DO = OFF_Q + C::TILE_BYTES;
     static constexpr int OFF_K = OFF_DO + C::TILE_BYTES;
     static constexpr int OFF_V = OFF_K + KST * KTILE;
-    static constexpr int OFF_DS = OFF_V + KST * KTILE;
-    static constexpr int OFF_BAR = OFF_DS + DS_BYTES;
+    static constexpr int OFF_BAR = OFF_V + KST * KTILE;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -702,7 +515,6 @@ __global__ void __launch_bounds__(320, 1)
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
             const uint32_t q_b = smem_u32(smem + Q::OFF_Q), do_b = smem_u32(smem + Q::OFF_DO);
-            const uint32_t ds_b = smem_u32(smem + Q::OFF_DS);
             int item_iter = 0, g = 0;
             bool ok = true;
             auto issue_sdp = [&](int gi) -> bool {
@@ -728,10 +540,12 @@ __global__ void __launch_bounds__(320, 1)
                     if (j + 1 < n && !issue_sdp(g + 1)) { ok = false; break; }
                     if (!mbar_wait(p_full, g & 1, abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
-                    const int s = g % Q::KST;
+                    const int s = g % Q::KST, b = g & 1;
                     const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
+                    // A = dS from TMEM: keys 16 kk.. at column 32 (kk / 2) + 8 (kk % 2)
                     for (int kk = 0; kk < Q::BK / 16; ++kk)
-                        umma_bf16(tmem + 256, pt_desc(ds_b, kk), mndesc64<DH>(k_b, kk), idG, (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(tmem + 256, tmem + 64 * b + (kk >> 1) * 32 + (kk & 1) * 8, mndesc64<DH>(k_b, kk),
+                                     idG, (j > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&k_empty[s]);
                     umma_commit(ds_free);
                 }
@@ -747,7 +561,6 @@ __global__ void __launch_bounds__(320, 1)
         const int quarter = warp & 3;
         const int trow = quarter * 32 + lane;   // query row of the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        uint8_t *sDS = smem + Q::OFF_DS;
         int g = 0;
         for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
             const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
@@ -761,27 +574,21 @@ __global__ void __launch_bounds__(320, 1)
                 const int b = g & 1;
                 if (!warp_wait(&s_full[b], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
-                float sv[32], dp[32], dsv[32];
+                float sv[32], dp[32];
                 tmem_ld32(tmem + lane_off + 64 * b + 32 * wg, sv);
                 tmem_ld32(tmem + lane_off + 128 + 64 * b + 32 * wg, dp);
                 tmem_ld_wait();
                 const int k0 = j * 64 + 32 * wg;
+                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float pe = ex2b(fmaf(sv[e], sl2, -lse));
-                    const float p = (k0 + e <= pos) ? pe : 0.f;
-                    dsv[e] = p * (dp[e] - dl);
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = (k0 + e <= pos) ? ex2b(fmaf(sv[e], sl2, -lse)) : 0.f;
+                    const float p1 = (k0 + e + 1 <= pos) ? ex2b(fmaf(sv[e + 1], sl2, -lse)) : 0.f;
+                    pk[e / 2] = pack_bf16(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
                 }
-                if (g > 0 && !warp_wait(ds_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int col = 32 * wg + qq * 8;
-                    const int chunk = (col >> 3) ^ (trow & 7);
-                    *reinterpret_cast<uint4 *>(sDS + trow * 128 + chunk * 16) =
-                        make_uint4(pack_bf16(dsv[8 * qq], dsv[8 * qq + 1]), pack_bf16(dsv[8 * qq + 2], dsv[8 * qq + 3]),
-                                   pack_bf16(dsv[8 * qq + 4], dsv[8 * qq + 5]), pack_bf16(dsv[8 * qq + 6], dsv[8 * qq + 7]));
-                }
-                fence_async_smem();
+                // packed into the first 16 of the 32 columns this group just read
+                tmem_st16(tmem + lane_off + 64 * b + 32 * wg, pk);
+                tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(p_full);
             }
@@ -803,201 +610,6 @@ __global__ void __launch_bounds__(320, 1)
                                             pack_bf16(v[8 * qq + 4] * scale, v[8 * qq + 5] * scale),
                                             pack_bf16(v[8 * qq + 6] * scale, v[8 * qq + 7] * scale));
                 }
-            }
-            tc_fence_before();
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
-// ---------------------------------------------------------------------------
-template <int DH>
-struct DqCfg {
-    using C = BCfg<DH>;
-    static constexpr int KVST = 2;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_DO = OFF_Q + C::TILE_BYTES;
-    static constexpr int OFF_K = OFF_DO + C::TILE_BYTES;
-    static constexpr int OFF_V = OFF_K + KVST * C::TILE_BYTES;
-    static constexpr int OFF_DS = OFF_V + KVST * C::TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_DS + C::SQ_BYTES;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;
-};
-
-template <int DH>
-__global__ void __launch_bounds__(kBwdThreads, 1)
-    attn_dq_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
-                   const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
-                   const BwdParams bp, const DevErr err) {
-    using C = BCfg<DH>;
-    using Q = DqCfg<DH>;
-    const AttnBwdDesc &a = bp.d;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Q::OFF_BAR);
-    uint64_t *q_full = bars + 0, *q_empty = bars + 1, *kv_full = bars + 2, *kv_empty = bars + 4,
-             *s_full = bars + 6, *p_full = bars + 7, *ds_done = bars + 8, *drain = bars + 9;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int h = a.H * DH;
-    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
-    const float scale = rsqrtf(static_cast<float>(DH));
-
-    if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
-        }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
-        mbar_init(ds_done, 1);
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    auto item_nkv = [&](int qt) { return bp.qtile_maxpos[qt] / 128 + 1; };
-
-    if (warp == 0) {
-        if (lane == 0) {
-            int item_iter = 0, kvc = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
-                const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
-                if (!mbar_wait(q_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
-                mbar_arrive_tx(q_full, 2 * C::TILE_BYTES);
-                for (int t = 0; t < C::NATOM; ++t) {
-                    tma_load_2d(smem + Q::OFF_Q + t * C::ATOM_BYTES, &mQ, q_full, head * DH + t * C::ATOM_COLS, qt * 128);
-                    tma_load_2d(smem + Q::OFF_DO + t * C::ATOM_BYTES, &mdO, q_full, head * DH + t * C::ATOM_COLS,
-                                qt * 128);
-                }
-                const int nkv = item_nkv(qt);
-                for (int j = 0; j < nkv; ++j) {
-                    const int s = kvc % Q::KVST;
-                    if (!mbar_wait(&kv_empty[s], ((kvc / Q::KVST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-                    mbar_arrive_tx(&kv_full[s], 2 * C::TILE_BYTES);
-                    for (int t = 0; t < C::NATOM; ++t) {
-                        tma_load_2d(smem + Q::OFF_K + s * C::TILE_BYTES + t * C::ATOM_BYTES, &mK, &kv_full[s],
-                                    head * DH + t * C::ATOM_COLS, j * 128);
-                        tma_load_2d(smem + Q::OFF_V + s * C::TILE_BYTES + t * C::ATOM_BYTES, &mV, &kv_full[s],
-                                    head * DH + t * C::ATOM_COLS, j * 128);
-                    }
-                    ++kvc;
-                }
-            }
-            for (int s = 0; s < Q::KVST; ++s)
-                if (kvc > s) {
-                    const int last = kvc - 1 - ((kvc - 1 - s) % Q::KVST);
-                    spin_drain(&kv_full[s], (last / Q::KVST) & 1, err.wait_limit);
-                }
-            if (item_iter > 0) spin_drain(q_full, (item_iter - 1) & 1, err.wait_limit);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
-            const uint32_t q_b = smem_u32(smem + Q::OFF_Q), do_b = smem_u32(smem + Q::OFF_DO);
-            const uint32_t ds_b = smem_u32(smem + Q::OFF_DS);
-            int item_iter = 0, kvc = 0, step = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
-                const int qt = a.q_order[it] / a.H;
-                if (!mbar_wait(q_full, item_iter & 1, abort_flag, err)) break;
-                const int nkv = item_nkv(qt);
-                for (int j = 0; j < nkv; ++j, ++step) {
-                    const int s = kvc % Q::KVST;
-                    if (!mbar_wait(&kv_full[s], (kvc / Q::KVST) & 1, abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * C::TILE_BYTES);
-                    const uint32_t v_b = smem_u32(smem + Q::OFF_V + s * C::TILE_BYTES);
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 0, kdesc<DH>(q_b, kk), kdesc<DH>(k_b, kk), idS, kk > 0);
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 128, kdesc<DH>(do_b, kk), kdesc<DH>(v_b, kk), idS, kk > 0);
-                    umma_commit(s_full);
-                    if (!mbar_wait(p_full, step & 1, abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(tmem + 256, sq_desc(ds_b, kk), mndesc<DH>(k_b, kk), idG, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(ds_done);
-                    umma_commit(&kv_empty[s]);
-                    ++kvc;
-                }
-                umma_commit(q_empty);
-            }
-            if (!ok || *abort_flag) {
-                umma_commit(drain);
-                spin_drain(drain, 0, err.wait_limit);
-            }
-        }
-    } else {
-        const int quarter = warp & 3;
-        const int trow = quarter * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        uint8_t *sDS = smem + Q::OFF_DS;
-        int step = 0;
-        for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
-            const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
-            const int lrow = qt * 128 + trow;
-            const int pos = bp.zig[lrow];
-            const float lse = a.lse[static_cast<int64_t>(head) * a.S + lrow];
-            const float dl = a.delta[static_cast<int64_t>(head) * a.S + lrow];
-            const int nkv = item_nkv(qt);
-            bool ok = true;
-            for (int j = 0; j < nkv; ++j, ++step) {
-                if (!warp_wait(s_full, step & 1, abort_flag, err)) { ok = false; break; }
-                tc_fence_after();
-                if (step > 0 && !warp_wait(ds_done, (step - 1) & 1, abort_flag, err)) { ok = false; break; }
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float s[32], dp[32], dsv[32];
-                    tmem_ld32(tmem + lane_off + c * 32, s);
-                    tmem_ld32(tmem + lane_off + 128 + c * 32, dp);
-                    tmem_ld_wait();
-                    const int k0 = j * 128 + c * 32;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float p = (k0 + e <= pos) ? ex2b(s[e] * sl2 - lse) : 0.f;
-                        dsv[e] = p * (dp[e] - dl);
-                    }
-                    store_row32(sDS, trow, c * 32, dsv);
-                }
-                fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(p_full);
-            }
-            if (!ok) break;
-            if (!warp_wait(ds_done, (step - 1) & 1, abort_flag, err)) break;
-            tc_fence_after();
-            __nv_bfloat16 *dqrow = static_cast<__nv_bfloat16 *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
-#pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
-                float v[32];
-                tmem_ld32(tmem + lane_off + 256 + c * 32, v);
-                tmem_ld_wait();
-                uint4 *d4 = reinterpret_cast<uint4 *>(dqrow + c * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    d4[q] = make_uint4(pack_bf16(v[8 * q] * scale, v[8 * q + 1] * scale),
-                                       pack_bf16(v[8 * q + 2] * scale, v[8 * q + 3] * scale),
-                                       pack_bf16(v[8 * q + 4] * scale, v[8 * q + 5] * scale),
-                                       pack_bf16(v[8 * q + 6] * scale, v[8 * q + 7] * scale));
             }
             tc_fence_before();
         }

@@ -8,17 +8,19 @@
 // Work item = (head, block of 256 local query rows) = two 128-row query tiles.
 // CTA layout (10 warps, persistent, one CTA per SM):
 //   warp 0     TMA producer: the two Q tiles of the item, then K_j / V_j tiles
-//              of 128 keys (K ring of 1 or 2 slots, V ring of 2).
+//              of 128 keys (K ring of 2, V ring of 2).
 //   warp 1     TMEM owner and MMA issuer: S_w = Q_w K_j^T (128x128, fp32 in
 //              TMEM) and O_w += P_w V_j (128 x dh, fp32 in TMEM) for w = 0, 1,
 //              ordered so that S of the next tile overlaps the softmax of the
 //              other tile (ping-pong between the two softmax groups).
 //   warps 2-5  softmax group 0 (query tile 0), warps 6-9 group 1: thread =
-//              query row; online softmax in the log2 domain, P written to
-//              shared memory as bf16 in the MMA's 128B-swizzled K-major
-//              layout; O rescaled in TMEM when the running max grows by more than 2^8; final
+//              query row; online softmax in the log2 domain; P written back
+//              into TMEM as packed bf16 over the first half of S_w's
+//              columns, where the P V MMA reads it as its A operand; O
+//              rescaled in TMEM when the running max grows by more than 2^8; final
 //              O / l written as bf16 and LSE (log2 domain) as fp32.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+dh), O1 [384,384+dh).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+dh), O1 [384,384+dh);
+// P_w overwrites the first 64 columns of S_w once S_w is in registers.
 #include "common.cuh"
 #include "internal.h"
 
@@ -48,17 +50,13 @@ struct FwdCfg {
     static constexpr int TILE_BYTES = 128 * DH * 2;           // one 128-row tile of Q, K or V
     static constexpr int ATOM_BYTES = 128 * SWB;
     static constexpr uint32_t LAYOUT = SWB == 128 ? kSwizzle128 : (SWB == 64 ? kSwizzle64 : kSwizzle32);
-    // K_j is read by both S MMAs long before P V needs V_j, so a single K slot
-    // is enough; V gets two so its next tile loads during the softmax.
-    static constexpr int KST = DH == 128 ? 1 : 2;
+    static constexpr int KST = 2;
     static constexpr int VST = 2;
-    static constexpr int P_BYTES = 128 * 128 * 2;
-    // smem map (1024-aligned pieces)
+    // smem map (1024-aligned pieces); P lives in TMEM
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
-    static constexpr int OFF_P = OFF_V + VST * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -76,12 +74,6 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
     using C = FwdCfg<DH>;
     return sdesc(base + kk * 16 * C::SWB, C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
 }
-// P[128 rows][128 keys] bf16, K-major with 128B swizzle (two 64-key atoms).
-__device__ __forceinline__ uint64_t p_desc(uint32_t base, int kk) {
-    const int col = kk * 16;
-    return sdesc(base + (col / 64) * 16384 + (col % 64) * 2, 16, 1024, kSwizzle128);
-}
-
 template <int DH>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
@@ -194,7 +186,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
             const uint32_t qbase = smem_u32(smem + C::OFF_Q);
-            const uint32_t pbase = smem_u32(smem + C::OFF_P);
             int kcount = 0, vcount = 0, tcount = 0, item_iter = 0;
             bool ok = true;
             for (int it = blockIdx.x; it < a.num_items && ok; it += gridDim.x, ++item_iter) {
@@ -225,9 +216,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     for (int w = 0; w < 2; ++w) {
                         if (!mbar_wait(&p_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
                         tc_fence_after();
+                        // P_w sits in TMEM columns [128 w, 128 w + 64): 16 keys per 8 columns
                         for (int kk = 0; kk < 8; ++kk)
-                            umma_bf16(tmem + 256 + w * 128, p_desc(pbase + w * C::P_BYTES, kk), mnmajor_desc<DH>(vb, kk),
-                                      idO, (j > 0 || kk > 0) ? 1u : 0u);
+                            umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, mnmajor_desc<DH>(vb, kk),
+                                         idO, (j > 0 || kk > 0) ? 1u : 0u);
                         umma_commit(&o_done[w]);
                         if (j + 1 < nkv) {
                             if (w == 0) {
@@ -264,7 +256,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + w * 128;
         const uint32_t o_addr = tmem + lane_off + 256 + w * 128;
-        uint8_t *prow = smem + C::OFF_P + w * C::P_BYTES + trow * 128;
         int tcount = 0;
         for (int it = blockIdx.x; it < a.num_items; it += gridDim.x) {
             const int qb = a.order[2 * it] / a.H, head = a.order[2 * it] % a.H, nkv = a.order[2 * it + 1];
@@ -286,8 +277,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tmem_ld_wait();
                 const int kv0 = j * 128;
                 // Row max on the raw scores (the scale is positive), masking
-                // only on tiles that reach past this row's position.
-                const bool full = kv0 + 127 <= pos;
+                // only on tiles that reach past this row's position.  `full` is
+                // warp-uniform: it selects code paths that end in warp-collective
+                // TMEM stores, which must never run on a partial warp.
+                const bool full = __all_sync(0xffffffffu, kv0 + 127 <= pos);
                 // eight independent partial maxima: no 128-long dependency chain
                 float mx[8];
 #pragma unroll
@@ -334,23 +327,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int e = 0; e < 8; ++e) ls[e] = 0.f;
                 const float neg_m = -m;
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    float p[8];
+                for (int half = 0; half < 2; ++half) {
+                    // 64 keys -> 32 TMEM columns of packed bf16 pairs (even key in the low half)
+                    float pk[32];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        p[e] = ex2(fmaf(s[q * 8 + e], sl2, neg_m));
-                        ls[e] += p[e];
+                    for (int c = 0; c < 32; ++c) {
+                        const int k0 = half * 64 + 2 * c;
+                        const float p0 = ex2(fmaf(s[k0], sl2, neg_m));
+                        const float p1 = ex2(fmaf(s[k0 + 1], sl2, neg_m));
+                        ls[(2 * c) & 7] += p0;
+                        ls[(2 * c + 1) & 7] += p1;
+                        pk[c] = __uint_as_float(pack_bf16(p0, p1));
                     }
-                    uint4 v;
-                    v.x = pack_bf16(p[0], p[1]);
-                    v.y = pack_bf16(p[2], p[3]);
-                    v.z = pack_bf16(p[4], p[5]);
-                    v.w = pack_bf16(p[6], p[7]);
-                    const int atom = q >> 3, chunk = (q & 7) ^ (trow & 7);
-                    *reinterpret_cast<uint4 *>(prow + atom * 16384 + chunk * 16) = v;
+                    tmem_st32(s_addr + half * 32, pk);
                 }
+                tmem_st_wait();
                 l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-                fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(&p_full[w]);
             }
