@@ -41,6 +41,13 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "7b_s128k"
 CPU_SAMPLE_S = 2048  # oracle sample: the same 7B layer at this many tokens
 
+# DRAM bytes (read + write) of one launch from an ncu capture of the current
+# kernel build, and the S of that capture (profiles/attention_kernels_7b_s16384_d8.md).
+# The traffic is the compulsory one and grows in proportion to S, so it is
+# scaled by S to the benchmarked launch.  Must be re-measured (or removed)
+# whenever the kernel changes.
+MEASURED_TRAFFIC = {"bwd_attn_dkdv": (564.265728e6 + 245.748224e6, 16384)}
+
 
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -391,7 +398,11 @@ def main():
         "fwd_bwd_frac_of_bf16_burst_peak": frac_step * sustained / burst,
         "peak_source": f"{src} (sustained {sustained} TFLOP/s for the step fractions)",
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                     "frac": achieved / sustained, "traffic": None,
+                     "frac": achieved / sustained,
+                     "traffic": (MEASURED_TRAFFIC[dom][0] * S / MEASURED_TRAFFIC[dom][1]) if dom in MEASURED_TRAFFIC
+                     else None,
+                     "traffic_note": "ncu dram bytes of one launch at S=16384 scaled by S" if dom in MEASURED_TRAFFIC
+                     else "not measured for this kernel",
                      "peak_note": f"{src} sustained bf16 (kernel timed inside a long step)"},
         "stage_ms_per_step": {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()},
         "stage_share": {k: round(v[0] / total_ms, 4) for k, v in stages.items()},

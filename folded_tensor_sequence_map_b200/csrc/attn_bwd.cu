@@ -369,6 +369,7 @@ __global__ void __launch_bounds__(320, 1)
                 // each group packs its 32 queries into the first 16 of the 32
                 // columns it has just read, so no group writes what the other
                 // still has to read
+                if (!warp_converged("P^T/dS^T TMEM store")) { ok = false; break; }
                 tmem_st16(tmem + lane_off + 64 * b + 32 * wg, pk);
                 tmem_st16(tmem + lane_off + 128 + 64 * b + 32 * wg, dk);
                 tmem_st_wait();
@@ -587,6 +588,7 @@ __global__ void __launch_bounds__(320, 1)
                     pk[e / 2] = pack_bf16(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
                 }
                 // packed into the first 16 of the 32 columns this group just read
+                if (!warp_converged("dS TMEM store")) { ok = false; break; }
                 tmem_st16(tmem + lane_off + 64 * b + 32 * wg, pk);
                 tmem_st_wait();
                 tc_fence_before();

@@ -321,6 +321,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     }
                 }
                 m = m_use;
+                if (!warp_converged("softmax TMEM store")) { ok = false; break; }
                 // eight independent partial sums
                 float ls[8];
 #pragma unroll

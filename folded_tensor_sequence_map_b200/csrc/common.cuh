@@ -171,9 +171,11 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 
 // tcgen05.ld / tcgen05.st are warp-collective (.sync.aligned): executed by
 // part of a warp they never complete, and no bounded wait can rescue the CTA.
-// Each wrapper therefore checks that the whole warp is converged; if not it
-// skips the instruction and reports, turning a hang into wrong results plus a
-// message (and, downstream, a bounded-wait timeout).
+// Kernels therefore keep every branch around them warp-uniform, and call
+// warp_converged() once per phase (not per instruction, which would split
+// batched TMEM loads) before their TMEM accesses: on a partially active warp
+// it reports and the phase is skipped, so a divergence mistake ends in a
+// bounded-wait timeout instead of a hang.
 __device__ __forceinline__ bool warp_converged(const char *what) {
     if (__activemask() == 0xffffffffu) return true;
     printf("tsp: %s on a partially active warp skipped (block %d thread %d)\n", what, blockIdx.x, threadIdx.x);
@@ -183,11 +185,6 @@ __device__ __forceinline__ bool warp_converged(const char *what) {
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane
 // (quarter*32 + i), columns [col, col+32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    if (!warp_converged("tcgen05.ld")) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        return;
-    }
     uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -203,7 +200,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-    if (!warp_converged("tcgen05.st")) return;
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -223,7 +219,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 }
 // Same as tmem_st32 for raw 32-bit words (e.g. packed bf16 pairs).
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
-    if (!warp_converged("tcgen05.st")) return;
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -236,7 +231,6 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
 }
 // 32 lanes x 16 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-    if (!warp_converged("tcgen05.st")) return;
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
@@ -244,12 +238,8 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
         "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait() {
-    if (warp_converged("tcgen05.wait::ld")) asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-    if (warp_converged("tcgen05.wait::st")) asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---- small numeric helpers -------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
