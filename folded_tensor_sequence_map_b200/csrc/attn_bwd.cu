@@ -17,7 +17,7 @@
 //                dV += P^T dO and dK += dS^T Q accumulate in TMEM.
 //   attn_dq2     one item = (head, 128-row query tile); steps of 64 keys.
 //                S = Q K^T, dP = dO V^T in TMEM; dS to smem; dQ += dS K.
-// Warp roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2-9 element-wise (two
+// Warp roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2-17 element-wise (four
 // groups of four; thread = TMEM lane = row of the 128-row tile).
 #include "common.cuh"
 #include "internal.h"
@@ -126,11 +126,12 @@ struct BwdParams {
 //   TMEM: S^T buffers [2] at columns 0 / 64, dP^T buffers [2] at 128 / 192,
 //         dV at 256, dK at 384 (128 key lanes each).
 //   The MMA warp issues S^T/dP^T of step g+1 before dV/dK of step g, so the
-//   tensor core works on the next step while the element-wise warps (two
-//   groups of four, 32 query columns each) turn step g into P^T and dS^T.
-//   P^T and dS^T go back into TMEM as packed bf16 (two queries per column) in
-//   the columns their S^T / dP^T values came from, where the dV / dK MMAs
-//   read them as the A operand.
+//   tensor core works on the next step while the element-wise warps (four
+//   groups of four, 16 query columns each: four warps per SM sub-partition
+//   to hide TMEM and barrier latency) turn step g into P^T and dS^T.  P^T and
+//   dS^T go back into TMEM as packed bf16 (two queries per column) in the
+//   columns their S^T / dP^T values came from, where the dV / dK MMAs read
+//   them as the A operand.
 template <int DH>
 struct KvCfg {
     using C = BCfg<DH>;
@@ -175,8 +176,11 @@ struct KvParams {
     int num_items;
 };
 
+constexpr int kEwGroups = 4;                          // element-wise groups of four warps
+constexpr int kBwdThreads2 = 64 + 128 * kEwGroups;     // + TMA warp + MMA warp
+
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kBwdThreads2, 1)
     attn_dkdv2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                       const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
                       const KvParams kp, const DevErr err) {
@@ -190,10 +194,10 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t *kv_full = bars + 0, *kv_empty = bars + 1;
     uint64_t *q_full = bars + 2;                 // [QST]
     uint64_t *q_empty = q_full + K::QST;         // [QST]
-    uint64_t *s_full = q_empty + K::QST;         // [2]
-    uint64_t *p_full = s_full + 2;
-    uint64_t *pd_free = p_full + 1;
-    uint64_t *drain = pd_free + 1;
+    uint64_t *s_full = q_empty + K::QST;         // [2] S^T / dP^T of a step ready
+    uint64_t *p_full = s_full + 2;               // [2] P^T / dS^T of a step packed
+    uint64_t *acc_full = p_full + 2;             // dV / dK of an item complete
+    uint64_t *drain = acc_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -211,8 +215,13 @@ __global__ void __launch_bounds__(320, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(p_full, 256);
-        mbar_init(pd_free, 1);
+        // One P barrier per S buffer: a group that has finished step g may take
+        // step g + 1 (its S is issued early) while others still work on g, so
+        // the two steps' arrivals must not land on the same barrier.  Step
+        // g + 2 cannot start before every group has arrived for g.
+        mbar_init(&p_full[0], 128 * kEwGroups);
+        mbar_init(&p_full[1], 128 * kEwGroups);
+        mbar_init(acc_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -263,7 +272,10 @@ __global__ void __launch_bounds__(320, 1)
                 }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        // The whole warp runs the issue loop (warp-uniform control flow and
+        // operands); one elected lane issues every MMA and commit.
+        {
+            const bool leader = elect_one();
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
             const uint32_t k_b = smem_u32(smem + K::OFF_K), v_b = smem_u32(smem + K::OFF_V);
@@ -271,21 +283,24 @@ __global__ void __launch_bounds__(320, 1)
             bool ok = true;
             auto issue_sdp = [&](int gi) -> bool {
                 const int s = gi % K::QST, b = gi & 1;
-                if (!mbar_wait(&q_full[s], (gi / K::QST) & 1, abort_flag, err)) return false;
+                if (!warp_wait(&q_full[s], (gi / K::QST) & 1, abort_flag, err)) return false;
                 tc_fence_after();
                 const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
                 const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
-                for (int kk = 0; kk < DH / 16; ++kk)
-                    umma_bf16(tmem + 64 * b, kdesc<DH>(k_b, kk), kdesc64<DH>(q_b, kk), idS, kk > 0);
-                for (int kk = 0; kk < DH / 16; ++kk)
-                    umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(v_b, kk), kdesc64<DH>(do_b, kk), idS, kk > 0);
-                umma_commit(&s_full[b]);
+                if (leader) {
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 64 * b, kdesc<DH>(k_b, kk), kdesc64<DH>(q_b, kk), idS, kk > 0);
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(v_b, kk), kdesc64<DH>(do_b, kk), idS, kk > 0);
+                    umma_commit(&s_full[b]);
+                }
+                __syncwarp();
                 return true;
             };
             for (int it = blockIdx.x; it < kp.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int kt = a.kv_order[it] / a.H;
                 const int kv0 = kt * 128;
-                if (!mbar_wait(kv_full, item_iter & 1, abort_flag, err)) break;
+                if (!warp_wait(kv_full, item_iter & 1, abort_flag, err)) break;
                 tc_fence_after();
                 int q = next_visible(kp.qmax64, nq64, 0, kv0);
                 if (q < nq64 && !issue_sdp(g)) break;
@@ -293,38 +308,49 @@ __global__ void __launch_bounds__(320, 1)
                 while (q < nq64) {
                     const int qn = next_visible(kp.qmax64, nq64, q + 1, kv0);
                     if (qn < nq64 && !issue_sdp(g + 1)) { ok = false; break; }
-                    if (!mbar_wait(p_full, g & 1, abort_flag, err)) { ok = false; break; }
+                    if (!warp_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
                     const int s = g % K::QST;
                     const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
                     const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
                     const int b = g & 1;
-                    // A operands from TMEM: queries 16 kk.. at column 32 (kk / 2) + 8 (kk % 2)
-                    for (int kk = 0; kk < K::BQ / 16; ++kk)
-                        umma_bf16_ts(tmem + 256, tmem + 64 * b + (kk >> 1) * 32 + (kk & 1) * 8, mndesc64<DH>(do_b, kk),
-                                     idG, (!first || kk > 0) ? 1u : 0u);
-                    for (int kk = 0; kk < K::BQ / 16; ++kk)
-                        umma_bf16_ts(tmem + 384, tmem + 128 + 64 * b + (kk >> 1) * 32 + (kk & 1) * 8,
-                                     mndesc64<DH>(q_b, kk), idG, (!first || kk > 0) ? 1u : 0u);
-                    umma_commit(&q_empty[s]);
-                    umma_commit(pd_free);
+                    if (leader) {
+                        // A operands from TMEM: queries 16 kk .. 16 kk + 15 packed at column 16 kk
+                        for (int kk = 0; kk < K::BQ / 16; ++kk)
+                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, mndesc64<DH>(do_b, kk), idG,
+                                         (!first || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < K::BQ / 16; ++kk)
+                            umma_bf16_ts(tmem + 384, tmem + 128 + 64 * b + kk * 16, mndesc64<DH>(q_b, kk), idG,
+                                         (!first || kk > 0) ? 1u : 0u);
+                        umma_commit(&q_empty[s]);
+                    }
+                    __syncwarp();
                     first = false;
                     ++g;
                     q = qn;
                 }
-                umma_commit(kv_empty);
+                // one commit per item that had steps, so the element-wise warps'
+                // wait for it is exact (a per-step commit would let a wait on
+                // the last step's parity pass while an earlier step runs)
+                if (leader) {
+                    if (ok && !first) umma_commit(acc_full);
+                    umma_commit(kv_empty);
+                }
+                __syncwarp();
             }
-            if (!ok || *abort_flag) {
+            const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
+            if (bad && leader) {
                 umma_commit(drain);
                 spin_drain(drain, 0, err.wait_limit);
             }
+            __syncwarp();
         }
     } else {
-        const int wg = (warp - 2) / 4;          // query columns [32 wg, 32 wg + 32) of a step
+        const int grp = (warp - 2) / 4;         // query columns [16 grp, 16 grp + 16) of a step
         const int quarter = warp & 3;
         const int trow = quarter * 32 + lane;   // key row of the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        int g = 0;
+        int g = 0, acc_iter = 0;
         for (int it = blockIdx.x; it < kp.num_items; it += gridDim.x) {
             const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
             const int kv0 = kt * 128;
@@ -336,21 +362,21 @@ __global__ void __launch_bounds__(320, 1)
                 const int b = g & 1, s = g % K::QST;
                 if (!warp_wait(&s_full[b], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
-                float sv[32], dp[32];
-                tmem_ld32(tmem + lane_off + 64 * b + 32 * wg, sv);
-                tmem_ld32(tmem + lane_off + 128 + 64 * b + 32 * wg, dp);
+                float sv[16], dp[16];
+                tmem_ld16(tmem + lane_off + 64 * b + 16 * grp, sv);
+                tmem_ld16(tmem + lane_off + 128 + 64 * b + 16 * grp, dp);
                 tmem_ld_wait();
                 const float *vec = reinterpret_cast<const float *>(smem + K::OFF_VEC + s * K::VEC_BYTES);
                 const int *pos = reinterpret_cast<const int *>(vec + 128);
                 // the 64 query rows of a step lie in one zigzag chunk (chunks are
                 // multiples of 64 rows), so their positions are consecutive: this
                 // key is visible to column e of the group iff e >= key - pos0
-                const int first_vis = key - pos[32 * wg];
-                const float4 *lse4 = reinterpret_cast<const float4 *>(vec + 32 * wg);
-                const float4 *dl4 = reinterpret_cast<const float4 *>(vec + 64 + 32 * wg);
-                uint32_t pk[16], dk[16];
+                const int first_vis = key - pos[16 * grp];
+                const float4 *lse4 = reinterpret_cast<const float4 *>(vec + 16 * grp);
+                const float4 *dl4 = reinterpret_cast<const float4 *>(vec + 64 + 16 * grp);
+                uint32_t pk[8], dk[8];
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
+                for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 l = lse4[e4], d = dl4[e4];
                     const int e = 4 * e4;
                     float p0 = ex2b(fmaf(sv[e], sl2, -l.x)), p1 = ex2b(fmaf(sv[e + 1], sl2, -l.y));
@@ -366,29 +392,32 @@ __global__ void __launch_bounds__(320, 1)
                     dk[2 * e4] = pack_bf16(p0 * (dp[e] - d.x), p1 * (dp[e + 1] - d.y));
                     dk[2 * e4 + 1] = pack_bf16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
                 }
-                // each group packs its 32 queries into the first 16 of the 32
-                // columns it has just read, so no group writes what the other
+                // each group packs its 16 queries into the first 8 of the 16
+                // columns it has just read, so no group writes what another
                 // still has to read
                 if (!warp_converged("P^T/dS^T TMEM store")) { ok = false; break; }
-                tmem_st16(tmem + lane_off + 64 * b + 32 * wg, pk);
-                tmem_st16(tmem + lane_off + 128 + 64 * b + 32 * wg, dk);
+                tmem_st8u(tmem + lane_off + 64 * b + 16 * grp, pk);
+                tmem_st8u(tmem + lane_off + 128 + 64 * b + 16 * grp, dk);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(p_full);
+                mbar_arrive(&p_full[b]);
             }
             if (!ok) break;
             if (!any) continue;
-            if (!warp_wait(pd_free, (g - 1) & 1, abort_flag, err)) break;
+            if (!warp_wait(acc_full, acc_iter & 1, abort_flag, err)) break;
+            ++acc_iter;
             tc_fence_after();
-            // group 0 writes dV, group 1 writes dK (scaled), at the key owner's local row
+            // groups 0, 1 write dV and groups 2, 3 write dK (scaled), at the key
+            // owner's local row; each pair splits the 32-column chunks
             const int lrow = a.inv_map[key];
-            void *dst = wg == 0 ? a.dv : a.dk;
-            const float f = wg == 0 ? 1.0f : scale;
+            const int which = grp >> 1;
+            void *dst = which == 0 ? a.dv : a.dk;
+            const float f = which == 0 ? 1.0f : scale;
             __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(dst) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
 #pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
+            for (int c = grp & 1; c < DH / 32; c += 2) {
                 float v[32];
-                tmem_ld32(tmem + lane_off + 256 + 128 * wg + c * 32, v);
+                tmem_ld32(tmem + lane_off + 256 + 128 * which + c * 32, v);
                 tmem_ld_wait();
                 uint4 *d4 = reinterpret_cast<uint4 *>(row + c * 32);
 #pragma unroll
@@ -428,7 +457,7 @@ struct Dq2Cfg {
 };
 
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kBwdThreads2, 1)
     attn_dq2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
                     const BwdParams bp, const DevErr err) {
@@ -442,10 +471,10 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t *q_full = bars + 0, *q_empty = bars + 1;
     uint64_t *k_full = bars + 2;            // [KST]
     uint64_t *k_empty = k_full + Q::KST;    // [KST]
-    uint64_t *s_full = k_empty + Q::KST;    // [2]
-    uint64_t *p_full = s_full + 2;
-    uint64_t *ds_free = p_full + 1;
-    uint64_t *drain = ds_free + 1;
+    uint64_t *s_full = k_empty + Q::KST;    // [2] S / dP of a step ready
+    uint64_t *p_full = s_full + 2;          // [2] dS of a step packed
+    uint64_t *acc_full = p_full + 2;        // dQ of an item complete
+    uint64_t *drain = acc_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -462,8 +491,11 @@ __global__ void __launch_bounds__(320, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(p_full, 256);
-        mbar_init(ds_free, 1);
+        // per-buffer dS barriers and a per-item accumulator barrier, for the
+        // reasons given in the dK/dV kernel
+        mbar_init(&p_full[0], 128 * kEwGroups);
+        mbar_init(&p_full[1], 128 * kEwGroups);
+        mbar_init(acc_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -512,7 +544,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        // warp-uniform issue loop, one elected lane issuing (as in the dK/dV kernel)
+        {
+            const bool leader = elect_one();
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
             const uint32_t q_b = smem_u32(smem + Q::OFF_Q), do_b = smem_u32(smem + Q::OFF_DO);
@@ -520,50 +554,61 @@ __global__ void __launch_bounds__(320, 1)
             bool ok = true;
             auto issue_sdp = [&](int gi) -> bool {
                 const int s = gi % Q::KST, b = gi & 1;
-                if (!mbar_wait(&k_full[s], (gi / Q::KST) & 1, abort_flag, err)) return false;
+                if (!warp_wait(&k_full[s], (gi / Q::KST) & 1, abort_flag, err)) return false;
                 tc_fence_after();
                 const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
                 const uint32_t v_b = smem_u32(smem + Q::OFF_V + s * Q::KTILE);
-                for (int kk = 0; kk < DH / 16; ++kk)
-                    umma_bf16(tmem + 64 * b, kdesc<DH>(q_b, kk), kdesc64<DH>(k_b, kk), idS, kk > 0);
-                for (int kk = 0; kk < DH / 16; ++kk)
-                    umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(do_b, kk), kdesc64<DH>(v_b, kk), idS, kk > 0);
-                umma_commit(&s_full[b]);
+                if (leader) {
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 64 * b, kdesc<DH>(q_b, kk), kdesc64<DH>(k_b, kk), idS, kk > 0);
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(do_b, kk), kdesc64<DH>(v_b, kk), idS, kk > 0);
+                    umma_commit(&s_full[b]);
+                }
+                __syncwarp();
                 return true;
             };
             for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int qt = a.q_order[it] / a.H;
-                if (!mbar_wait(q_full, item_iter & 1, abort_flag, err)) break;
+                if (!warp_wait(q_full, item_iter & 1, abort_flag, err)) break;
                 tc_fence_after();
                 const int n = nkv64(qt);
                 if (!issue_sdp(g)) break;
                 for (int j = 0; j < n; ++j, ++g) {
                     if (j + 1 < n && !issue_sdp(g + 1)) { ok = false; break; }
-                    if (!mbar_wait(p_full, g & 1, abort_flag, err)) { ok = false; break; }
+                    if (!warp_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
                     const int s = g % Q::KST, b = g & 1;
                     const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
-                    // A = dS from TMEM: keys 16 kk.. at column 32 (kk / 2) + 8 (kk % 2)
-                    for (int kk = 0; kk < Q::BK / 16; ++kk)
-                        umma_bf16_ts(tmem + 256, tmem + 64 * b + (kk >> 1) * 32 + (kk & 1) * 8, mndesc64<DH>(k_b, kk),
-                                     idG, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&k_empty[s]);
-                    umma_commit(ds_free);
+                    if (leader) {
+                        // A = dS from TMEM: keys 16 kk .. 16 kk + 15 packed at column 16 kk
+                        for (int kk = 0; kk < Q::BK / 16; ++kk)
+                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, mndesc64<DH>(k_b, kk), idG,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&k_empty[s]);
+                    }
+                    __syncwarp();
                 }
-                umma_commit(q_empty);
+                if (leader) {
+                    if (ok) umma_commit(acc_full);
+                    umma_commit(q_empty);
+                }
+                __syncwarp();
             }
-            if (!ok || *abort_flag) {
+            const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
+            if (bad && leader) {
                 umma_commit(drain);
                 spin_drain(drain, 0, err.wait_limit);
             }
+            __syncwarp();
         }
     } else {
-        const int wg = (warp - 2) / 4;          // key columns [32 wg, 32 wg + 32) of a step
+        const int grp = (warp - 2) / 4;         // key columns [16 grp, 16 grp + 16) of a step
         const int quarter = warp & 3;
         const int trow = quarter * 32 + lane;   // query row of the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         int g = 0;
-        for (int it = blockIdx.x; it < bp.num_items; it += gridDim.x) {
+        for (int it = blockIdx.x, item_iter = 0; it < bp.num_items; it += gridDim.x, ++item_iter) {
             const int qt = a.q_order[it] / a.H, head = a.q_order[it] % a.H;
             const int lrow = qt * 128 + trow;
             const int pos = bp.zig[lrow];
@@ -575,32 +620,32 @@ __global__ void __launch_bounds__(320, 1)
                 const int b = g & 1;
                 if (!warp_wait(&s_full[b], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
-                float sv[32], dp[32];
-                tmem_ld32(tmem + lane_off + 64 * b + 32 * wg, sv);
-                tmem_ld32(tmem + lane_off + 128 + 64 * b + 32 * wg, dp);
+                float sv[16], dp[16];
+                tmem_ld16(tmem + lane_off + 64 * b + 16 * grp, sv);
+                tmem_ld16(tmem + lane_off + 128 + 64 * b + 16 * grp, dp);
                 tmem_ld_wait();
-                const int k0 = j * 64 + 32 * wg;
-                uint32_t pk[16];
+                const int k0 = j * 64 + 16 * grp;
+                uint32_t pk[8];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
+                for (int e = 0; e < 16; e += 2) {
                     const float p0 = (k0 + e <= pos) ? ex2b(fmaf(sv[e], sl2, -lse)) : 0.f;
                     const float p1 = (k0 + e + 1 <= pos) ? ex2b(fmaf(sv[e + 1], sl2, -lse)) : 0.f;
                     pk[e / 2] = pack_bf16(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
                 }
-                // packed into the first 16 of the 32 columns this group just read
+                // packed into the first 8 of the 16 columns this group just read
                 if (!warp_converged("dS TMEM store")) { ok = false; break; }
-                tmem_st16(tmem + lane_off + 64 * b + 32 * wg, pk);
+                tmem_st8u(tmem + lane_off + 64 * b + 16 * grp, pk);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(p_full);
+                mbar_arrive(&p_full[b]);
             }
             if (!ok) break;
-            if (!warp_wait(ds_free, (g - 1) & 1, abort_flag, err)) break;
+            if (!warp_wait(acc_full, item_iter & 1, abort_flag, err)) break;
             tc_fence_after();
-            if (wg == 0) {
+            {
                 __nv_bfloat16 *dqrow = static_cast<__nv_bfloat16 *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
 #pragma unroll 1
-                for (int c = 0; c < DH / 32; ++c) {
+                for (int c = grp; c < DH / 32; c += kEwGroups) {
                     float v[32];
                     tmem_ld32(tmem + lane_off + 256 + c * 32, v);
                     tmem_ld_wait();
@@ -667,7 +712,7 @@ cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sm
     auto k1 = attn_dkdv2_kernel<DH>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, KvCfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
-    k1<<<grid, 320, KvCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, kp, err);
+    k1<<<grid, kBwdThreads2, KvCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, kp, err);
     return cudaGetLastError();
 }
 
@@ -688,7 +733,7 @@ cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms,
     auto k2 = attn_dq2_kernel<DH>;
     cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, Dq2Cfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
-    k2<<<grid, 320, Dq2Cfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, bp, err);
+    k2<<<grid, kBwdThreads2, Dq2Cfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, bp, err);
     return cudaGetLastError();
 }
 

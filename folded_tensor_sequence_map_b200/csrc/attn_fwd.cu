@@ -182,7 +182,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop, so its control flow and operands stay
+        // warp-uniform; one elected lane issues every MMA and commit (a commit
+        // tracks the MMAs of the thread that issues it).
+        {
+            const bool leader = elect_one();
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
             const uint32_t qbase = smem_u32(smem + C::OFF_Q);
@@ -190,63 +194,74 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             bool ok = true;
             for (int it = blockIdx.x; it < a.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int nkv = a.order[2 * it + 1];
-                if (!mbar_wait(q_full, item_iter & 1, abort_flag, err)) break;
+                if (!warp_wait(q_full, item_iter & 1, abort_flag, err)) break;
                 tc_fence_after();
                 // prologue: S_w for key tile 0
                 {
                     const int ks = kcount % C::KST;
-                    if (!mbar_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) break;
+                    if (!warp_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) break;
                     tc_fence_after();
                     const uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
-                    for (int w = 0; w < 2; ++w) {
-                        for (int kk = 0; kk < DH / 16; ++kk)
-                            umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
-                                      kmajor_desc<DH>(kb, kk), idS, kk > 0);
-                        umma_commit(&s_full[w]);
-                    }
-                    umma_commit(&k_empty[ks]);
-                    ++kcount;
-                }
-                for (int j = 0; j < nkv && ok; ++j, ++tcount) {
-                    const int vs = vcount % C::VST;
-                    if (!mbar_wait(&v_full[vs], (vcount / C::VST) & 1, abort_flag, err)) { ok = false; break; }
-                    const uint32_t vb = smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES);
-                    int ks = kcount % C::KST;
-                    uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
-                    for (int w = 0; w < 2; ++w) {
-                        if (!mbar_wait(&p_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
-                        tc_fence_after();
-                        // P_w sits in TMEM columns [128 w, 128 w + 64): 16 keys per 8 columns
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, mnmajor_desc<DH>(vb, kk),
-                                         idO, (j > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit(&o_done[w]);
-                        if (j + 1 < nkv) {
-                            if (w == 0) {
-                                if (!mbar_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) { ok = false; break; }
-                                tc_fence_after();
-                            }
+                    if (leader) {
+                        for (int w = 0; w < 2; ++w) {
                             for (int kk = 0; kk < DH / 16; ++kk)
                                 umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
                                           kmajor_desc<DH>(kb, kk), idS, kk > 0);
                             umma_commit(&s_full[w]);
-                            if (w == 1) {
-                                umma_commit(&k_empty[ks]);
-                                ++kcount;
+                        }
+                        umma_commit(&k_empty[ks]);
+                    }
+                    __syncwarp();
+                    ++kcount;
+                }
+                for (int j = 0; j < nkv && ok; ++j, ++tcount) {
+                    const int vs = vcount % C::VST;
+                    if (!warp_wait(&v_full[vs], (vcount / C::VST) & 1, abort_flag, err)) { ok = false; break; }
+                    const uint32_t vb = smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES);
+                    int ks = kcount % C::KST;
+                    uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
+                    for (int w = 0; w < 2; ++w) {
+                        if (!warp_wait(&p_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
+                        tc_fence_after();
+                        // P_w sits in TMEM columns [128 w, 128 w + 64): 16 keys per 8 columns
+                        if (leader) {
+                            for (int kk = 0; kk < 8; ++kk)
+                                umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, mnmajor_desc<DH>(vb, kk),
+                                             idO, (j > 0 || kk > 0) ? 1u : 0u);
+                            umma_commit(&o_done[w]);
+                        }
+                        __syncwarp();
+                        if (j + 1 < nkv) {
+                            if (w == 0) {
+                                if (!warp_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) { ok = false; break; }
+                                tc_fence_after();
                             }
+                            if (leader) {
+                                for (int kk = 0; kk < DH / 16; ++kk)
+                                    umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
+                                              kmajor_desc<DH>(kb, kk), idS, kk > 0);
+                                umma_commit(&s_full[w]);
+                                if (w == 1) umma_commit(&k_empty[ks]);
+                            }
+                            __syncwarp();
+                            if (w == 1) ++kcount;
                         }
                     }
                     if (!ok) break;
-                    umma_commit(&v_empty[vs]);
+                    if (leader) umma_commit(&v_empty[vs]);
+                    __syncwarp();
                     ++vcount;
                 }
-                umma_commit(q_empty);
+                if (leader) umma_commit(q_empty);
+                __syncwarp();
             }
-            if (!ok || *abort_flag) {
+            const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
+            if (bad && leader) {
                 umma_commit(drain);
                 long long t0 = clock64();
                 while (!mbar_try_wait(drain, 0) && clock64() - t0 < err.wait_limit) {}
             }
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------ softmax groups
