@@ -164,15 +164,49 @@ __device__ __forceinline__ uint64_t mndesc64(uint32_t base, int kk) {
     using K = KvCfg<DH>;
     return sdesc(base + kk * 16 * C::SWB, K::QATOM, 8 * C::SWB, C::LAYOUT);
 }
-__device__ __forceinline__ int next_visible(const int *qmax64, int nq64, int from, int kv0) {
-    while (from < nq64 && qmax64[from] < kv0) ++from;
-    return from;
+// Byte offsets of K step kk from step 0 in the three operand layouts above,
+// so an issue loop builds each descriptor once and advances it (desc_plus).
+template <int DH>
+__host__ __device__ constexpr uint32_t kdesc_off(int kk) {
+    return (kk * 16 / BCfg<DH>::ATOM_COLS) * BCfg<DH>::ATOM_BYTES + (kk * 16 % BCfg<DH>::ATOM_COLS) * 2;
+}
+template <int DH>
+__host__ __device__ constexpr uint32_t kdesc64_off(int kk) {
+    return (kk * 16 / BCfg<DH>::ATOM_COLS) * (64 * BCfg<DH>::SWB) + (kk * 16 % BCfg<DH>::ATOM_COLS) * 2;
+}
+template <int DH>
+__host__ __device__ constexpr uint32_t mndesc64_off(int kk) {
+    return kk * 16 * BCfg<DH>::SWB;
 }
 
+// Visibility of 64-row query steps to a key tile, from the zigzag layout.
+struct StepVis {
+    int D, chunk, nq64;
+};
+__device__ __forceinline__ int next_visible(const StepVis &v, int from, int kv0) {
+    return zz_next_visible(from, kv0, v.D, v.chunk, v.nq64);
+}
+
+// Walks the query steps that can see a key tile, in ascending order.  Within
+// a zigzag chunk the visible steps form a suffix, so after a chunk's first
+// visible step every later step of that chunk is visible too: the closed form
+// runs once per chunk and a step costs one compare.
+struct StepWalk {
+    int q;        // current step; nq64 once the walk is over
+    int run_end;  // end (exclusive) of the chunk holding q
+    __device__ __forceinline__ void seek(const StepVis &v, int from, int kv0) {
+        q = next_visible(v, from, kv0);
+        const int spc = v.chunk >> 6;
+        run_end = q < v.nq64 ? (q / spc + 1) * spc : v.nq64;
+    }
+    __device__ __forceinline__ void next(const StepVis &v, int kv0) {
+        if (q + 1 < run_end) ++q;
+        else seek(v, q + 1, kv0);
+    }
+};
 struct KvParams {
     AttnBwdDesc d;
     const int *zig;
-    const int *qmax64;  // per 64-row local query tile, largest global position
     int num_items;
 };
 
@@ -203,6 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nq64 = a.S / 64;
+    const StepVis vis{a.D, a.chunk, nq64};
     const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
     const float scale = rsqrtf(static_cast<float>(DH));
 
@@ -247,8 +282,9 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                     tma_load_2d(smem + K::OFF_K + t * C::ATOM_BYTES, &mK, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
                     tma_load_2d(smem + K::OFF_V + t * C::ATOM_BYTES, &mV, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
                 }
-                for (int q = next_visible(kp.qmax64, nq64, 0, kt * 128); q < nq64;
-                     q = next_visible(kp.qmax64, nq64, q + 1, kt * 128), ++g) {
+                StepWalk w;
+                for (w.seek(vis, 0, kt * 128); w.q < nq64; w.next(vis, kt * 128), ++g) {
+                    const int q = w.q;
                     const int s = g % K::QST;
                     if (!mbar_wait(&q_empty[s], ((g / K::QST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
                     mbar_arrive_tx(&q_full[s], 2 * K::QTILE + K::VEC_BYTES);
@@ -272,62 +308,73 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                 }
         }
     } else if (warp == 1) {
-        // The whole warp runs the issue loop (warp-uniform control flow and
-        // operands); one elected lane issues every MMA and commit.
+        // The whole warp runs the issue loop (warp-uniform control flow); one
+        // elected lane polls the barriers and issues every MMA and commit.
+        // Operand descriptors are built once per tile and advanced by
+        // compile-time offsets.
         {
             const bool leader = elect_one();
+            const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
-            const uint32_t k_b = smem_u32(smem + K::OFF_K), v_b = smem_u32(smem + K::OFF_V);
+            const uint64_t dK0 = kdesc<DH>(smem_u32(smem + K::OFF_K), 0);
+            const uint64_t dV0 = kdesc<DH>(smem_u32(smem + K::OFF_V), 0);
             int item_iter = 0, g = 0;
             bool ok = true;
             auto issue_sdp = [&](int gi) -> bool {
                 const int s = gi % K::QST, b = gi & 1;
-                if (!warp_wait(&q_full[s], (gi / K::QST) & 1, abort_flag, err)) return false;
-                tc_fence_after();
-                const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
-                const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
+                if (!lead_wait(leader, leader_lane, &q_full[s], (gi / K::QST) & 1, abort_flag, err)) return false;
                 if (leader) {
+                    tc_fence_after();
+                    const uint64_t dQ0 = kdesc64<DH>(smem_u32(smem + K::OFF_Q + s * K::QTILE), 0);
+                    const uint64_t dO0 = kdesc64<DH>(smem_u32(smem + K::OFF_DO + s * K::QTILE), 0);
+#pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 64 * b, kdesc<DH>(k_b, kk), kdesc64<DH>(q_b, kk), idS, kk > 0);
+                        umma_bf16(tmem + 64 * b, desc_plus(dK0, kdesc_off<DH>(kk)), desc_plus(dQ0, kdesc64_off<DH>(kk)),
+                                  idS, kk > 0);
+#pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(v_b, kk), kdesc64<DH>(do_b, kk), idS, kk > 0);
+                        umma_bf16(tmem + 128 + 64 * b, desc_plus(dV0, kdesc_off<DH>(kk)),
+                                  desc_plus(dO0, kdesc64_off<DH>(kk)), idS, kk > 0);
                     umma_commit(&s_full[b]);
                 }
-                __syncwarp();
                 return true;
             };
             for (int it = blockIdx.x; it < kp.num_items && ok; it += gridDim.x, ++item_iter) {
-                const int kt = a.kv_order[it] / a.H;
-                const int kv0 = kt * 128;
-                if (!warp_wait(kv_full, item_iter & 1, abort_flag, err)) break;
-                tc_fence_after();
-                int q = next_visible(kp.qmax64, nq64, 0, kv0);
-                if (q < nq64 && !issue_sdp(g)) break;
+                const int kv0 = (a.kv_order[it] / a.H) * 128;
+                if (!lead_wait(leader, leader_lane, kv_full, item_iter & 1, abort_flag, err)) break;
+                if (leader) tc_fence_after();
+                StepWalk w;
+                w.seek(vis, 0, kv0);
+                if (w.q < nq64 && !issue_sdp(g)) break;
                 bool first = true;
-                while (q < nq64) {
-                    const int qn = next_visible(kp.qmax64, nq64, q + 1, kv0);
-                    if (qn < nq64 && !issue_sdp(g + 1)) { ok = false; break; }
-                    if (!warp_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const int s = g % K::QST;
-                    const uint32_t q_b = smem_u32(smem + K::OFF_Q + s * K::QTILE);
-                    const uint32_t do_b = smem_u32(smem + K::OFF_DO + s * K::QTILE);
-                    const int b = g & 1;
+                while (w.q < nq64) {
+                    StepWalk wn = w;
+                    wn.next(vis, kv0);
+                    if (wn.q < nq64 && !issue_sdp(g + 1)) { ok = false; break; }
+                    if (!lead_wait(leader, leader_lane, &p_full[g & 1], (g >> 1) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
                     if (leader) {
+                        tc_fence_after();
+                        const int s = g % K::QST, b = g & 1;
+                        const uint64_t gQ0 = mndesc64<DH>(smem_u32(smem + K::OFF_Q + s * K::QTILE), 0);
+                        const uint64_t gO0 = mndesc64<DH>(smem_u32(smem + K::OFF_DO + s * K::QTILE), 0);
                         // A operands from TMEM: queries 16 kk .. 16 kk + 15 packed at column 16 kk
+#pragma unroll
                         for (int kk = 0; kk < K::BQ / 16; ++kk)
-                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, mndesc64<DH>(do_b, kk), idG,
+                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, desc_plus(gO0, mndesc64_off<DH>(kk)), idG,
                                          (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
                         for (int kk = 0; kk < K::BQ / 16; ++kk)
-                            umma_bf16_ts(tmem + 384, tmem + 128 + 64 * b + kk * 16, mndesc64<DH>(q_b, kk), idG,
-                                         (!first || kk > 0) ? 1u : 0u);
+                            umma_bf16_ts(tmem + 384, tmem + 128 + 64 * b + kk * 16, desc_plus(gQ0, mndesc64_off<DH>(kk)),
+                                         idG, (!first || kk > 0) ? 1u : 0u);
                         umma_commit(&q_empty[s]);
                     }
-                    __syncwarp();
                     first = false;
                     ++g;
-                    q = qn;
+                    w = wn;
                 }
                 // one commit per item that had steps, so the element-wise warps'
                 // wait for it is exact (a per-step commit would let a wait on
@@ -336,7 +383,6 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                     if (ok && !first) umma_commit(acc_full);
                     umma_commit(kv_empty);
                 }
-                __syncwarp();
             }
             const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
             if (bad && leader) {
@@ -356,8 +402,8 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             const int kv0 = kt * 128;
             const int key = kv0 + trow;
             bool ok = true, any = false;
-            for (int q = next_visible(kp.qmax64, nq64, 0, kv0); q < nq64;
-                 q = next_visible(kp.qmax64, nq64, q + 1, kv0), ++g) {
+            StepWalk w;
+            for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
                 any = true;
                 const int b = g & 1, s = g % K::QST;
                 if (!warp_wait(&s_full[b], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
@@ -544,56 +590,64 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                 }
         }
     } else if (warp == 1) {
-        // warp-uniform issue loop, one elected lane issuing (as in the dK/dV kernel)
+        // warp-uniform issue loop: one elected lane polls and issues, with
+        // descriptors advanced by constant offsets (as in the dK/dV kernel)
         {
             const bool leader = elect_one();
+            const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
-            const uint32_t q_b = smem_u32(smem + Q::OFF_Q), do_b = smem_u32(smem + Q::OFF_DO);
+            const uint64_t dQ0 = kdesc<DH>(smem_u32(smem + Q::OFF_Q), 0);
+            const uint64_t dO0 = kdesc<DH>(smem_u32(smem + Q::OFF_DO), 0);
             int item_iter = 0, g = 0;
             bool ok = true;
             auto issue_sdp = [&](int gi) -> bool {
                 const int s = gi % Q::KST, b = gi & 1;
-                if (!warp_wait(&k_full[s], (gi / Q::KST) & 1, abort_flag, err)) return false;
-                tc_fence_after();
-                const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
-                const uint32_t v_b = smem_u32(smem + Q::OFF_V + s * Q::KTILE);
+                if (!lead_wait(leader, leader_lane, &k_full[s], (gi / Q::KST) & 1, abort_flag, err)) return false;
                 if (leader) {
+                    tc_fence_after();
+                    const uint64_t dK0 = kdesc64<DH>(smem_u32(smem + Q::OFF_K + s * Q::KTILE), 0);
+                    const uint64_t dV0 = kdesc64<DH>(smem_u32(smem + Q::OFF_V + s * Q::KTILE), 0);
+#pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 64 * b, kdesc<DH>(q_b, kk), kdesc64<DH>(k_b, kk), idS, kk > 0);
+                        umma_bf16(tmem + 64 * b, desc_plus(dQ0, kdesc_off<DH>(kk)), desc_plus(dK0, kdesc64_off<DH>(kk)),
+                                  idS, kk > 0);
+#pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 128 + 64 * b, kdesc<DH>(do_b, kk), kdesc64<DH>(v_b, kk), idS, kk > 0);
+                        umma_bf16(tmem + 128 + 64 * b, desc_plus(dO0, kdesc_off<DH>(kk)),
+                                  desc_plus(dV0, kdesc64_off<DH>(kk)), idS, kk > 0);
                     umma_commit(&s_full[b]);
                 }
-                __syncwarp();
                 return true;
             };
             for (int it = blockIdx.x; it < bp.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int qt = a.q_order[it] / a.H;
-                if (!warp_wait(q_full, item_iter & 1, abort_flag, err)) break;
-                tc_fence_after();
+                if (!lead_wait(leader, leader_lane, q_full, item_iter & 1, abort_flag, err)) break;
+                if (leader) tc_fence_after();
                 const int n = nkv64(qt);
                 if (!issue_sdp(g)) break;
                 for (int j = 0; j < n; ++j, ++g) {
                     if (j + 1 < n && !issue_sdp(g + 1)) { ok = false; break; }
-                    if (!warp_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const int s = g % Q::KST, b = g & 1;
-                    const uint32_t k_b = smem_u32(smem + Q::OFF_K + s * Q::KTILE);
+                    if (!lead_wait(leader, leader_lane, &p_full[g & 1], (g >> 1) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
                     if (leader) {
+                        tc_fence_after();
+                        const int s = g % Q::KST, b = g & 1;
+                        const uint64_t gK0 = mndesc64<DH>(smem_u32(smem + Q::OFF_K + s * Q::KTILE), 0);
                         // A = dS from TMEM: keys 16 kk .. 16 kk + 15 packed at column 16 kk
+#pragma unroll
                         for (int kk = 0; kk < Q::BK / 16; ++kk)
-                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, mndesc64<DH>(k_b, kk), idG,
+                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, desc_plus(gK0, mndesc64_off<DH>(kk)), idG,
                                          (j > 0 || kk > 0) ? 1u : 0u);
                         umma_commit(&k_empty[s]);
                     }
-                    __syncwarp();
                 }
                 if (leader) {
                     if (ok) umma_commit(acc_full);
                     umma_commit(q_empty);
                 }
-                __syncwarp();
             }
             const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
             if (bad && leader) {
@@ -692,8 +746,7 @@ BwdParams make_params(const AttnBwdDesc &a, const int *zig, const int *qtile_max
 }
 
 template <int DH>
-cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
-                             const int *qmax64) {
+cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig) {
     using C = BCfg<DH>;
     BwdMaps<DH> m;
     if (!m.make(a)) return cudaErrorInvalidValue;
@@ -706,7 +759,6 @@ cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sm
     KvParams kp;
     kp.d = a;
     kp.zig = zig;
-    kp.qmax64 = qmax64;
     kp.num_items = (a.S / 128) * a.H;
     const int grid = kp.num_items < num_sms ? kp.num_items : num_sms;
     auto k1 = attn_dkdv2_kernel<DH>;
@@ -747,12 +799,11 @@ cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
-                             const int *qtile_maxpos) {
+cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig) {
     switch (a.dh) {
-        case 32: return launch_dkdv_impl<32>(a, err, num_sms, st, zig, qtile_maxpos);
-        case 64: return launch_dkdv_impl<64>(a, err, num_sms, st, zig, qtile_maxpos);
-        case 128: return launch_dkdv_impl<128>(a, err, num_sms, st, zig, qtile_maxpos);
+        case 32: return launch_dkdv_impl<32>(a, err, num_sms, st, zig);
+        case 64: return launch_dkdv_impl<64>(a, err, num_sms, st, zig);
+        case 128: return launch_dkdv_impl<128>(a, err, num_sms, st, zig);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -74,6 +74,17 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
     using C = FwdCfg<DH>;
     return sdesc(base + kk * 16 * C::SWB, C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
 }
+// Byte offsets of K step kk from step 0 in the two layouts above, so the issue
+// loop builds each descriptor once per tile and advances it (desc_plus).
+template <int DH>
+__host__ __device__ constexpr uint32_t kmajor_off(int kk) {
+    return (kk * 16 / FwdCfg<DH>::ATOM_COLS) * FwdCfg<DH>::ATOM_BYTES + (kk * 16 % FwdCfg<DH>::ATOM_COLS) * 2;
+}
+template <int DH>
+__host__ __device__ constexpr uint32_t mnmajor_off(int kk) {
+    return kk * 16 * FwdCfg<DH>::SWB;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
@@ -182,78 +193,82 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // The whole warp runs this loop, so its control flow and operands stay
-        // warp-uniform; one elected lane issues every MMA and commit (a commit
-        // tracks the MMAs of the thread that issues it).
+        // The whole warp runs this loop (warp-uniform control flow); one
+        // elected lane polls the barriers and issues every MMA and commit (a
+        // commit tracks the MMAs of the thread that issues it).  Descriptors
+        // are built once per tile and advanced by compile-time offsets.
         {
             const bool leader = elect_one();
+            const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
             const uint32_t qbase = smem_u32(smem + C::OFF_Q);
+            const uint64_t dQa = kmajor_desc<DH>(qbase, 0), dQb = kmajor_desc<DH>(qbase + C::TILE_BYTES, 0);
             int kcount = 0, vcount = 0, tcount = 0, item_iter = 0;
             bool ok = true;
+            // S_w = Q_w K^T for the K tile in stage ks
+            auto issue_s = [&](int w, int ks) {
+                const uint64_t dK0 = kmajor_desc<DH>(smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES), 0);
+                const uint64_t dQ0 = w ? dQb : dQa;
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    umma_bf16(tmem + w * 128, desc_plus(dQ0, kmajor_off<DH>(kk)), desc_plus(dK0, kmajor_off<DH>(kk)),
+                              idS, kk > 0);
+                umma_commit(&s_full[w]);
+            };
             for (int it = blockIdx.x; it < a.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int nkv = a.order[2 * it + 1];
-                if (!warp_wait(q_full, item_iter & 1, abort_flag, err)) break;
-                tc_fence_after();
+                if (!lead_wait(leader, leader_lane, q_full, item_iter & 1, abort_flag, err)) break;
                 // prologue: S_w for key tile 0
                 {
                     const int ks = kcount % C::KST;
-                    if (!warp_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) break;
-                    tc_fence_after();
-                    const uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
+                    if (!lead_wait(leader, leader_lane, &k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) break;
                     if (leader) {
-                        for (int w = 0; w < 2; ++w) {
-                            for (int kk = 0; kk < DH / 16; ++kk)
-                                umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
-                                          kmajor_desc<DH>(kb, kk), idS, kk > 0);
-                            umma_commit(&s_full[w]);
-                        }
+                        tc_fence_after();
+                        issue_s(0, ks);
+                        issue_s(1, ks);
                         umma_commit(&k_empty[ks]);
                     }
-                    __syncwarp();
                     ++kcount;
                 }
                 for (int j = 0; j < nkv && ok; ++j, ++tcount) {
                     const int vs = vcount % C::VST;
-                    if (!warp_wait(&v_full[vs], (vcount / C::VST) & 1, abort_flag, err)) { ok = false; break; }
-                    const uint32_t vb = smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES);
-                    int ks = kcount % C::KST;
-                    uint32_t kb = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
+                    if (!lead_wait(leader, leader_lane, &v_full[vs], (vcount / C::VST) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t dV0 = mnmajor_desc<DH>(smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES), 0);
+                    const int ks = kcount % C::KST;
                     for (int w = 0; w < 2; ++w) {
-                        if (!warp_wait(&p_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
-                        tc_fence_after();
-                        // P_w sits in TMEM columns [128 w, 128 w + 64): 16 keys per 8 columns
+                        if (!lead_wait(leader, leader_lane, &p_full[w], tcount & 1, abort_flag, err)) { ok = false; break; }
                         if (leader) {
+                            tc_fence_after();
+                            // P_w sits in TMEM columns [128 w, 128 w + 64): 16 keys per 8 columns
+#pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, mnmajor_desc<DH>(vb, kk),
+                                umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, desc_plus(dV0, mnmajor_off<DH>(kk)),
                                              idO, (j > 0 || kk > 0) ? 1u : 0u);
                             umma_commit(&o_done[w]);
                         }
-                        __syncwarp();
                         if (j + 1 < nkv) {
-                            if (w == 0) {
-                                if (!warp_wait(&k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) { ok = false; break; }
-                                tc_fence_after();
+                            if (w == 0 &&
+                                !lead_wait(leader, leader_lane, &k_full[ks], (kcount / C::KST) & 1, abort_flag, err)) {
+                                ok = false;
+                                break;
                             }
                             if (leader) {
-                                for (int kk = 0; kk < DH / 16; ++kk)
-                                    umma_bf16(tmem + w * 128, kmajor_desc<DH>(qbase + w * C::TILE_BYTES, kk),
-                                              kmajor_desc<DH>(kb, kk), idS, kk > 0);
-                                umma_commit(&s_full[w]);
+                                tc_fence_after();
+                                issue_s(w, ks);
                                 if (w == 1) umma_commit(&k_empty[ks]);
                             }
-                            __syncwarp();
                             if (w == 1) ++kcount;
                         }
                     }
                     if (!ok) break;
                     if (leader) umma_commit(&v_empty[vs]);
-                    __syncwarp();
                     ++vcount;
                 }
                 if (leader) umma_commit(q_empty);
-                __syncwarp();
             }
             const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
             if (bad && leader) {

@@ -93,6 +93,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
+// Wait run by one lane for its whole warp: the leader polls the barrier (with
+// the usual bound) and the outcome is broadcast from `leader_lane`.  Every lane
+// of the warp must call it.
+__device__ __forceinline__ bool lead_wait(bool leader, int leader_lane, uint64_t *bar, uint32_t parity,
+                                          volatile int *abort, const DevErr &e) {
+    int ok = 1;
+    if (leader) ok = mbar_wait(bar, parity, abort, e) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, leader_lane) != 0;
+}
+
 // ---- TMA --------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -127,6 +137,12 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
     d |= static_cast<uint64_t>(layout & 7u) << 61;
     return d;
 }
+
+// Descriptor of an operand `off` bytes past the one `d` describes, with the
+// same layout, strides and swizzle.  The start-address field counts 16-byte
+// units and shared-memory addresses stay below 256 KB, so the sum never
+// carries out of the field.
+__device__ __forceinline__ uint64_t desc_plus(uint64_t d, uint32_t off) { return d + (off >> 4); }
 
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator.
 // a_mn / b_mn select MN-major operands (else K-major).

@@ -85,6 +85,27 @@ struct AttnDesc {
 };
 cudaError_t launch_attn_fwd(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st);
 
+// First local 64-row query step q >= from whose largest global position is at
+// least kv0 (so at least one of its rows sees key kv0), or nq64 when there is
+// none.  The local rows of rank r are its low zigzag chunk r followed by its
+// high chunk 2D - 1 - r, each `chunk` rows (a multiple of 64) with ascending
+// positions; so every step lies in one chunk, and within a chunk the steps
+// that see kv0 form a suffix.  At most 2D chunks are examined.
+__host__ __device__ inline int zz_next_visible(int from, int kv0, int D, int chunk, int nq64) {
+    const int spc = chunk / 64;  // steps per chunk
+    for (int lc = from / spc; lc < 2 * D; ++lc) {
+        const int r = lc >> 1;
+        const int start = ((lc & 1) ? 2 * D - 1 - r : r) * chunk;  // position of the chunk's first row
+        // step t of the chunk ends at position start + 64 t + 63
+        const int need = kv0 - 63 - start;
+        const int t0 = need <= 0 ? 0 : (need + 63) / 64;
+        const int lo = lc * spc;
+        const int t = (from > lo ? from - lo : 0) > t0 ? (from > lo ? from - lo : 0) : t0;
+        if (t < spc) return lo + t;
+    }
+    return nq64;
+}
+
 struct AttnBwdDesc {
     int S, L, D, H, dh, chunk;
     const void *q, *k, *v, *o, *dout;  // q, o, dout local rows; k, v global rows
@@ -98,11 +119,11 @@ struct AttnBwdDesc {
     const int *q_order;                // work order of (head, 128-row query block), longest first
 };
 // Delta = rowsum(dO * O) per head; then dK/dV (key-tile items, 64-row query
-// steps) and dQ (query-tile items).  zig: local row -> global position;
-// qmax64 / qtile_maxpos: largest position of each 64- / 128-row local query tile.
+// steps, visibility from zz_next_visible) and dQ (query-tile items).  zig:
+// local row -> global position; qtile_maxpos: largest position of each
+// 128-row local query tile.
 cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st);
-cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
-                             const int *qmax64);
+cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig);
 cudaError_t launch_attn_dq(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
                            const int *qtile_maxpos);
 

@@ -28,7 +28,7 @@ struct tsp_plan_s {
     bool dev_ready = false;
     int device = -1;
     int num_sms = 0;
-    int32_t *d_zig = nullptr, *d_inv = nullptr, *d_qmax = nullptr, *d_qmax64 = nullptr;
+    int32_t *d_zig = nullptr, *d_inv = nullptr, *d_qmax = nullptr;
     int32_t *d_fwd_order = nullptr, *d_kv_order = nullptr, *d_q_order = nullptr;
     unsigned int *d_err = nullptr;
     int fwd_items = 0;
@@ -124,13 +124,8 @@ tsp_status ensure_device(tsp_plan_s *p) {
     if (!get_encode()) return TSP_ERR_CUDA;
     const int64_t S = p->S;
     const int H = p->H;
-    std::vector<int32_t> inv(S), qmax(S / 128), qmax64(S / 64);
+    std::vector<int32_t> inv(S), qmax(S / 128);
     for (int64_t i = 0; i < S; ++i) inv[p->zig[i]] = static_cast<int32_t>(i);
-    for (int64_t t = 0; t < S / 64; ++t) {
-        int32_t m = 0;
-        for (int64_t i = t * 64; i < t * 64 + 64; ++i) m = std::max(m, p->zig[i]);
-        qmax64[t] = m;
-    }
     for (int64_t t = 0; t < S / 128; ++t) {
         int32_t m = 0;
         for (int64_t i = t * 128; i < t * 128 + 128; ++i) m = std::max(m, p->zig[i]);
@@ -177,7 +172,7 @@ tsp_status ensure_device(tsp_plan_s *p) {
         if (cudaMalloc(dst, v.size() * 4) != cudaSuccess) return false;
         return cudaMemcpy(*dst, v.data(), v.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess;
     };
-    if (!upload(&p->d_zig, p->zig) || !upload(&p->d_inv, inv) || !upload(&p->d_qmax, qmax) || !upload(&p->d_qmax64, qmax64) ||
+    if (!upload(&p->d_zig, p->zig) || !upload(&p->d_inv, inv) || !upload(&p->d_qmax, qmax) ||
         !upload(&p->d_fwd_order, forder) || !upload(&p->d_kv_order, korder) || !upload(&p->d_q_order, qorder))
         return TSP_ERR_CUDA;
     if (cudaMalloc(&p->d_err, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
@@ -353,7 +348,6 @@ TSP_API void tsp_plan_destroy(tsp_plan_t p) {
         cudaFree(p->d_zig);
         cudaFree(p->d_inv);
         cudaFree(p->d_qmax);
-        cudaFree(p->d_qmax64);
         cudaFree(p->d_fwd_order);
         cudaFree(p->d_kv_order);
         cudaFree(p->d_q_order);
@@ -565,7 +559,7 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     ab.kv_order = p->d_kv_order;
     ab.q_order = p->d_q_order;
     TSP_STAGE(14, 1, launch_attn_delta(ab, s));
-    TSP_STAGE(15, 1, launch_attn_dkdv(ab, err, p->num_sms, s, p->d_zig, p->d_qmax64));
+    TSP_STAGE(15, 1, launch_attn_dkdv(ab, err, p->num_sms, s, p->d_zig));
     TSP_STAGE(16, 1, launch_attn_dq(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
     // projection backward: dWqkv = [dQ|dK|dV]^T a, da = [dQ|dK|dV] Wqkv
     TSP_STAGE(17, 1, launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h), err, p->num_sms, s));
@@ -614,6 +608,14 @@ TSP_API tsp_status tsp_test_buffer_offset(tsp_plan_t p, const char *name, size_t
             return TSP_OK;
         }
     return TSP_ERR_INVALID_ARG;
+}
+
+TSP_API tsp_status tsp_test_next_visible(tsp_plan_t p, int from, int kv0, int *out) {
+    if (!p || !out) return TSP_ERR_INVALID_ARG;
+    const int nq64 = static_cast<int>(p->S / 64);
+    if (from < 0 || from > nq64 || kv0 < 0 || kv0 >= p->S) return TSP_ERR_INVALID_ARG;
+    *out = zz_next_visible(from, kv0, p->D, static_cast<int>(p->c), nq64);
+    return TSP_OK;
 }
 
 // ===========================================================================

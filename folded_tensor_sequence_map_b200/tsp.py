@@ -45,6 +45,7 @@ EXPORTED = (
     "tsp_rmsnorm_backward_noalloc",
     "tsp_test_gemm",
     "tsp_test_buffer_offset",
+    "tsp_test_next_visible",
     "tsp_test_wait_timeout",
 )
 TSP_NUM_STAGES = 20
@@ -85,6 +86,8 @@ def _load() -> ctypes.CDLL:
     lib.tsp_test_gemm.restype = I
     lib.tsp_test_buffer_offset.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(SZ)]
     lib.tsp_test_buffer_offset.restype = I
+    lib.tsp_test_next_visible.argtypes = [P, I, I, ctypes.POINTER(I)]
+    lib.tsp_test_next_visible.restype = I
     lib.tsp_profile_enable.argtypes = [P, I]
     lib.tsp_profile_enable.restype = I
     lib.tsp_profile_read.argtypes = [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
@@ -281,6 +284,12 @@ def tsp_test_buffer_offset(plan: Plan, name: str) -> int:
     off = ctypes.c_size_t()
     _check(_lib.tsp_test_buffer_offset(plan.handle, name.encode(), ctypes.byref(off)), "tsp_test_buffer_offset")
     return off.value
+
+
+def tsp_test_next_visible(plan: Plan, start: int, kv0: int) -> int:
+    out = ctypes.c_int()
+    _check(_lib.tsp_test_next_visible(plan.handle, start, kv0, ctypes.byref(out)), "tsp_test_next_visible")
+    return out.value
 
 
 def tsp_test_wait_timeout(plan: Plan, limit_cycles: int, result, stream=None) -> None:

@@ -36,6 +36,14 @@ tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A,
  * log2(e)/sqrt(dh)); rstd f32 [S].  TSP_ERR_INVALID_ARG for an unknown name. */
 tsp_status tsp_test_buffer_offset(tsp_plan_t plan, const char *name, size_t *offset);
 
+/* Host evaluation of the rule the dK/dV kernel uses to walk the 64-row query
+ * steps that can see a key: writes to *out the first local step q >= from
+ * (step q = local rows [64 q, 64 q + 64)) whose largest global position is at
+ * least kv0, or S / 64 when there is none.  It is the same function the
+ * kernel runs, so a test can check it against a scan of the zigzag map.
+ * TSP_ERR_INVALID_ARG for from outside [0, S / 64] or kv0 outside [0, S). */
+tsp_status tsp_test_next_visible(tsp_plan_t plan, int from, int kv0, int *out);
+
 /* Self-test of the bounded device-side wait used by every kernel: launches one
  * CTA that waits on an mbarrier nothing ever completes, with a limit of
  * `limit_cycles` SM cycles.  The wait gives up, the kernel writes 0 to

@@ -44,6 +44,31 @@ def test_zigzag_and_schedules_match_oracle(h, H, F, S, D):
         assert np.array_equal(T.tsp_shard_schedule(p, phase), O.shard_schedule(D, phase))
 
 
+@pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
+                                       (256, 4, 1024, 2048, 1), (4096, 32, 16384, 131072, 8)])
+def test_next_visible_matches_zigzag_scan(h, H, F, S, D):
+    """The dK/dV kernel's walk over query steps: the first 64-row local step at
+    or after `start` holding a row whose position (oracle zigzag map) is at
+    least kv0, found here by scanning every step."""
+    p = T.tsp_plan(h, H, F, S, D)
+    nq = S // 64
+    step_max = O.zigzag_map(S, D).ravel().reshape(nq, 64).max(axis=1)
+    rng = np.random.default_rng(S + D)
+    kv0s = np.unique(np.concatenate([[0, 1, 63, 64, 127, S // 2, S - 128, S - 64, S - 1],
+                                     rng.integers(0, S, 60), np.arange(0, S, max(128, S // 256))]))
+    for kv0 in kv0s:
+        vis = np.nonzero(step_max >= kv0)[0]
+        starts = np.unique(np.concatenate([[0, 1, nq - 1, nq], rng.integers(0, nq + 1, 10), vis[:2], vis[-2:],
+                                           np.maximum(vis[:2] - 1, 0)]).astype(int))
+        for st in starts:
+            later = vis[vis >= st]
+            want = int(later[0]) if len(later) else nq
+            assert T.tsp_test_next_visible(p, int(st), int(kv0)) == want, (S, D, kv0, st)
+    for bad in ((-1, 0), (nq + 1, 0), (0, -1), (0, S)):
+        with pytest.raises(T.TSPError):
+            T.tsp_test_next_visible(p, *bad)
+
+
 def test_flops_formula_matches_workload_figures():
     # algorithmic FLOPs of the forward: 24 S h^2 + 2 h S (S+1) for the 7B shape
     for S, expect in ((256, None), (8192, 3.848e12), (32768, 2.199e13), (131072, 1.935e14)):
