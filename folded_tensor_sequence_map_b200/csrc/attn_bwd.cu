@@ -25,8 +25,6 @@
 namespace tsp {
 namespace {
 
-constexpr int kBwdThreads = 192;
-
 __device__ __forceinline__ float ex2b(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -54,7 +52,6 @@ struct BCfg {
     static constexpr int TILE_BYTES = 128 * DH * 2;
     static constexpr int ATOM_BYTES = 128 * SWB;
     static constexpr uint32_t LAYOUT = SWB == 128 ? kSwizzle128 : (SWB == 64 ? kSwizzle64 : kSwizzle32);
-    static constexpr int SQ_BYTES = 128 * 128 * 2;  // a 128 x 128 bf16 operand (P^T, dS^T or dS)
 };
 
 template <int DH>
@@ -63,31 +60,6 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
     const int col = kk * 16;
     return sdesc(base + (col / C::ATOM_COLS) * C::ATOM_BYTES + (col % C::ATOM_COLS) * 2, 16, 8 * C::SWB, C::LAYOUT);
 }
-template <int DH>
-__device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk) {
-    using C = BCfg<DH>;
-    return sdesc(base + kk * 16 * C::SWB, C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
-}
-__device__ __forceinline__ uint64_t sq_desc(uint32_t base, int kk) {
-    const int col = kk * 16;
-    return sdesc(base + (col / 64) * 16384 + (col % 64) * 2, 16, 1024, kSwizzle128);
-}
-// Write 32 consecutive bf16 values (columns c0..c0+31 of a 128-column row) of
-// a K-major 128B-swizzled 128x128 operand.
-__device__ __forceinline__ void store_row32(uint8_t *tile, int row, int c0, const float (&v)[32]) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int col = c0 + q * 8;
-        uint4 w;
-        w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-        w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-        w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-        w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-        const int atom = col >> 6, chunk = ((col & 63) >> 3) ^ (row & 7);
-        *reinterpret_cast<uint4 *>(tile + atom * 16384 + row * 128 + chunk * 16) = w;
-    }
-}
-
 template <int DH>
 CUtensorMapSwizzle swz_of() {
     return BCfg<DH>::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B

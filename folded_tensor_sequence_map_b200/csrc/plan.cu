@@ -432,10 +432,9 @@ TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g
     auto *rstd2 = reinterpret_cast<float *>(base + l.rstd2);
     void *b = base + l.b, *u = base + l.u, *g = base + l.g;
 
-    cudaError_t e;
 #define TSP_STAGE(id, nk, call)                                                  \
     do {                                                                         \
-        if ((e = stage(p, id, nk, s, [&] { return (call); })) != cudaSuccess) \
+        if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
             return TSP_ERR_CUDA;                                                 \
     } while (0)
     TSP_STAGE(0, 1, launch_rmsnorm_fwd(x, nullptr, g1, a, rstd1, S, h, s));
@@ -514,10 +513,9 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     float *delta = reinterpret_cast<float *>(w + l.delta);
     float *da = reinterpret_cast<float *>(w + l.da);
     float *dgp = reinterpret_cast<float *>(w + l.dgp);
-    cudaError_t e;
 #define TSP_STAGE(id, nk, call)                                                  \
     do {                                                                         \
-        if ((e = stage(p, id, nk, s, [&] { return (call); })) != cudaSuccess) \
+        if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
             return TSP_ERR_CUDA;                                                 \
     } while (0)
     // MLP ring backward: dU = (dY W2) * GELU'(U); dW2 = dY^T G; dW1 = dU^T b; db = dU W1 (ring K order)
