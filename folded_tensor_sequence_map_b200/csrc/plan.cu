@@ -411,22 +411,20 @@ TSP_API tsp_status tsp_sync_status(tsp_plan_t p, void *stream) {
     return check_pending_error(p);
 }
 
-TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g1, const void *wqkv, const void *wo,
-                                     const float *g2, const void *w1, const void *w2, void *y, void *saved, void *ws,
-                                     void *stream) {
-    if (!p || !x || !g1 || !wqkv || !wo || !g2 || !w1 || !w2 || !y || !ws) return TSP_ERR_INVALID_ARG;
-    for (const void *q : {x, (const void *)g1, wqkv, wo, (const void *)g2, w1, w2, (const void *)y, (const void *)ws})
-        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
-    if (saved && !aligned16(saved)) return TSP_ERR_ALIGNMENT;
-    tsp_status st = ensure_device(p);
-    if (st != TSP_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+namespace {
+
+// The forward's launch sequence.  Intermediates live in `base` (the saved
+// buffer, or the workspace of an inference call) with the layout of
+// layout_of(); K and V, in global row order, go to `k` and `v`, which are
+// base's K/V slots unless a caller-owned cache takes their place.
+tsp_status forward_impl(tsp_plan_s *p, const void *x, const float *g1, const void *wqkv, const void *wo,
+                        const float *g2, const void *w1, const void *w2, void *y, uint8_t *base, void *k, void *v,
+                        cudaStream_t s) {
     const Layout l = layout_of(p);
-    uint8_t *base = static_cast<uint8_t *>(saved ? saved : ws);
     const int S = static_cast<int>(p->S), h = p->h, F = p->F, L = static_cast<int>(p->L);
     const DevErr err = dev_err(p);
     auto *rstd1 = reinterpret_cast<float *>(base + l.rstd1);
-    void *a = base + l.a, *q = base + l.q, *k = base + l.k, *v = base + l.v, *o = base + l.o;
+    void *a = base + l.a, *q = base + l.q, *o = base + l.o;
     auto *lse = reinterpret_cast<float *>(base + l.lse);
     auto *yres = reinterpret_cast<float *>(base + l.y);
     auto *rstd2 = reinterpret_cast<float *>(base + l.rstd2);
@@ -479,6 +477,37 @@ TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g
     TSP_STAGE(6, 1, launch_gemm(g2d, err, p->num_sms, s));
 #undef TSP_STAGE
     return TSP_OK;
+}
+
+}  // namespace
+
+TSP_API tsp_status tsp_layer_forward(tsp_plan_t p, const void *x, const float *g1, const void *wqkv, const void *wo,
+                                     const float *g2, const void *w1, const void *w2, void *y, void *saved, void *ws,
+                                     void *stream) {
+    if (!p || !x || !g1 || !wqkv || !wo || !g2 || !w1 || !w2 || !y || !ws) return TSP_ERR_INVALID_ARG;
+    for (const void *q : {x, (const void *)g1, wqkv, wo, (const void *)g2, w1, w2, (const void *)y, (const void *)ws})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    if (saved && !aligned16(saved)) return TSP_ERR_ALIGNMENT;
+    tsp_status st = ensure_device(p);
+    if (st != TSP_OK) return st;
+    const Layout l = layout_of(p);
+    uint8_t *base = static_cast<uint8_t *>(saved ? saved : ws);
+    return forward_impl(p, x, g1, wqkv, wo, g2, w1, w2, y, base, base + l.k, base + l.v,
+                        static_cast<cudaStream_t>(stream));
+}
+
+TSP_API tsp_status tsp_layer_prefill(tsp_plan_t p, const void *x, const float *g1, const void *wqkv, const void *wo,
+                                     const float *g2, const void *w1, const void *w2, void *y, void *k_cache,
+                                     void *v_cache, void *ws, void *stream) {
+    if (!p || !x || !g1 || !wqkv || !wo || !g2 || !w1 || !w2 || !y || !k_cache || !v_cache || !ws)
+        return TSP_ERR_INVALID_ARG;
+    for (const void *q : {x, (const void *)g1, wqkv, wo, (const void *)g2, w1, w2, (const void *)y, (const void *)k_cache,
+                          (const void *)v_cache, (const void *)ws})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    tsp_status st = ensure_device(p);
+    if (st != TSP_OK) return st;
+    return forward_impl(p, x, g1, wqkv, wo, g2, w1, w2, y, static_cast<uint8_t *>(ws), k_cache, v_cache,
+                        static_cast<cudaStream_t>(stream));
 }
 
 TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *x, const float *g1, const void *wqkv,

@@ -35,6 +35,7 @@ EXPORTED = (
     "tsp_shard_schedule",
     "tsp_workspace_size",
     "tsp_layer_forward",
+    "tsp_layer_prefill",
     "tsp_layer_backward",
     "tsp_sync_status",
     "tsp_status_string",
@@ -74,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.tsp_workspace_size.restype = I
     lib.tsp_layer_forward.argtypes = [P] + [V] * 11
     lib.tsp_layer_forward.restype = I
+    lib.tsp_layer_prefill.argtypes = [P] + [V] * 12
+    lib.tsp_layer_prefill.restype = I
     lib.tsp_layer_backward.argtypes = [P] + [V] * 18
     lib.tsp_layer_backward.restype = I
     lib.tsp_sync_status.argtypes = [P, V]
@@ -207,6 +210,28 @@ def tsp_layer_forward(plan: Plan, x, g1, wqkv, wo, g2, w1, w2, y, saved, ws, str
         _stream(stream),
     ]
     _check(_lib.tsp_layer_forward(plan.handle, *args), "tsp_layer_forward")
+
+
+def tsp_layer_prefill(plan: Plan, x, g1, wqkv, wo, g2, w1, w2, y, k_cache, v_cache, ws, stream=None) -> None:
+    import torch
+
+    h, F, S = plan.h, plan.ffn, plan.S
+    bf, f32 = torch.bfloat16, torch.float32
+    args = [
+        _ptr(x, "x", bf, (S, h)),
+        _ptr(g1, "g1", f32, (h,)),
+        _ptr(wqkv, "wqkv", bf, (3 * h, h)),
+        _ptr(wo, "wo", bf, (h, h)),
+        _ptr(g2, "g2", f32, (h,)),
+        _ptr(w1, "w1", bf, (F, h)),
+        _ptr(w2, "w2", bf, (h, F)),
+        _ptr(y, "y", bf, (S, h)),
+        _ptr(k_cache, "k_cache", bf, (S, h)),
+        _ptr(v_cache, "v_cache", bf, (S, h)),
+        _ptr(ws, "ws"),
+        _stream(stream),
+    ]
+    _check(_lib.tsp_layer_prefill(plan.handle, *args), "tsp_layer_prefill")
 
 
 def tsp_layer_backward(plan: Plan, dy, x, g1, wqkv, wo, g2, w1, w2, saved, ws, dx, dg1, dwqkv, dwo, dg2, dw1, dw2,

@@ -118,6 +118,27 @@ tsp_status tsp_layer_forward(tsp_plan_t plan, const void *x, const float *g1, co
                              const void *wo, const float *g2, const void *w1, const void *w2,
                              void *y, void *saved, void *ws, void *stream);
 
+/* Inference prefill: the forward above without training state, keeping the
+ * layer's keys and values as a cache for later decoding.  The review page
+ * "Zyphra TSP: 2.6x Faster AI Training Review" (What's New) extends the
+ * method's benefits to inference; this is the forward run for that use.
+ * Device pointers:
+ *   x, g1, wqkv, wo, g2, w1, w2, y  as for tsp_layer_forward
+ *   k_cache, v_cache  bf16 [S][h] each (outputs, owned by the caller): the
+ *       keys and values of all S tokens in GLOBAL position order (row p =
+ *       token at position p, the all-gathered layout), head n in columns
+ *       [n*dh, (n+1)*dh).  The attention of this call reads them there.
+ *   ws  the ws_bytes that tsp_workspace_size(plan, 0, ...) reports (scratch)
+ * Same kernels and arithmetic as tsp_layer_forward with saved = NULL, so y is
+ * identical to that call's output and the caches hold exactly the K and V it
+ * computes.  Errors: TSP_ERR_INVALID_ARG for a NULL pointer,
+ * TSP_ERR_ALIGNMENT unless every pointer is 16-byte aligned (both checked
+ * before anything is enqueued), TSP_ERR_UNSUPPORTED off sm_100, TSP_ERR_CUDA
+ * for a failed launch. */
+tsp_status tsp_layer_prefill(tsp_plan_t plan, const void *x, const float *g1, const void *wqkv,
+                             const void *wo, const float *g2, const void *w1, const void *w2,
+                             void *y, void *k_cache, void *v_cache, void *ws, void *stream);
+
 /* Backward of the folded layer (exact gradient of the forward; the pages give
  * no backward schedule, so it runs the forward's collectives in reverse:
  * weight-gradient pieces are summed over ranks in rank order, and key/value

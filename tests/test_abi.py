@@ -69,6 +69,24 @@ def test_next_visible_matches_zigzag_scan(h, H, F, S, D):
             T.tsp_test_next_visible(p, *bad)
 
 
+def test_prefill_checks_arguments_before_enqueueing():
+    """tsp_layer_prefill refuses a NULL or misaligned pointer before it touches
+    the device (the addresses below are never dereferenced)."""
+    p = T.tsp_plan(128, 4, 512, 256, 2)
+    good = [0x10000 * (i + 1) for i in range(11)]
+    for i in range(11):
+        args = list(good)
+        args[i] = None
+        with pytest.raises(T.TSPError) as e:
+            T.tsp_layer_prefill(p, *args, stream=0)
+        assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_INVALID_ARG"
+        args = list(good)
+        args[i] += 8
+        with pytest.raises(T.TSPError) as e:
+            T.tsp_layer_prefill(p, *args, stream=0)
+        assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_ALIGNMENT"
+
+
 def test_flops_formula_matches_workload_figures():
     # algorithmic FLOPs of the forward: 24 S h^2 + 2 h S (S+1) for the 7B shape
     for S, expect in ((256, None), (8192, 3.848e12), (32768, 2.199e13), (131072, 1.935e14)):
