@@ -510,6 +510,46 @@ TSP_API tsp_status tsp_layer_prefill(tsp_plan_t p, const void *x, const float *g
                         static_cast<cudaStream_t>(stream));
 }
 
+TSP_API tsp_status tsp_ring_mlp_workspace_size(tsp_plan_t p, size_t *ws_bytes) {
+    if (!p || !ws_bytes) return TSP_ERR_INVALID_ARG;
+    *ws_bytes = 2 * up(static_cast<size_t>(p->S) * static_cast<size_t>(p->F) * 2);  // U and G, bf16 [S][F]
+    return TSP_OK;
+}
+
+// The layer's W1 + GELU and W2 ring steps, launched exactly as the forward
+// launches them, on caller buffers.
+TSP_API tsp_status tsp_ring_mlp_forward(tsp_plan_t p, const void *b, const void *w1, const void *w2, const float *resid,
+                                        void *out, void *ws, void *stream) {
+    if (!p || !b || !w1 || !w2 || !resid || !out || !ws) return TSP_ERR_INVALID_ARG;
+    for (const void *q : {b, w1, w2, (const void *)resid, (const void *)out, (const void *)ws})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    tsp_status st = ensure_device(p);
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int S = static_cast<int>(p->S), h = p->h, F = p->F, L = static_cast<int>(p->L);
+    const DevErr err = dev_err(p);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    void *u = base, *g = base + up(static_cast<size_t>(S) * F * 2);
+#define TSP_STAGE(id, nk, call)                                                  \
+    do {                                                                         \
+        if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
+            return TSP_ERR_CUDA;                                                 \
+    } while (0)
+    GemmDesc g1d = gemm(b, h, false, w1, h, false, S, F, h, EPI_GELU, u, F);
+    g1d.out2 = g;
+    g1d.ldo2 = F;
+    TSP_STAGE(5, 1, launch_gemm(g1d, err, p->num_sms, s));
+    // K loop over FFN shards in ring order (r + t) mod D for rank r's rows, + residual
+    GemmDesc g2d = gemm(g, F, false, w2, F, false, S, h, F, EPI_RESID_BF16, out, h);
+    g2d.aux = resid;
+    g2d.ldaux = h;
+    g2d.ring_rows = L;
+    g2d.ring_kblocks = (F / p->D) / 64;
+    TSP_STAGE(6, 1, launch_gemm(g2d, err, p->num_sms, s));
+#undef TSP_STAGE
+    return TSP_OK;
+}
+
 TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *x, const float *g1, const void *wqkv,
                                       const void *wo, const float *g2, const void *w1, const void *w2,
                                       const void *saved, void *ws, void *dx, float *dg1, float *dwqkv, float *dwo,

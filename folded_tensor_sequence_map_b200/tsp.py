@@ -36,6 +36,8 @@ EXPORTED = (
     "tsp_workspace_size",
     "tsp_layer_forward",
     "tsp_layer_prefill",
+    "tsp_ring_mlp_workspace_size",
+    "tsp_ring_mlp_forward",
     "tsp_layer_backward",
     "tsp_sync_status",
     "tsp_status_string",
@@ -77,6 +79,10 @@ def _load() -> ctypes.CDLL:
     lib.tsp_layer_forward.restype = I
     lib.tsp_layer_prefill.argtypes = [P] + [V] * 12
     lib.tsp_layer_prefill.restype = I
+    lib.tsp_ring_mlp_workspace_size.argtypes = [P, ctypes.POINTER(SZ)]
+    lib.tsp_ring_mlp_workspace_size.restype = I
+    lib.tsp_ring_mlp_forward.argtypes = [P] + [V] * 7
+    lib.tsp_ring_mlp_forward.restype = I
     lib.tsp_layer_backward.argtypes = [P] + [V] * 18
     lib.tsp_layer_backward.restype = I
     lib.tsp_sync_status.argtypes = [P, V]
@@ -232,6 +238,29 @@ def tsp_layer_prefill(plan: Plan, x, g1, wqkv, wo, g2, w1, w2, y, k_cache, v_cac
         _stream(stream),
     ]
     _check(_lib.tsp_layer_prefill(plan.handle, *args), "tsp_layer_prefill")
+
+
+def tsp_ring_mlp_workspace_size(plan: Plan) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.tsp_ring_mlp_workspace_size(plan.handle, ctypes.byref(n)), "tsp_ring_mlp_workspace_size")
+    return n.value
+
+
+def tsp_ring_mlp_forward(plan: Plan, b, w1, w2, resid, out, ws, stream=None) -> None:
+    import torch
+
+    h, F, S = plan.h, plan.ffn, plan.S
+    bf, f32 = torch.bfloat16, torch.float32
+    args = [
+        _ptr(b, "b", bf, (S, h)),
+        _ptr(w1, "w1", bf, (F, h)),
+        _ptr(w2, "w2", bf, (h, F)),
+        _ptr(resid, "resid", f32, (S, h)),
+        _ptr(out, "out", bf, (S, h)),
+        _ptr(ws, "ws"),
+        _stream(stream),
+    ]
+    _check(_lib.tsp_ring_mlp_forward(plan.handle, *args), "tsp_ring_mlp_forward")
 
 
 def tsp_layer_backward(plan: Plan, dy, x, g1, wqkv, wo, g2, w1, w2, saved, ws, dx, dg1, dwqkv, dwo, dg2, dw1, dw2,

@@ -139,6 +139,27 @@ tsp_status tsp_layer_prefill(tsp_plan_t plan, const void *x, const float *g1, co
                              const void *wo, const float *g2, const void *w1, const void *w2,
                              void *y, void *k_cache, void *v_cache, void *ws, void *stream);
 
+/* The MLP alone, in the ring schedule with no all-reduce.  The zubnet.ai page
+ * "Zyphra TSP folds TP+SP onto one GPU axis, 2.6x throughput on 1,024
+ * MI300Xs" (paragraph 4) calls this part of the method worth taking on its
+ * own into an existing tensor-parallel setup; it is steps W1 + GELU and W2 of
+ * tsp_layer_forward on caller buffers.  For every virtual rank r (rows
+ * [r*L, (r+1)*L) of the rank-major layout):
+ *   out_r = resid_r + sum_{t=0}^{D-1} GELU_tanh(b_r W1[s_t]^T) W2[:, s_t]^T,
+ *   s_t = (r + t) mod D (FFN shard s_t = units [s_t*F/D, (s_t+1)*F/D)),
+ * the partial sums staying in the rank's fp32 accumulator.  Device pointers:
+ *   b      bf16 [S][h], rank-major (input, the normalised activations)
+ *   w1     bf16 [F][h]; w2 bf16 [h][F] (inputs)
+ *   resid  float32 [S][h], rank-major (input; pass zeros for no residual)
+ *   out    bf16 [S][h], rank-major (output)
+ *   ws     tsp_ring_mlp_workspace_size bytes of scratch (holds U and G)
+ * Errors: TSP_ERR_INVALID_ARG for a NULL pointer, TSP_ERR_ALIGNMENT unless
+ * every pointer is 16-byte aligned (both before anything is enqueued),
+ * TSP_ERR_UNSUPPORTED off sm_100, TSP_ERR_CUDA for a failed launch. */
+tsp_status tsp_ring_mlp_workspace_size(tsp_plan_t plan, size_t *ws_bytes);
+tsp_status tsp_ring_mlp_forward(tsp_plan_t plan, const void *b, const void *w1, const void *w2,
+                                const float *resid, void *out, void *ws, void *stream);
+
 /* Backward of the folded layer (exact gradient of the forward; the pages give
  * no backward schedule, so it runs the forward's collectives in reverse:
  * weight-gradient pieces are summed over ranks in rank order, and key/value

@@ -380,6 +380,25 @@ def tsp_layer_forward(x_local, w, H, D, eps=EPS):
     return np.concatenate(z, axis=0), cache
 
 
+def tsp_ring_mlp(b_local, w1, w2, resid_local, D):
+    """[Z2], [Z4]: the MLP in its ring schedule on its own.  b_local and
+    resid_local are rank-major [S][h] (rank r holds rows r*L .. (r+1)*L - 1);
+    at step t rank r applies FFN shard (r+t) mod D to its own rows, and the
+    partial sums stay in that rank's accumulator, which is added to the
+    residual at the end (no sum across ranks)."""
+    b_local = np.asarray(b_local, dtype=np.float64)
+    S, h = b_local.shape
+    F = w1.shape[0]
+    L = S // D
+    ring = shard_schedule(D, 1)
+    accs = [np.zeros((L, h)) for _ in range(D)]
+    for t in range(D):
+        for r in range(D):
+            units = ffn_units(int(ring[t, r]), F, D)
+            accs[r] += gelu_tanh(b_local[r * L:(r + 1) * L] @ w1[units].T) @ w2[:, units].T
+    return np.asarray(resid_local, dtype=np.float64) + np.concatenate(accs, axis=0)
+
+
 def tsp_layer_backward(dz_local, w, cache):
     """Exact gradient of ``tsp_layer_forward``, rank by rank.
 

@@ -87,6 +87,25 @@ def test_prefill_checks_arguments_before_enqueueing():
         assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_ALIGNMENT"
 
 
+def test_ring_mlp_workspace_and_argument_checks():
+    """Scratch for U and G (bf16 [S][F] each, 256-byte aligned pieces); NULL or
+    misaligned pointers are refused before anything is enqueued."""
+    p = T.tsp_plan(128, 4, 512, 256, 2)
+    assert T.tsp_ring_mlp_workspace_size(p) == 2 * 256 * 512 * 2
+    good = [0x10000 * (i + 1) for i in range(6)]
+    for i in range(6):
+        args = list(good)
+        args[i] = None
+        with pytest.raises(T.TSPError) as e:
+            T.tsp_ring_mlp_forward(p, *args, stream=0)
+        assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_INVALID_ARG"
+        args = list(good)
+        args[i] += 4
+        with pytest.raises(T.TSPError) as e:
+            T.tsp_ring_mlp_forward(p, *args, stream=0)
+        assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_ALIGNMENT"
+
+
 def test_flops_formula_matches_workload_figures():
     # algorithmic FLOPs of the forward: 24 S h^2 + 2 h S (S+1) for the 7B shape
     for S, expect in ((256, None), (8192, 3.848e12), (32768, 2.199e13), (131072, 1.935e14)):

@@ -97,3 +97,37 @@ def test_planted_zigzag_mistake_is_caught(monkeypatch):
     pairs = T.causal_pairs_per_rank(zig)
     c = 64 // 8
     assert not np.all(pairs == c * c * 7 + c * (c + 1))
+
+
+def _ring_mlp_error():
+    """True when the ring-MLP pin fails."""
+    from tests.test_oracle_pins import test_ring_mlp_is_the_whole_mlp
+    try:
+        for D in (2, 4):
+            test_ring_mlp_is_the_whole_mlp(D)
+    except AssertionError:
+        return True
+    return False
+
+
+@pytest.mark.parametrize("mistake", ["shard_repeats", "rows_of_next_rank"])
+def test_planted_ring_mlp_mistake_is_caught(monkeypatch, mistake):
+    if mistake == "shard_repeats":
+        # every step applies the rank's own shard again instead of rotating
+        monkeypatch.setattr(T, "shard_schedule",
+                            lambda D, phase: np.array([[r for r in range(D)] for _ in range(D)]))
+    else:
+        # each rank's partial sums are built from the next rank's rows
+        orig = T.tsp_ring_mlp
+
+        def shifted(b, w1, w2, resid, D):
+            L = b.shape[0] // D
+            return orig(np.roll(b, -L, axis=0), w1, w2, resid, D)
+        monkeypatch.setattr(T, "tsp_ring_mlp", shifted)
+        import oracle as O
+        monkeypatch.setattr(O, "tsp_ring_mlp", shifted)
+    assert _ring_mlp_error()
+
+
+def test_unmutated_ring_mlp_passes():
+    assert not _ring_mlp_error()

@@ -343,3 +343,34 @@ def test_ring_partial_sums_stay_on_rank():
     z2, _ = O.tsp_layer_forward(x2, w, H, D)
     assert np.array_equal(z1[: S // 2], z2[: S // 2])
     assert not np.allclose(z1[S // 2:], z2[S // 2:])
+
+
+# ---------------------------------------------------------------------------
+# ring MLP on its own
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D", [1, 2, 4, 8])
+def test_ring_mlp_is_the_whole_mlp(D):
+    """The ring's per-rank shard sums add up to the undivided MLP
+    resid + GELU(b W1^T) W2^T on every row: a missing, repeated or misplaced
+    shard, or a row block paired with the wrong rank, breaks the equality."""
+    rng = np.random.default_rng(70 + D)
+    S, h, F_ = 32 * D, 24, 8 * D
+    b = rng.standard_normal((S, h))
+    resid = rng.standard_normal((S, h))
+    w1 = rng.standard_normal((F_, h)) * 0.3
+    w2 = rng.standard_normal((h, F_)) * 0.3
+    full = resid + O.gelu_tanh(b @ w1.T) @ w2.T
+    assert _relerr(O.tsp_ring_mlp(b, w1, w2, resid, D), full) < 1e-12
+
+
+def test_ring_mlp_matches_the_layer_oracle():
+    """Given the layer's own normalised activations b and residual stream y,
+    the standalone ring MLP reproduces the layer oracle's output z."""
+    rng = np.random.default_rng(77)
+    S, h, H, F_, D = 64, 16, 4, 32, 4
+    x, w = _rand_layer(rng, S, h, H, F_)
+    zl, cache = O.tsp_layer_forward(x[O.zigzag_map(S, D).ravel()], w, H, D)
+    b = np.concatenate(cache["b"], axis=0)
+    y = np.concatenate(cache["y"], axis=0)
+    assert _relerr(O.tsp_ring_mlp(b, w["w1"], w["w2"], y, D), zl) < 1e-12
