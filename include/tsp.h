@@ -67,7 +67,9 @@ typedef enum {
  * FFN units split D ways): TSP_ERR_INDIVISIBLE if S % (2D), heads % D,
  * ffn % D or h % heads is non-zero.  TSP_ERR_UNSUPPORTED when the shape is
  * outside what the kernels tile: dh not in {32, 64, 128}, h % 128, S % 256,
- * (S/D) % 128, ffn % 128 or (ffn/D) % 64 non-zero.  Needs no GPU.
+ * (S/D) % 128, ffn % 128 or (ffn/D) % 64 non-zero; and when it is too large
+ * for their 32-bit thread numbering: S > 2^28 or heads * S > 67,108,856
+ * (S up to about 2.1 million tokens at 32 heads).  Needs no GPU.
  * On success *out receives a new plan. */
 tsp_status tsp_plan(int h, int heads, int ffn, int64_t S, int D, tsp_plan_t *out);
 

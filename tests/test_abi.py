@@ -149,6 +149,20 @@ def test_plan_rejects_bad_shapes(args, status):
     assert T.tsp_status_string(e.value.status) == status
 
 
+def test_plan_size_limit_of_the_thread_numbering():
+    """heads * S may not exceed 67,108,856 (one warp per token and head,
+    numbered with 32-bit integers); the largest S below it is accepted."""
+    ok = T.tsp_plan(128, 4, 512, (1 << 24) - 256, 2)
+    assert ok.S == (1 << 24) - 256
+    del ok
+    with pytest.raises(T.TSPError) as e:
+        T.tsp_plan(128, 4, 512, 1 << 24, 2)
+    assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_UNSUPPORTED"
+    with pytest.raises(T.TSPError) as e:
+        T.tsp_plan(4096, 32, 16384, 1 << 21, 8)
+    assert T.STATUS_NAMES[e.value.status] == "TSP_ERR_UNSUPPORTED"
+
+
 def test_bad_phase_is_rejected():
     p = T.tsp_plan(128, 4, 512, 256, 2)
     with pytest.raises(T.TSPError):
