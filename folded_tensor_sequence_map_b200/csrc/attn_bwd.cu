@@ -119,6 +119,10 @@ struct KvCfg {
     static constexpr int OFF_VEC = OFF_DO + QST * QTILE;
     static constexpr int OFF_BAR = OFF_VEC + QST * VEC_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static_assert(SMEM <= kMaxDynSmem, "dK/dV tiles exceed the shared-memory limit");
+    // kv_full/empty, q_full/empty[QST], s_full[2], p_full[2], acc_full, drain + TMEM slot + abort flag
+    static_assert(8 * (2 * QST + 8) + 8 <= 256, "dK/dV barriers exceed their slot");
+    static_assert(384 + DH <= 512, "dK/dV TMEM columns: S^T/dP^T buffers 0-255, dV 256, dK 384");
 };
 
 // K-major descriptor of a [64 rows][DH] sub-tile for K step kk (16 columns of DH).
@@ -472,6 +476,10 @@ struct Dq2Cfg {
     static constexpr int OFF_V = OFF_K + KST * KTILE;
     static constexpr int OFF_BAR = OFF_V + KST * KTILE;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static_assert(SMEM <= kMaxDynSmem, "dQ tiles exceed the shared-memory limit");
+    // q_full/empty, k_full/empty[KST], s_full[2], p_full[2], acc_full, drain + TMEM slot + abort flag
+    static_assert(8 * (2 * KST + 8) + 8 <= 256, "dQ barriers exceed their slot");
+    static_assert(256 + DH <= 512, "dQ TMEM columns: S/dP buffers 0-255, dQ 256");
 };
 
 template <int DH>

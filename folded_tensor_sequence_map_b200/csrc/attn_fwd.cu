@@ -58,6 +58,11 @@ struct FwdCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static_assert(SMEM <= kMaxDynSmem, "forward tiles exceed the shared-memory limit");
+    // q_full/empty, k_full/empty[KST], v_full/empty[VST], s_full[2], p_full[2], o_done[2], drain
+    // + TMEM slot + abort flag
+    static_assert(8 * (2 * KST + 2 * VST + 9) + 8 <= 256, "forward barriers exceed their slot");
+    static_assert(384 + DH <= 512, "forward TMEM columns: S0 0, S1 128, O0 256, O1 384");
 };
 
 // K-major descriptor of a [128 rows][DH] bf16 tile for K step kk (16 columns).

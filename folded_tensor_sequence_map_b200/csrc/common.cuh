@@ -17,6 +17,9 @@ namespace tsp {
 // which every other wait of the CTA returns at once so the CTA can drain,
 // free its TMEM and exit.
 // ---------------------------------------------------------------------------
+// Largest dynamic shared memory a CTA may opt into on sm_100 (227 KB).
+constexpr int kMaxDynSmem = 232448;
+
 struct DevErr {
     unsigned int *word;       // global error word (plan-owned)
     long long wait_limit;     // cycles a single wait may spin

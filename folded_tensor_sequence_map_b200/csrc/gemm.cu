@@ -61,6 +61,9 @@ struct Cfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static_assert(SMEM <= kMaxDynSmem, "GEMM stages exceed the shared-memory limit");
+    // full/empty[STAGES], acc_full/empty[2], TMEM slot + abort flag, spare, drain
+    static_assert(8 * (2 * STAGES + 7) <= 256, "GEMM barriers exceed their slot");
 };
 
 __device__ __forceinline__ void tile_coords(int t, int mt, int nt, int &mb, int &nb) {
