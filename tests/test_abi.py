@@ -141,6 +141,15 @@ def test_workspace_sizes_cover_the_layout():
     ((128, 4, 512, 128, 1), "TSP_ERR_UNSUPPORTED"),     # S % 256
     ((128, 4, 512, 256, 4), "TSP_ERR_UNSUPPORTED"),     # S/D = 64 tokens per rank
     ((0, 4, 512, 256, 2), "TSP_ERR_INVALID_ARG"),
+    ((128, 4, 512, 0, 2), "TSP_ERR_INVALID_ARG"),      # no tokens
+    ((128, 4, 512, 256, 0), "TSP_ERR_INVALID_ARG"),    # no ranks
+    ((128, 0, 512, 256, 2), "TSP_ERR_INVALID_ARG"),
+    ((128, 4, 0, 256, 2), "TSP_ERR_INVALID_ARG"),
+    ((128, 4, 512, -256, 2), "TSP_ERR_INVALID_ARG"),
+    ((128, 4, 512, 256, -2), "TSP_ERR_INVALID_ARG"),
+    ((128, 4, 512, 384, 2), "TSP_ERR_UNSUPPORTED"),     # ragged: S % 256
+    ((128, 4, 448, 256, 2), "TSP_ERR_UNSUPPORTED"),     # ffn % 128
+    ((128, 4, 512, 768, 3), "TSP_ERR_INDIVISIBLE"),     # heads % D
 ])
 def test_plan_rejects_bad_shapes(args, status):
     with pytest.raises(T.TSPError) as e:
