@@ -155,31 +155,6 @@ __host__ __device__ constexpr uint32_t mndesc64_off(int kk) {
     return kk * 16 * BCfg<DH>::SWB;
 }
 
-// Visibility of 64-row query steps to a key tile, from the zigzag layout.
-struct StepVis {
-    int D, chunk, nq64;
-};
-__device__ __forceinline__ int next_visible(const StepVis &v, int from, int kv0) {
-    return zz_next_visible(from, kv0, v.D, v.chunk, v.nq64);
-}
-
-// Walks the query steps that can see a key tile, in ascending order.  Within
-// a zigzag chunk the visible steps form a suffix, so after a chunk's first
-// visible step every later step of that chunk is visible too: the closed form
-// runs once per chunk and a step costs one compare.
-struct StepWalk {
-    int q;        // current step; nq64 once the walk is over
-    int run_end;  // end (exclusive) of the chunk holding q
-    __device__ __forceinline__ void seek(const StepVis &v, int from, int kv0) {
-        q = next_visible(v, from, kv0);
-        const int spc = v.chunk >> 6;
-        run_end = q < v.nq64 ? (q / spc + 1) * spc : v.nq64;
-    }
-    __device__ __forceinline__ void next(const StepVis &v, int kv0) {
-        if (q + 1 < run_end) ++q;
-        else seek(v, q + 1, kv0);
-    }
-};
 struct KvParams {
     AttnBwdDesc d;
     const int *zig;

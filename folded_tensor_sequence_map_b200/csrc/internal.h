@@ -106,6 +106,30 @@ __host__ __device__ inline int zz_next_visible(int from, int kv0, int D, int chu
     return nq64;
 }
 
+// Visibility of 64-row query steps to a key tile, from the zigzag layout.
+struct StepVis {
+    int D, chunk, nq64;
+};
+
+// Walks the query steps that can see a key tile kv0, in ascending order.
+// Within a zigzag chunk the visible steps form a suffix, so after a chunk's
+// first visible step every later step of that chunk is visible too: the
+// closed form runs once per chunk and a step costs one compare.  Used by the
+// dK/dV kernel; host-callable so that tests can replay the walk.
+struct StepWalk {
+    int q;        // current step; nq64 once the walk is over
+    int run_end;  // end (exclusive) of the chunk holding q
+    __host__ __device__ inline void seek(const StepVis &v, int from, int kv0) {
+        q = zz_next_visible(from, kv0, v.D, v.chunk, v.nq64);
+        const int spc = v.chunk >> 6;
+        run_end = q < v.nq64 ? (q / spc + 1) * spc : v.nq64;
+    }
+    __host__ __device__ inline void next(const StepVis &v, int kv0) {
+        if (q + 1 < run_end) ++q;
+        else seek(v, q + 1, kv0);
+    }
+};
+
 struct AttnBwdDesc {
     int S, L, D, H, dh, chunk;
     const void *q, *k, *v, *o, *dout;  // q, o, dout local rows; k, v global rows

@@ -687,6 +687,18 @@ TSP_API tsp_status tsp_test_next_visible(tsp_plan_t p, int from, int kv0, int *o
     return TSP_OK;
 }
 
+TSP_API tsp_status tsp_test_step_walk(tsp_plan_t p, int kv0, int32_t *steps, int capacity, int *count) {
+    if (!p || !count || capacity < 0 || (capacity > 0 && !steps)) return TSP_ERR_INVALID_ARG;
+    if (kv0 < 0 || kv0 >= p->S) return TSP_ERR_INVALID_ARG;
+    const StepVis vis{p->D, static_cast<int>(p->c), static_cast<int>(p->S / 64)};
+    int n = 0;
+    StepWalk w;
+    for (w.seek(vis, 0, kv0); w.q < vis.nq64; w.next(vis, kv0), ++n)
+        if (n < capacity) steps[n] = w.q;
+    *count = n;
+    return n <= capacity ? TSP_OK : TSP_ERR_INVALID_ARG;
+}
+
 // ===========================================================================
 // Profiling (tsp.h)
 // ===========================================================================

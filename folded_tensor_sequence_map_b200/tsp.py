@@ -49,6 +49,7 @@ EXPORTED = (
     "tsp_test_gemm",
     "tsp_test_buffer_offset",
     "tsp_test_next_visible",
+    "tsp_test_step_walk",
     "tsp_test_wait_timeout",
 )
 TSP_NUM_STAGES = 20
@@ -97,6 +98,8 @@ def _load() -> ctypes.CDLL:
     lib.tsp_test_buffer_offset.restype = I
     lib.tsp_test_next_visible.argtypes = [P, I, I, ctypes.POINTER(I)]
     lib.tsp_test_next_visible.restype = I
+    lib.tsp_test_step_walk.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I, ctypes.POINTER(I)]
+    lib.tsp_test_step_walk.restype = I
     lib.tsp_profile_enable.argtypes = [P, I]
     lib.tsp_profile_enable.restype = I
     lib.tsp_profile_read.argtypes = [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
@@ -344,6 +347,15 @@ def tsp_test_next_visible(plan: Plan, start: int, kv0: int) -> int:
     out = ctypes.c_int()
     _check(_lib.tsp_test_next_visible(plan.handle, start, kv0, ctypes.byref(out)), "tsp_test_next_visible")
     return out.value
+
+
+def tsp_test_step_walk(plan: Plan, kv0: int) -> np.ndarray:
+    cap = plan.S // 64
+    out = np.zeros(cap, dtype=np.int32)
+    n = ctypes.c_int()
+    _check(_lib.tsp_test_step_walk(plan.handle, kv0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cap,
+                                   ctypes.byref(n)), "tsp_test_step_walk")
+    return out[:n.value].copy()
 
 
 def tsp_test_wait_timeout(plan: Plan, limit_cycles: int, result, stream=None) -> None:

@@ -44,6 +44,15 @@ tsp_status tsp_test_buffer_offset(tsp_plan_t plan, const char *name, size_t *off
  * TSP_ERR_INVALID_ARG for from outside [0, S / 64] or kv0 outside [0, S). */
 tsp_status tsp_test_next_visible(tsp_plan_t plan, int from, int kv0, int *out);
 
+/* Host replay of the walk the dK/dV kernel makes over the 64-row query steps
+ * that can see the key tile starting at position kv0: writes the visited
+ * steps, in the kernel's order, to steps[0 .. *count) (host memory, at most
+ * `capacity` entries; *count always receives the full length).  The same
+ * code as the kernel's, so a test can compare it with a scan of the zigzag
+ * map.  TSP_ERR_INVALID_ARG for kv0 outside [0, S), a NULL pointer, or a
+ * walk longer than `capacity`. */
+tsp_status tsp_test_step_walk(tsp_plan_t plan, int kv0, int32_t *steps, int capacity, int *count);
+
 /* Self-test of the bounded device-side wait used by every kernel: launches one
  * CTA that waits on an mbarrier nothing ever completes, with a limit of
  * `limit_cycles` SM cycles.  The wait gives up, the kernel writes 0 to

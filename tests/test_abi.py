@@ -69,6 +69,22 @@ def test_next_visible_matches_zigzag_scan(h, H, F, S, D):
             T.tsp_test_next_visible(p, *bad)
 
 
+@pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
+                                       (256, 4, 1024, 2048, 1), (4096, 32, 16384, 131072, 8)])
+def test_step_walk_visits_exactly_the_visible_steps(h, H, F, S, D):
+    """The dK/dV kernel's walk for a key tile at kv0 visits, in ascending
+    order and once each, exactly the 64-row local steps holding a row at a
+    position >= kv0 (oracle zigzag map)."""
+    p = T.tsp_plan(h, H, F, S, D)
+    step_max = O.zigzag_map(S, D).ravel().reshape(S // 64, 64).max(axis=1)
+    rng = np.random.default_rng(S * 3 + D)
+    tiles = np.unique(np.concatenate([[0, 1, S // 256, S // 128 - 1], rng.integers(0, S // 128, 24)]))
+    for kt in tiles:
+        kv0 = int(kt) * 128
+        want = np.nonzero(step_max >= kv0)[0]
+        assert np.array_equal(T.tsp_test_step_walk(p, kv0), want), (S, D, kv0)
+
+
 def test_prefill_checks_arguments_before_enqueueing():
     """tsp_layer_prefill refuses a NULL or misaligned pointer before it touches
     the device (the addresses below are never dereferenced)."""
