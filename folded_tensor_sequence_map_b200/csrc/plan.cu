@@ -112,20 +112,20 @@ EncodeFn get_encode() {
 
 tsp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA; }
 
-// Device tables: map, inverse map, per-query-tile max position and the work
-// orders of the attention kernels (head-major, longest item first per head).
-tsp_status ensure_device(tsp_plan_s *p) {
-    std::lock_guard<std::mutex> g(p->mu);
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return TSP_ERR_CUDA;
-    if (p->dev_ready) return dev == p->device ? TSP_OK : TSP_ERR_INVALID_ARG;
-    cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return TSP_ERR_CUDA;
-    if (prop.major != 10) return TSP_ERR_UNSUPPORTED;
-    if (!get_encode()) return TSP_ERR_CUDA;
+// Host copies of the kernels' tables: inverse map, largest position of each
+// 128-row local query tile, and the work orders of the attention kernels
+// (head-major, longest item first per head).  Needs no GPU.
+struct HostTables {
+    std::vector<int32_t> inv, qmax, forder, korder, qorder;
+};
+
+HostTables host_tables(const tsp_plan_s *p) {
+    HostTables t;
     const int64_t S = p->S;
     const int H = p->H;
-    std::vector<int32_t> inv(S), qmax(S / 128);
+    std::vector<int32_t> &inv = t.inv, &qmax = t.qmax;
+    inv.resize(S);
+    qmax.resize(S / 128);
     for (int64_t i = 0; i < S; ++i) inv[p->zig[i]] = static_cast<int32_t>(i);
     for (int64_t t = 0; t < S / 128; ++t) {
         int32_t m = 0;
@@ -145,7 +145,7 @@ tsp_status ensure_device(tsp_plan_s *p) {
         const int hx = x.first % H, hy = y.first % H;
         return hx != hy ? hx < hy : x.second > y.second;
     });
-    std::vector<int32_t> forder;
+    std::vector<int32_t> &forder = t.forder;
     for (auto &it : fitems) {
         forder.push_back(it.first);
         forder.push_back(it.second);
@@ -165,20 +165,35 @@ tsp_status ensure_device(tsp_plan_s *p) {
     };
     std::stable_sort(kitems.begin(), kitems.end(), by_cost);
     std::stable_sort(qitems.begin(), qitems.end(), by_cost);
-    std::vector<int32_t> korder, qorder;
+    std::vector<int32_t> &korder = t.korder, &qorder = t.qorder;
     for (auto &it : kitems) korder.push_back(it.first);
     for (auto &it : qitems) qorder.push_back(it.first);
+    return t;
+}
+
+// Device tables: map, inverse map, per-query-tile max position and the work
+// orders of the attention kernels (head-major, longest item first per head).
+tsp_status ensure_device(tsp_plan_s *p) {
+    std::lock_guard<std::mutex> g(p->mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TSP_ERR_CUDA;
+    if (p->dev_ready) return dev == p->device ? TSP_OK : TSP_ERR_INVALID_ARG;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return TSP_ERR_CUDA;
+    if (prop.major != 10) return TSP_ERR_UNSUPPORTED;
+    if (!get_encode()) return TSP_ERR_CUDA;
+    const HostTables t = host_tables(p);
 
     auto upload = [](int32_t **dst, const std::vector<int32_t> &v) {
         if (cudaMalloc(dst, v.size() * 4) != cudaSuccess) return false;
         return cudaMemcpy(*dst, v.data(), v.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess;
     };
-    if (!upload(&p->d_zig, p->zig) || !upload(&p->d_inv, inv) || !upload(&p->d_qmax, qmax) ||
-        !upload(&p->d_fwd_order, forder) || !upload(&p->d_kv_order, korder) || !upload(&p->d_q_order, qorder))
+    if (!upload(&p->d_zig, p->zig) || !upload(&p->d_inv, t.inv) || !upload(&p->d_qmax, t.qmax) ||
+        !upload(&p->d_fwd_order, t.forder) || !upload(&p->d_kv_order, t.korder) || !upload(&p->d_q_order, t.qorder))
         return TSP_ERR_CUDA;
     if (cudaMalloc(&p->d_err, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
     if (cudaMemset(p->d_err, 0, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
-    p->fwd_items = static_cast<int>(fitems.size());
+    p->fwd_items = static_cast<int>(t.forder.size() / 2);
     p->num_sms = prop.multiProcessorCount;
     // A single device-side wait may spin for about 2 s at the boost clock.
     p->wait_limit = 4000000000LL;
@@ -684,6 +699,24 @@ TSP_API tsp_status tsp_test_next_visible(tsp_plan_t p, int from, int kv0, int *o
     const int nq64 = static_cast<int>(p->S / 64);
     if (from < 0 || from > nq64 || kv0 < 0 || kv0 >= p->S) return TSP_ERR_INVALID_ARG;
     *out = zz_next_visible(from, kv0, p->D, static_cast<int>(p->c), nq64);
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_test_tables(tsp_plan_t p, int which, int32_t *out, int64_t capacity, int64_t *count) {
+    if (!p || !count || capacity < 0 || (capacity > 0 && !out)) return TSP_ERR_INVALID_ARG;
+    const HostTables t = host_tables(p);
+    const std::vector<int32_t> *v = nullptr;
+    switch (which) {
+        case 0: v = &t.inv; break;
+        case 1: v = &t.qmax; break;
+        case 2: v = &t.forder; break;
+        case 3: v = &t.korder; break;
+        case 4: v = &t.qorder; break;
+        default: return TSP_ERR_INVALID_ARG;
+    }
+    *count = static_cast<int64_t>(v->size());
+    if (*count > capacity) return TSP_ERR_INVALID_ARG;
+    std::copy(v->begin(), v->end(), out);
     return TSP_OK;
 }
 

@@ -50,6 +50,7 @@ EXPORTED = (
     "tsp_test_buffer_offset",
     "tsp_test_next_visible",
     "tsp_test_step_walk",
+    "tsp_test_tables",
     "tsp_test_wait_timeout",
 )
 TSP_NUM_STAGES = 20
@@ -100,6 +101,8 @@ def _load() -> ctypes.CDLL:
     lib.tsp_test_next_visible.restype = I
     lib.tsp_test_step_walk.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I, ctypes.POINTER(I)]
     lib.tsp_test_step_walk.restype = I
+    lib.tsp_test_tables.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I64, ctypes.POINTER(I64)]
+    lib.tsp_test_tables.restype = I
     lib.tsp_profile_enable.argtypes = [P, I]
     lib.tsp_profile_enable.restype = I
     lib.tsp_profile_read.argtypes = [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
@@ -356,6 +359,19 @@ def tsp_test_step_walk(plan: Plan, kv0: int) -> np.ndarray:
     _check(_lib.tsp_test_step_walk(plan.handle, kv0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cap,
                                    ctypes.byref(n)), "tsp_test_step_walk")
     return out[:n.value].copy()
+
+
+TABLES = {"inv": 0, "qtile_maxpos": 1, "fwd_order": 2, "kv_order": 3, "q_order": 4}
+
+
+def tsp_test_tables(plan: Plan, name: str) -> np.ndarray:
+    n = ctypes.c_int64()
+    which = TABLES[name]
+    _lib.tsp_test_tables(plan.handle, which, None, 0, ctypes.byref(n))
+    out = np.zeros(n.value, dtype=np.int32)
+    _check(_lib.tsp_test_tables(plan.handle, which, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n.value,
+                                ctypes.byref(n)), "tsp_test_tables")
+    return out
 
 
 def tsp_test_wait_timeout(plan: Plan, limit_cycles: int, result, stream=None) -> None:

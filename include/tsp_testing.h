@@ -44,6 +44,20 @@ tsp_status tsp_test_buffer_offset(tsp_plan_t plan, const char *name, size_t *off
  * TSP_ERR_INVALID_ARG for from outside [0, S / 64] or kv0 outside [0, S). */
 tsp_status tsp_test_next_visible(tsp_plan_t plan, int from, int kv0, int *out);
 
+/* Host copy of a table the plan uploads for the kernels (computed on the
+ * host, no GPU needed), written to out[0 .. *count) (host memory; *count
+ * always receives the length).  which:
+ *   0  inverse zigzag map: position -> local row, [S]
+ *   1  largest position of each 128-row local query tile, [S/128]
+ *   2  forward attention work order: pairs (query block * heads + head,
+ *      number of 128-key tiles to visit) for 256-row query blocks
+ *   3  dK/dV work order: key tile * heads + head, [S/128 * heads]
+ *   4  dQ work order: query tile * heads + head, [S/128 * heads]
+ * Work orders are head-major with the longest items of a head first.
+ * TSP_ERR_INVALID_ARG for another `which`, a NULL pointer or a table longer
+ * than `capacity`. */
+tsp_status tsp_test_tables(tsp_plan_t plan, int which, int32_t *out, int64_t capacity, int64_t *count);
+
 /* Host replay of the walk the dK/dV kernel makes over the 64-row query steps
  * that can see the key tile starting at position kv0: writes the visited
  * steps, in the kernel's order, to steps[0 .. *count) (host memory, at most

@@ -2,6 +2,7 @@
 every symbol the headers declare, and its integer outputs (zigzag map, shard
 schedules) match the oracle bit for bit; argument errors are reported."""
 
+import ctypes
 import os
 import re
 
@@ -10,6 +11,7 @@ import pytest
 
 import oracle as O
 import folded_tensor_sequence_map_b200 as T
+import folded_tensor_sequence_map_b200.tsp as TT
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -83,6 +85,48 @@ def test_step_walk_visits_exactly_the_visible_steps(h, H, F, S, D):
         kv0 = int(kt) * 128
         want = np.nonzero(step_max >= kv0)[0]
         assert np.array_equal(T.tsp_test_step_walk(p, kv0), want), (S, D, kv0)
+
+
+@pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
+                                       (256, 4, 1024, 2048, 1)])
+def test_kernel_tables_match_the_zigzag_map(h, H, F, S, D):
+    """The tables the plan uploads, rebuilt from the oracle's zigzag map: the
+    inverse map, each 128-row tile's largest position, and three attention
+    work orders.  Each order covers every item once, head-major, longest
+    first within a head."""
+    p = T.tsp_plan(h, H, F, S, D)
+    zig = O.zigzag_map(S, D).ravel()
+    inv = T.tsp_test_tables(p, "inv")
+    assert np.array_equal(zig[inv], np.arange(S))
+    qmax = T.tsp_test_tables(p, "qtile_maxpos")
+    assert np.array_equal(qmax, zig.reshape(S // 128, 128).max(axis=1))
+
+    def head_major_longest_first(items, cost):
+        heads = items % H
+        assert np.all(np.diff(heads) >= 0)
+        for hd in range(H):
+            c = cost[heads == hd]
+            assert np.all(np.diff(c) <= 0)
+
+    fwd = T.tsp_test_tables(p, "fwd_order").reshape(-1, 2)
+    items, nkv = fwd[:, 0], fwd[:, 1]
+    assert np.array_equal(np.sort(items), np.arange((S // 256) * H))
+    block_max = zig.reshape(S // 256, 256).max(axis=1)
+    assert np.array_equal(nkv, block_max[items // H] // 128 + 1)
+    head_major_longest_first(items, nkv)
+
+    kv = T.tsp_test_tables(p, "kv_order")
+    assert np.array_equal(np.sort(kv), np.arange((S // 128) * H))
+    seen_by = np.array([(qmax >= kt * 128).sum() for kt in range(S // 128)])
+    head_major_longest_first(kv, seen_by[kv // H])
+
+    q = T.tsp_test_tables(p, "q_order")
+    assert np.array_equal(np.sort(q), np.arange((S // 128) * H))
+    head_major_longest_first(q, qmax[q // H])
+
+    n = ctypes.c_int64()
+    rc = TT._lib.tsp_test_tables(p.handle, 7, None, 0, ctypes.byref(n))
+    assert T.STATUS_NAMES[rc] == "TSP_ERR_INVALID_ARG"
 
 
 def test_prefill_checks_arguments_before_enqueueing():
