@@ -83,6 +83,21 @@ def stage_flops(s: LayerShape) -> dict:
     }
 
 
+def hbm_stage_bytes(s: LayerShape) -> dict:
+    """Algorithmic HBM bytes of one launch of each memory-bound stage: every
+    tensor the stage reads or writes, once (gains and norm statistics
+    included; the dg partial sums are written and read back once)."""
+    S, h, H = float(s.S), float(s.h), float(s.heads)
+    partials = S / 64 * h * 4
+    return {
+        "fwd_rmsnorm1": S * h * (2 + 2) + S * 4 + h * 4,                  # x bf16 -> a bf16, rstd
+        "fwd_rmsnorm2": S * h * (4 + 2) + S * 4 + h * 4,                  # y f32 -> b bf16, rstd
+        "bwd_rmsnorm2": S * h * (4 + 4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,  # db, y, dY -> dy f32+bf16
+        "bwd_rmsnorm1": S * h * (4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,      # da, x, dy -> dx bf16
+        "bwd_attn_delta": S * h * (2 + 2) + S * H * 4,                    # O, dO -> delta f32 [H][S]
+    }
+
+
 # ---------------------------------------------------------------------------
 # multi-process plumbing (N > 1: independent replicas)
 # ---------------------------------------------------------------------------
@@ -404,6 +419,12 @@ def main():
                      "traffic_note": "ncu dram bytes of one launch at S=16384 scaled by S" if dom in MEASURED_TRAFFIC
                      else "not measured for this kernel",
                      "peak_note": f"{src} sustained bf16 (kernel timed inside a long step)"},
+        "hbm_stages": {k: {"bytes": b, "ms": stages[k][0] / max(stages[k][1], 1),
+                           "achieved": b / (stages[k][0] / max(stages[k][1], 1) / 1e3) / 1e9,
+                           "peak": hbm, "unit": "GB/s",
+                           "frac": b / (stages[k][0] / max(stages[k][1], 1) / 1e3) / 1e9 / hbm}
+                       for k, b in hbm_stage_bytes(shape).items() if stages.get(k, (0, 0))[0] > 0},
+        "hbm_peak_note": f"{src} HBM copy bandwidth",
         "stage_ms_per_step": {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()},
         "stage_share": {k: round(v[0] / total_ms, 4) for k, v in stages.items()},
         "gpu_launches": int(launches),

@@ -57,3 +57,25 @@ def test_clock_summary_parses_reasons():
                "garbage"]
     s = c.summary()
     assert s["sm_mhz"] == 1850 and s["sm_max_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+
+
+def test_stage_accounting_covers_every_library_stage_once():
+    """Each library stage is either a contraction (FLOPs) or memory-bound
+    (bytes), never both and never neither."""
+    import folded_tensor_sequence_map_b200 as T
+
+    s, _ = WORKLOADS["7b_s128k"]
+    p = T.tsp_plan(s.h, s.heads, s.ffn, s.S, s.D)
+    names = {T.tsp_profile_read(p, i)[0] for i in range(T.TSP_NUM_STAGES)}
+    flops, hbm = set(bench.stage_flops(s)), set(bench.hbm_stage_bytes(s))
+    assert not flops & hbm
+    assert flops | hbm == names
+
+
+def test_hbm_stage_bytes_of_the_forward_norm():
+    """RMSNorm1 forward at the 7B shape reads x and writes a (bf16, 1 GiB
+    each) plus rstd and the gain."""
+    s, _ = WORKLOADS["7b_s128k"]
+    b = bench.hbm_stage_bytes(s)
+    assert b["fwd_rmsnorm1"] == 2 * 2 * s.S * s.h + 4 * s.S + 4 * s.h
+    assert all(v > 0 for v in b.values())
