@@ -374,3 +374,17 @@ def test_ring_mlp_matches_the_layer_oracle():
     b = np.concatenate(cache["b"], axis=0)
     y = np.concatenate(cache["y"], axis=0)
     assert _relerr(O.tsp_ring_mlp(b, w["w1"], w["w2"], y, D), zl) < 1e-12
+
+
+@pytest.mark.parametrize("H,dh,F,D", [(4, 32, 512, 2), (32, 128, 16384, 8), (16, 64, 4096, 16), (8, 32, 256, 1)])
+def test_shards_partition_heads_and_ffn_units(H, dh, F, D):
+    """Shard t of the attention weights is the contiguous block of heads
+    [t H/D, (t+1) H/D) (their dh-wide column groups), and shard s of the MLP
+    the units [s F/D, (s+1) F/D): over all shards, each column or unit
+    exactly once, in order."""
+    heads = [O.head_cols(t, H, D, dh) for t in range(D)]
+    units = [O.ffn_units(s, F, D) for s in range(D)]
+    assert np.array_equal(np.concatenate([np.arange(H * dh)[c] for c in heads]), np.arange(H * dh))
+    assert np.array_equal(np.concatenate([np.arange(F)[u] for u in units]), np.arange(F))
+    assert all((c.stop - c.start) == (H // D) * dh for c in heads)
+    assert all((u.stop - u.start) == F // D for u in units)
