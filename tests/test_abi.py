@@ -72,7 +72,8 @@ def test_next_visible_matches_zigzag_scan(h, H, F, S, D):
 
 
 @pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
-                                       (256, 4, 1024, 2048, 1), (4096, 32, 16384, 131072, 8)])
+                                       (256, 4, 1024, 2048, 1), (4096, 32, 16384, 32768, 8),
+                                       (4096, 32, 16384, 131072, 8)])
 def test_step_walk_visits_exactly_the_visible_steps(h, H, F, S, D):
     """The dK/dV kernel's walk for a key tile at kv0 visits, in ascending
     order and once each, exactly the 64-row local steps holding a row at a
@@ -88,7 +89,7 @@ def test_step_walk_visits_exactly_the_visible_steps(h, H, F, S, D):
 
 
 @pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
-                                       (256, 4, 1024, 2048, 1)])
+                                       (256, 4, 1024, 2048, 1), (4096, 32, 16384, 32768, 8)])
 def test_kernel_tables_match_the_zigzag_map(h, H, F, S, D):
     """The tables the plan uploads, rebuilt from the oracle's zigzag map: the
     inverse map, each 128-row tile's largest position, and three attention
