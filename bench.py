@@ -39,24 +39,31 @@ from synth_inputs import WORKLOADS, LayerShape, make_layer_inputs  # noqa: E402
 METRIC = "TSP layer tokens/s (fwd, fwd+bwd) at S=128K, D=8; % bf16 tensor-core peak"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "7b_s128k"
-CPU_SAMPLE_S = 2048  # oracle sample: the same 7B layer at this many tokens
+# oracle samples: the same 7B layer (fwd+bwd) at these token counts; the
+# reference arm times the first, cpu_baseline times both
+CPU_SAMPLE_S = (1024, 2048)
+NOMINAL_TFLOPS = 2250.0   # dense bf16/fp16 datasheet figure
+NOMINAL_MHZ = 1965.0      # clocks.max.sm of this part
 
 # DRAM bytes (read + write) of one launch from an ncu capture of the current
-# kernel build, and the S of that capture (profiles/attention_kernels_7b_s16384_d8.md).
-# The traffic is the compulsory one and grows in proportion to S, so it is
-# scaled by S to the benchmarked launch.  Must be re-measured (or removed)
-# whenever the kernel changes.
-MEASURED_TRAFFIC = {"bwd_attn_dkdv": (559.84256e6 + 244.09344e6, 16384)}
+# kernel build, and the S of that capture.  The traffic is the compulsory one
+# and grows in proportion to S, so it is scaled by S to the benchmarked
+# launch.  Must be re-measured (or removed) whenever the kernel changes.
+MEASURED_TRAFFIC = {}
 
 
 def peaks():
+    """(burst TFLOP/s, sustained TFLOP/s, HBM GB/s, source): the measured copy
+    bandwidth and cuBLAS GEMM rates of this machine's B200s when the driver has
+    written them, else an earlier measurement on this machine (fp16 and bf16
+    dense MMAs have the same rate)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
         return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
     except (OSError, KeyError, ValueError):
-        return 1590.0, 1400.0, 6650.0, "fallback"
+        return 1590.0, 1400.0, 6650.0, "fallback (earlier measurement on this pool)"
 
 
 def layer_flops(s: LayerShape, backward: bool) -> float:
@@ -89,10 +96,13 @@ def hbm_stage_bytes(s: LayerShape) -> dict:
     included; the dg partial sums are written and read back once)."""
     S, h, H = float(s.S), float(s.h), float(s.heads)
     partials = S / 64 * h * 4
+    wts = (4.0 * h * h + 2.0 * h * s.ffn) * 2                             # the four weights, 16-bit
     return {
-        "fwd_rmsnorm1": S * h * (2 + 2) + S * 4 + h * 4,                  # x bf16 -> a bf16, rstd
-        "fwd_rmsnorm2": S * h * (4 + 2) + S * 4 + h * 4,                  # y f32 -> b bf16, rstd
-        "bwd_rmsnorm2": S * h * (4 + 4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,  # db, y, dY -> dy f32+bf16
+        "fwd_convert_weights": 3 * wts,                                   # read twice (max, convert), write fp16
+        "fwd_rmsnorm1": S * h * (2 + 2) + S * 4 + h * 4,                  # x bf16 -> a fp16, rstd
+        "fwd_rmsnorm2": S * h * (4 + 2) + S * 4 + h * 4,                  # y f32 -> b fp16, rstd
+        "bwd_convert_dy": 3 * S * h * 2,                                  # dY read twice, fp16 copy written
+        "bwd_rmsnorm2": S * h * (4 + 4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,  # db, y, dY -> dy f32+fp16
         "bwd_rmsnorm1": S * h * (4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,      # da, x, dy -> dx bf16
         "bwd_attn_delta": S * h * (2 + 2) + S * H * 4,                    # O, dO -> delta f32 [H][S]
     }
@@ -198,13 +208,13 @@ class ClockSampler:
 # CPU oracle timing (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_seconds(shape: LayerShape, seed: int) -> tuple:
-    """Time the fp64 oracle's folded forward + backward of the same layer at
-    CPU_SAMPLE_S tokens.  Returns (seconds, sample_shape)."""
+def oracle_sample_seconds(shape: LayerShape, seed: int, S: int) -> float:
+    """Wall time of the fp64 oracle's folded forward + backward of the same
+    layer at S tokens (inputs drawn and converted outside the timed part)."""
     import oracle as O
     from synth_inputs import bits_to_f32
 
-    s = LayerShape(h=shape.h, heads=shape.heads, ffn=shape.ffn, S=CPU_SAMPLE_S, D=shape.D)
+    s = LayerShape(h=shape.h, heads=shape.heads, ffn=shape.ffn, S=S, D=shape.D)
     inp = make_layer_inputs(s, seed)
     zig = O.zigzag_map(s.S, s.D).ravel()
     w = {k: bits_to_f32(inp[k]).astype(np.float64) for k in ("wqkv", "wo", "w1", "w2")}
@@ -215,7 +225,7 @@ def oracle_sample_seconds(shape: LayerShape, seed: int) -> tuple:
     t0 = time.perf_counter()
     _, cache = O.tsp_layer_forward(x, w, s.heads, s.D)
     O.tsp_layer_backward(dy, w, cache)
-    return time.perf_counter() - t0, s
+    return time.perf_counter() - t0
 
 
 def cpu_threads() -> int:
@@ -230,44 +240,61 @@ def cpu_threads() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_baseline(shape: LayerShape, seed: int, steps: int = 1) -> dict:
-    secs = []
-    for _ in range(steps):
-        t, s = oracle_sample_seconds(shape, seed)
-        secs.append(t)
-    t = statistics.median(secs)
-    full = step_flops(shape)
-    samp = step_flops(s)
-    projected = t * full / samp
+def project_two_sizes(t1: float, s1: int, t2: float, s2: int, S: int) -> float:
+    """Seconds at S from a fit T(s) = a s + b s^2 through two measured runs:
+    the token-local work grows with s, the causal attention with s^2."""
+    b = (t2 / s2 - t1 / s1) / (s2 - s1)
+    a = t1 / s1 - b * s1
+    return max(a, 0.0) * S + max(b, 0.0) * S * S
+
+
+def cpu_baseline(shape: LayerShape, seed: int) -> dict:
+    """The oracle timed on this host at the two sample sizes.  `value` is what
+    was timed: tokens/s of the larger sample; the S=131072 figure is a
+    projection, in its own field."""
+    (s1, s2) = CPU_SAMPLE_S
+    t1 = oracle_sample_seconds(shape, seed, s1)
+    t2 = oracle_sample_seconds(shape, seed, s2)
+    proj = project_two_sizes(t1, s1, t2, s2, shape.S)
     return {
-        "value": shape.S / projected,
+        "value": s2 / t2,
         "unit": UNIT,
         "cores": cpu_threads(),
         "kind": "oracle",
-        "sample": (f"fp64 NumPy oracle, folded forward+backward of the same 7B layer at S={s.S}, D={s.D} "
-                   f"({t:.2f} s median of {len(secs)}), projected to S={shape.S} by algorithmic FLOPs "
-                   f"({full:.3e} / {samp:.3e})"),
-        "sample_seconds": t,
+        "sample": (f"fp64 NumPy oracle, folded forward+backward of the same 7B layer (D={shape.D}) at "
+                   f"S={s2}: {t2:.2f} s measured, one run (value = {s2} tokens / {t2:.2f} s); also S={s1}: "
+                   f"{t1:.2f} s measured"),
+        "projected_to_S": shape.S,
+        "projected_value": shape.S / proj,
+        "projection": f"T(S) = a S + b S^2 through the two measured runs: {proj:.0f} s at S={shape.S}",
     }
 
 
 def run_reference(args, shape: LayerShape, seed: int):
+    """--impl reference: the oracle itself, timed on the host cores.  One step
+    is the oracle's folded forward + backward of the same layer at the first
+    sample size; `value` and `ms_per_step` describe exactly the timed steps."""
     rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
+    S = CPU_SAMPLE_S[0]
     for _ in range(args.warmup):
-        oracle_sample_seconds(shape, seed)
-    base = cpu_baseline(shape, seed, steps=args.steps)
-    per_step = shape.S / base["value"]
+        oracle_sample_seconds(shape, seed, S)
+    secs = [oracle_sample_seconds(shape, seed, S) for _ in range(args.steps)]
+    total = sum(secs)
+    value = S * args.steps / total
     line = {
-        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "h": shape.h, "heads": shape.heads, "ffn": shape.ffn, "seq_len": shape.S,
                    "D": shape.D, "global_batch": 1, "parallelism": "virtual ranks on one device",
-                   "l2": "inputs larger than L2"},
-        "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
-        "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                   "l2": "inputs larger than L2", "timed_sample_seq_len": S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": (f"fp64 NumPy oracle, folded forward+backward of the same 7B layer at S={S}, "
+                                    f"D={shape.D}: {args.steps} timed runs, {total:.2f} s in all "
+                                    f"(median {statistics.median(secs):.2f} s); value = tokens timed / seconds")},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -374,8 +401,9 @@ def main():
     # end to end: pinned host inputs in, results out, inside the timed region
     e2e = None
     if not args.no_e2e:
+        # every result comes back: the output, dx and all weight and gain gradients
         y_host = torch.empty(S, h, dtype=bf).pin_memory()
-        dx_host = torch.empty(S, h, dtype=bf).pin_memory()
+        g_host = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in grads.items()}
 
         def e2e_step():
             x.copy_(x_host, non_blocking=True)
@@ -383,12 +411,15 @@ def main():
             fwd()
             bwd()
             y_host.copy_(y, non_blocking=True)
-            dx_host.copy_(grads["dx"], non_blocking=True)
+            for k, v in grads.items():
+                g_host[k].copy_(v, non_blocking=True)
 
         e2e_step()
         t_e2e = timed(e2e_step, args.steps)
+        d2h = y.numel() * y.element_size() + sum(v.numel() * v.element_size() for v in grads.values())
         e2e = {"value": world * S * args.steps / t_e2e, "unit": UNIT,
-               "h2d_bytes_per_step": 2 * S * h * 2, "d2h_bytes_per_step": 2 * S * h * 2}
+               "h2d_bytes_per_step": x.numel() * 2 + dy.numel() * 2, "d2h_bytes_per_step": d2h,
+               "copied": "x, dY in; z, dx, dg1, dWqkv, dWo, dg2, dW1, dW2 out (pinned host memory)"}
 
     burst, sustained, hbm, src = peaks()
     flops = stage_flops(shape)
@@ -400,10 +431,18 @@ def main():
     fwd_value = world * S * args.steps / t_fwd
     frac_step = step_flops(shape) * args.steps / t_step / 1e12 / sustained
     frac_fwd = layer_flops(shape, False) * args.steps / t_fwd / 1e12 / sustained
+    clocks = clk.summary()
+    run_mhz = clocks.get("sm_mhz") or NOMINAL_MHZ
+    # the datasheet dense peak taken at the run's median SM clock: the tensor
+    # pipe's rate scales with the clock, and the power cap sets the clock
+    at_clock = NOMINAL_TFLOPS * run_mhz / NOMINAL_MHZ
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_step / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
+        "dtype": "f16", "data": "synthetic",
+        "dtype_note": ("bf16 inputs and outputs; every tensor-core operand is fp16 (exact power-of-two-scaled "
+                       "copies of the bf16 weights and dY, fp16 intermediates), fp32 accumulation; fp16 and "
+                       "bf16 dense MMAs have the same rate"),
         "config": {"workload": args.workload, "h": h, "heads": shape.heads, "ffn": F, "seq_len": S, "D": shape.D,
                    "global_batch": 1, "parallelism": "virtual ranks on one device; replicas across GPUs",
                    "l2": "inputs larger than L2 (1 GiB activations per tensor)"},
@@ -411,13 +450,19 @@ def main():
                 "frac_of_bf16_peak": frac_fwd},
         "fwd_bwd_frac_of_bf16_peak": frac_step,
         "fwd_bwd_frac_of_bf16_burst_peak": frac_step * sustained / burst,
-        "peak_source": f"{src} (sustained {sustained} TFLOP/s for the step fractions)",
+        "fwd_bwd_frac_of_nominal_at_run_clock": frac_step * sustained / at_clock,
+        "fwd_frac_of_bf16_burst_peak": frac_fwd * sustained / burst,
+        "fwd_frac_of_nominal_at_run_clock": frac_fwd * sustained / at_clock,
+        "peak_source": (f"{src} (sustained {sustained} TFLOP/s for the step fractions, burst {burst}; "
+                        f"nominal {NOMINAL_TFLOPS:.0f} TFLOP/s at {NOMINAL_MHZ:.0f} MHz scaled to the run's "
+                        f"median {run_mhz:.0f} MHz = {at_clock:.0f} TFLOP/s)"),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                     "frac": achieved / sustained,
+                     "frac": achieved / sustained, "frac_of_burst": achieved / burst,
+                     "frac_of_nominal_at_run_clock": achieved / at_clock,
                      "traffic": (MEASURED_TRAFFIC[dom][0] * S / MEASURED_TRAFFIC[dom][1]) if dom in MEASURED_TRAFFIC
                      else None,
-                     "traffic_note": "ncu dram bytes of one launch at S=16384 scaled by S" if dom in MEASURED_TRAFFIC
-                     else "not measured for this kernel",
+                     "traffic_note": "ncu dram bytes of one launch at a smaller S scaled by S" if dom in MEASURED_TRAFFIC
+                     else "not measured for this kernel build",
                      "peak_note": f"{src} sustained bf16 (kernel timed inside a long step)"},
         "hbm_stages": {k: {"bytes": b, "ms": stages[k][0] / max(stages[k][1], 1),
                            "achieved": b / (stages[k][0] / max(stages[k][1], 1) / 1e3) / 1e9,
@@ -428,12 +473,11 @@ def main():
         "stage_ms_per_step": {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()},
         "stage_share": {k: round(v[0] / total_ms, 4) for k, v in stages.items()},
         "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        base = cpu_baseline(shape, seed)
-        line["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        line["cpu_baseline"] = cpu_baseline(shape, seed)
     if rank == 0:
         print(json.dumps(line), flush=True)
     del plan

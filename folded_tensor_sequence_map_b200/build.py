@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtsp.so")
-SOURCES = ["plan.cu", "gemm.cu", "norm.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu"]
+SOURCES = ["plan.cu", "gemm.cu", "norm.cu", "convert.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

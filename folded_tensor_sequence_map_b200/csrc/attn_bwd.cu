@@ -10,13 +10,18 @@
 // for the backward).
 //
 // Three kernels, no atomics (deterministic):
-//   attn_delta   Delta[h][row] = sum_d dO * O (bf16 inputs, fp32 sum).
+//   attn_delta   Delta[h][row] = sum_d dO * O (fp16 inputs, fp32 sum).
 //   attn_dkdv2   one item = (head, 128-key tile); steps of 64 query rows over
 //                the query tiles that see any of its keys.  S^T = K Q^T and
-//                dP^T = V dO^T in TMEM; P^T, dS^T written to smem as bf16;
-//                dV += P^T dO and dK += dS^T Q accumulate in TMEM.
+//                dP^T = V dO^T in TMEM; P^T and dS^T go back into TMEM as
+//                packed fp16 over the columns they were read from; dV += P^T dO
+//                and dK += dS^T Q (A operand from TMEM) accumulate in TMEM.
 //   attn_dq2     one item = (head, 128-row query tile); steps of 64 keys.
-//                S = Q K^T, dP = dO V^T in TMEM; dS to smem; dQ += dS K.
+//                S = Q K^T, dP = dO V^T in TMEM; dS back into TMEM as packed
+//                fp16; dQ += dS K.
+// Q, K, V, O, dO and the outputs dQ, dK, dV are fp16 (gradients in the
+// backward's scaled domain).  The P^T feeding dV carries a factor 2^kPOff so
+// small probabilities stay normal fp16 numbers; the dV epilogue takes it out.
 // Warp roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2-17 element-wise (four
 // groups of four; thread = TMEM lane = row of the 128-row tile).
 #include "common.cuh"
@@ -24,6 +29,9 @@
 
 namespace tsp {
 namespace {
+
+constexpr float kPOff = 7.0f;                 // log2 of the factor carried by the fp16 P^T
+constexpr float kPOffInv = 1.0f / 128.0f;     // 2^-kPOff
 
 __device__ __forceinline__ float ex2b(float x) {
     float y;
@@ -68,8 +76,7 @@ CUtensorMapSwizzle swz_of() {
 }
 
 // ---------------------------------------------------------------------------
-__global__ void attn_delta_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *dout, float *delta, int S, int H,
-                                  int dh) {
+__global__ void attn_delta_kernel(const __half *o, const __half *dout, float *delta, int S, int H, int dh) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32, lane = threadIdx.x % 32;
     if (warp >= S * H) return;
     const int row = warp / H, head = warp % H;
@@ -78,7 +85,7 @@ __global__ void attn_delta_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *d
     for (int c = lane * 2; c < dh; c += 64) {
         uint32_t a = *reinterpret_cast<const uint32_t *>(o + base + c);
         uint32_t b = *reinterpret_cast<const uint32_t *>(dout + base + c);
-        s += bf16_lo(a) * bf16_lo(b) + bf16_hi(a) * bf16_hi(b);
+        s += f16_lo(a) * f16_lo(b) + f16_hi(a) * f16_hi(b);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
@@ -101,7 +108,7 @@ struct BwdParams {
 //   tensor core works on the next step while the element-wise warps (four
 //   groups of four, 16 query columns each: four warps per SM sub-partition
 //   to hide TMEM and barrier latency) turn step g into P^T and dS^T.  P^T and
-//   dS^T go back into TMEM as packed bf16 (two queries per column) in the
+//   dS^T go back into TMEM as packed fp16 (two queries per column) in the
 //   columns their S^T / dP^T values came from, where the dV / dK MMAs read
 //   them as the A operand.
 template <int DH>
@@ -266,8 +273,8 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
         {
             const bool leader = elect_one();
             const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
-            constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
-            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
+            constexpr uint32_t idS = idesc_f16(128, 64, false, false);
+            constexpr uint32_t idG = idesc_f16(128, DH, false, true);
             const uint64_t dK0 = kdesc<DH>(smem_u32(smem + K::OFF_K), 0);
             const uint64_t dV0 = kdesc<DH>(smem_u32(smem + K::OFF_V), 0);
             int item_iter = 0, g = 0;
@@ -281,11 +288,11 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                     const uint64_t dO0 = kdesc64<DH>(smem_u32(smem + K::OFF_DO + s * K::QTILE), 0);
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 64 * b, desc_plus(dK0, kdesc_off<DH>(kk)), desc_plus(dQ0, kdesc64_off<DH>(kk)),
+                        umma_ss(tmem + 64 * b, desc_plus(dK0, kdesc_off<DH>(kk)), desc_plus(dQ0, kdesc64_off<DH>(kk)),
                                   idS, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 128 + 64 * b, desc_plus(dV0, kdesc_off<DH>(kk)),
+                        umma_ss(tmem + 128 + 64 * b, desc_plus(dV0, kdesc_off<DH>(kk)),
                                   desc_plus(dO0, kdesc64_off<DH>(kk)), idS, kk > 0);
                     umma_commit(&s_full[b]);
                 }
@@ -315,11 +322,11 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                         // A operands from TMEM: queries 16 kk .. 16 kk + 15 packed at column 16 kk
 #pragma unroll
                         for (int kk = 0; kk < K::BQ / 16; ++kk)
-                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, desc_plus(gO0, mndesc64_off<DH>(kk)), idG,
+                            umma_ts(tmem + 256, tmem + 64 * b + kk * 16, desc_plus(gO0, mndesc64_off<DH>(kk)), idG,
                                          (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
                         for (int kk = 0; kk < K::BQ / 16; ++kk)
-                            umma_bf16_ts(tmem + 384, tmem + 128 + 64 * b + kk * 16, desc_plus(gQ0, mndesc64_off<DH>(kk)),
+                            umma_ts(tmem + 384, tmem + 128 + 64 * b + kk * 16, desc_plus(gQ0, mndesc64_off<DH>(kk)),
                                          idG, (!first || kk > 0) ? 1u : 0u);
                         umma_commit(&q_empty[s]);
                     }
@@ -376,18 +383,24 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 l = lse4[e4], d = dl4[e4];
                     const int e = 4 * e4;
-                    float p0 = ex2b(fmaf(sv[e], sl2, -l.x)), p1 = ex2b(fmaf(sv[e + 1], sl2, -l.y));
-                    float p2 = ex2b(fmaf(sv[e + 2], sl2, -l.z)), p3 = ex2b(fmaf(sv[e + 3], sl2, -l.w));
+                    // p = 2^kPOff P (the offset rides in the exponent)
+                    float p0 = ex2b(fmaf(sv[e], sl2, kPOff - l.x)), p1 = ex2b(fmaf(sv[e + 1], sl2, kPOff - l.y));
+                    float p2 = ex2b(fmaf(sv[e + 2], sl2, kPOff - l.z)), p3 = ex2b(fmaf(sv[e + 3], sl2, kPOff - l.w));
                     if (first_vis > 0) {
                         p0 = e >= first_vis ? p0 : 0.f;
                         p1 = e + 1 >= first_vis ? p1 : 0.f;
                         p2 = e + 2 >= first_vis ? p2 : 0.f;
                         p3 = e + 3 >= first_vis ? p3 : 0.f;
                     }
-                    pk[2 * e4] = pack_bf16(p0, p1);
-                    pk[2 * e4 + 1] = pack_bf16(p2, p3);
-                    dk[2 * e4] = pack_bf16(p0 * (dp[e] - d.x), p1 * (dp[e + 1] - d.y));
-                    dk[2 * e4 + 1] = pack_bf16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
+                    pk[2 * e4] = pack_f16(p0, p1);
+                    pk[2 * e4 + 1] = pack_f16(p2, p3);
+                    // dS = P (dP - Delta), without the offset
+                    p0 *= kPOffInv;
+                    p1 *= kPOffInv;
+                    p2 *= kPOffInv;
+                    p3 *= kPOffInv;
+                    dk[2 * e4] = pack_f16(p0 * (dp[e] - d.x), p1 * (dp[e + 1] - d.y));
+                    dk[2 * e4 + 1] = pack_f16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
                 }
                 // each group packs its 16 queries into the first 8 of the 16
                 // columns it has just read, so no group writes what another
@@ -404,23 +417,27 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             if (!warp_wait(acc_full, acc_iter & 1, abort_flag, err)) break;
             ++acc_iter;
             tc_fence_after();
-            // groups 0, 1 write dV and groups 2, 3 write dK (scaled), at the key
-            // owner's local row; each pair splits the 32-column chunks
+            // groups 0, 1 write dV (offset removed) and groups 2, 3 write dK
+            // (scaled), at the key owner's local row; each pair splits the
+            // 32-column chunks
             const int lrow = a.inv_map[key];
             const int which = grp >> 1;
             void *dst = which == 0 ? a.dv : a.dk;
-            const float f = which == 0 ? 1.0f : scale;
-            __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(dst) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+            const float f = which == 0 ? kPOffInv : scale;
+            __half *row = static_cast<__half *>(dst) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
 #pragma unroll 1
             for (int c = grp & 1; c < DH / 32; c += 2) {
                 float v[32];
                 tmem_ld32(tmem + lane_off + 256 + 128 * which + c * 32, v);
                 tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= f;
+                flag_range(maxabs32(v), a.err);
                 uint4 *d4 = reinterpret_cast<uint4 *>(row + c * 32);
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq)
-                    d4[qq] = make_uint4(pack_bf16(v[8 * qq] * f, v[8 * qq + 1] * f), pack_bf16(v[8 * qq + 2] * f, v[8 * qq + 3] * f),
-                                        pack_bf16(v[8 * qq + 4] * f, v[8 * qq + 5] * f), pack_bf16(v[8 * qq + 6] * f, v[8 * qq + 7] * f));
+                    d4[qq] = make_uint4(pack_f16(v[8 * qq], v[8 * qq + 1]), pack_f16(v[8 * qq + 2], v[8 * qq + 3]),
+                                        pack_f16(v[8 * qq + 4], v[8 * qq + 5]), pack_f16(v[8 * qq + 6], v[8 * qq + 7]));
             }
             tc_fence_before();
         }
@@ -437,7 +454,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 //   256 (128 query lanes).  The MMA warp issues S/dP of step j+1 before dQ of
 //   step j, so the tensor core works while the element-wise warps (two groups
 //   of four, 32 key columns each) turn step j into dS, which goes back into
-//   TMEM as packed bf16 in the S columns it came from (the dQ MMA's A).
+//   TMEM as packed fp16 in the S columns it came from (the dQ MMA's A).
 template <int DH>
 struct Dq2Cfg {
     using C = BCfg<DH>;
@@ -550,8 +567,8 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
         {
             const bool leader = elect_one();
             const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
-            constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
-            constexpr uint32_t idG = idesc_bf16(128, DH, false, true);
+            constexpr uint32_t idS = idesc_f16(128, 64, false, false);
+            constexpr uint32_t idG = idesc_f16(128, DH, false, true);
             const uint64_t dQ0 = kdesc<DH>(smem_u32(smem + Q::OFF_Q), 0);
             const uint64_t dO0 = kdesc<DH>(smem_u32(smem + Q::OFF_DO), 0);
             int item_iter = 0, g = 0;
@@ -565,11 +582,11 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                     const uint64_t dV0 = kdesc64<DH>(smem_u32(smem + Q::OFF_V + s * Q::KTILE), 0);
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 64 * b, desc_plus(dQ0, kdesc_off<DH>(kk)), desc_plus(dK0, kdesc64_off<DH>(kk)),
+                        umma_ss(tmem + 64 * b, desc_plus(dQ0, kdesc_off<DH>(kk)), desc_plus(dK0, kdesc64_off<DH>(kk)),
                                   idS, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_bf16(tmem + 128 + 64 * b, desc_plus(dO0, kdesc_off<DH>(kk)),
+                        umma_ss(tmem + 128 + 64 * b, desc_plus(dO0, kdesc_off<DH>(kk)),
                                   desc_plus(dV0, kdesc64_off<DH>(kk)), idS, kk > 0);
                     umma_commit(&s_full[b]);
                 }
@@ -594,7 +611,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                         // A = dS from TMEM: keys 16 kk .. 16 kk + 15 packed at column 16 kk
 #pragma unroll
                         for (int kk = 0; kk < Q::BK / 16; ++kk)
-                            umma_bf16_ts(tmem + 256, tmem + 64 * b + kk * 16, desc_plus(gK0, mndesc64_off<DH>(kk)), idG,
+                            umma_ts(tmem + 256, tmem + 64 * b + kk * 16, desc_plus(gK0, mndesc64_off<DH>(kk)), idG,
                                          (j > 0 || kk > 0) ? 1u : 0u);
                         umma_commit(&k_empty[s]);
                     }
@@ -639,7 +656,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
                 for (int e = 0; e < 16; e += 2) {
                     const float p0 = (k0 + e <= pos) ? ex2b(fmaf(sv[e], sl2, -lse)) : 0.f;
                     const float p1 = (k0 + e + 1 <= pos) ? ex2b(fmaf(sv[e + 1], sl2, -lse)) : 0.f;
-                    pk[e / 2] = pack_bf16(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
+                    pk[e / 2] = pack_f16(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
                 }
                 // packed into the first 8 of the 16 columns this group just read
                 if (!warp_converged("dS TMEM store")) { ok = false; break; }
@@ -652,19 +669,20 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             if (!warp_wait(acc_full, item_iter & 1, abort_flag, err)) break;
             tc_fence_after();
             {
-                __nv_bfloat16 *dqrow = static_cast<__nv_bfloat16 *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+                __half *dqrow = static_cast<__half *>(a.dq) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
 #pragma unroll 1
                 for (int c = grp; c < DH / 32; c += kEwGroups) {
                     float v[32];
                     tmem_ld32(tmem + lane_off + 256 + c * 32, v);
                     tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] *= scale;
+                    flag_range(maxabs32(v), a.err);
                     uint4 *d4 = reinterpret_cast<uint4 *>(dqrow + c * 32);
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq)
-                        d4[qq] = make_uint4(pack_bf16(v[8 * qq] * scale, v[8 * qq + 1] * scale),
-                                            pack_bf16(v[8 * qq + 2] * scale, v[8 * qq + 3] * scale),
-                                            pack_bf16(v[8 * qq + 4] * scale, v[8 * qq + 5] * scale),
-                                            pack_bf16(v[8 * qq + 6] * scale, v[8 * qq + 7] * scale));
+                        d4[qq] = make_uint4(pack_f16(v[8 * qq], v[8 * qq + 1]), pack_f16(v[8 * qq + 2], v[8 * qq + 3]),
+                                            pack_f16(v[8 * qq + 4], v[8 * qq + 5]), pack_f16(v[8 * qq + 6], v[8 * qq + 7]));
                 }
             }
             tc_fence_before();
@@ -683,10 +701,10 @@ struct BwdMaps {
         using C = BCfg<DH>;
         const int h = a.H * DH;
         const auto swz = swz_of<DH>();
-        bool ok = encode_tensor_map_2d(&q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-        ok = ok && encode_tensor_map_2d(&k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-        ok = ok && encode_tensor_map_2d(&v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-        ok = ok && encode_tensor_map_2d(&dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        bool ok = encode_tensor_map_2d(&q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&k, a.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&v, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
         return ok;
     }
 };
@@ -708,8 +726,8 @@ cudaError_t launch_dkdv_impl(const AttnBwdDesc &a, const DevErr &err, int num_sm
     // Q and dO sub-tiles of 64 rows
     const int h = a.H * DH;
     const auto swz = swz_of<DH>();
-    bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
-    ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
     if (!ok) return cudaErrorInvalidValue;
     KvParams kp;
     kp.d = a;
@@ -732,8 +750,8 @@ cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms,
     // K and V sub-tiles of 64 keys
     const int h = a.H * DH;
     const auto swz = swz_of<DH>();
-    bool ok = encode_tensor_map_2d(&m.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
-    ok = ok && encode_tensor_map_2d(&m.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    bool ok = encode_tensor_map_2d(&m.k, a.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    ok = ok && encode_tensor_map_2d(&m.v, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
     if (!ok) return cudaErrorInvalidValue;
     const BwdParams bp = make_params(a, zig, qtile_maxpos);
     const int grid = bp.num_items < num_sms ? bp.num_items : num_sms;
@@ -748,9 +766,9 @@ cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms,
 
 cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st) {
     const int warps = a.S * a.H;
-    attn_delta_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.o),
-                                                                 static_cast<const __nv_bfloat16 *>(a.dout), a.delta,
-                                                                 a.S, a.H, a.dh);
+    attn_delta_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(static_cast<const __half *>(a.o),
+                                                                 static_cast<const __half *>(a.dout), a.delta, a.S,
+                                                                 a.H, a.dh);
     return cudaGetLastError();
 }
 

@@ -15,10 +15,15 @@
 //              other tile (ping-pong between the two softmax groups).
 //   warps 2-5  softmax group 0 (query tile 0), warps 6-9 group 1: thread =
 //              query row; online softmax in the log2 domain; P written back
-//              into TMEM as packed bf16 over the first half of S_w's
+//              into TMEM as packed fp16 over the first half of S_w's
 //              columns, where the P V MMA reads it as its A operand; O
 //              rescaled in TMEM when the running max grows by more than 2^8; final
-//              O / l written as bf16 and LSE (log2 domain) as fp32.
+//              O / l written as fp16 and LSE (log2 domain) as fp32.
+// Q, K, V, P and O are fp16.  P carries a factor 2^kPOff (exact: it is added
+// to the exponent), which O / l cancels and the LSE takes out again: with the
+// lazy rescale P stays below 2^(8 + kPOff) = 2^15 < 65504, and probabilities
+// down to 2^-(14 + kPOff) stay normal fp16 numbers, which matters at long
+// sequences, where most of a row's probabilities are small.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+dh), O1 [384,384+dh);
 // P_w overwrites the first 64 columns of S_w once S_w is in registers.
 #include "common.cuh"
@@ -28,6 +33,7 @@ namespace tsp {
 namespace {
 
 constexpr int kFwdThreads = 320;
+constexpr float kPOff = 7.0f;  // log2 of the factor carried by the fp16 P
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -45,7 +51,7 @@ __device__ __forceinline__ int zig_pos(int i, int L, int D, int c) {
 template <int DH>
 struct FwdCfg {
     static constexpr int SWB = DH * 2 < 128 ? DH * 2 : 128;   // swizzle span in bytes
-    static constexpr int ATOM_COLS = SWB / 2;                 // bf16 columns per swizzle atom
+    static constexpr int ATOM_COLS = SWB / 2;                 // 16-bit columns per swizzle atom
     static constexpr int NATOM = DH / ATOM_COLS;
     static constexpr int TILE_BYTES = 128 * DH * 2;           // one 128-row tile of Q, K or V
     static constexpr int ATOM_BYTES = 128 * SWB;
@@ -65,7 +71,7 @@ struct FwdCfg {
     static_assert(384 + DH <= 512, "forward TMEM columns: S0 0, S1 128, O0 256, O1 384");
 };
 
-// K-major descriptor of a [128 rows][DH] bf16 tile for K step kk (16 columns).
+// K-major descriptor of a [128 rows][DH] 16-bit tile for K step kk (16 columns).
 template <int DH>
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
     using C = FwdCfg<DH>;
@@ -205,8 +211,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         {
             const bool leader = elect_one();
             const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
-            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
+            constexpr uint32_t idS = idesc_f16(128, 128, false, false);
+            constexpr uint32_t idO = idesc_f16(128, DH, false, true);
             const uint32_t qbase = smem_u32(smem + C::OFF_Q);
             const uint64_t dQa = kmajor_desc<DH>(qbase, 0), dQb = kmajor_desc<DH>(qbase + C::TILE_BYTES, 0);
             int kcount = 0, vcount = 0, tcount = 0, item_iter = 0;
@@ -217,7 +223,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const uint64_t dQ0 = w ? dQb : dQa;
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk)
-                    umma_bf16(tmem + w * 128, desc_plus(dQ0, kmajor_off<DH>(kk)), desc_plus(dK0, kmajor_off<DH>(kk)),
+                    umma_ss(tmem + w * 128, desc_plus(dQ0, kmajor_off<DH>(kk)), desc_plus(dK0, kmajor_off<DH>(kk)),
                               idS, kk > 0);
                 umma_commit(&s_full[w]);
             };
@@ -251,7 +257,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                             // P_w sits in TMEM columns [128 w, 128 w + 64): 16 keys per 8 columns
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, desc_plus(dV0, mnmajor_off<DH>(kk)),
+                                umma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, desc_plus(dV0, mnmajor_off<DH>(kk)),
                                              idO, (j > 0 || kk > 0) ? 1u : 0u);
                             umma_commit(&o_done[w]);
                         }
@@ -361,10 +367,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 float ls[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ls[e] = 0.f;
-                const float neg_m = -m;
+                const float neg_m = kPOff - m;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    // 64 keys -> 32 TMEM columns of packed bf16 pairs (even key in the low half)
+                    // 64 keys -> 32 TMEM columns of packed fp16 pairs (even key in the low half)
                     float pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
@@ -373,7 +379,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         const float p1 = ex2(fmaf(s[k0 + 1], sl2, neg_m));
                         ls[(2 * c) & 7] += p0;
                         ls[(2 * c + 1) & 7] += p1;
-                        pk[c] = __uint_as_float(pack_bf16(p0, p1));
+                        pk[c] = __uint_as_float(pack_f16(p0, p1));
                     }
                     tmem_st32(s_addr + half * 32, pk);
                 }
@@ -387,7 +393,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!warp_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             const float inv = 1.0f / l;
-            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.o) + static_cast<int64_t>(lrow) * h + head * DH;
+            __half *orow = static_cast<__half *>(a.o) + static_cast<int64_t>(lrow) * h + head * DH;
 #pragma unroll 1
             for (int c = 0; c < DH / 32; ++c) {
                 float o[32];
@@ -397,14 +403,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint4 v;
-                    v.x = pack_bf16(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-                    v.y = pack_bf16(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-                    v.z = pack_bf16(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-                    v.w = pack_bf16(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+                    v.x = pack_f16(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+                    v.y = pack_f16(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+                    v.z = pack_f16(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+                    v.w = pack_f16(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
                     d[q] = v;
                 }
             }
-            a.lse[static_cast<int64_t>(head) * a.S + lrow] = m + __log2f(l);
+            // l sums the offset probabilities: log2(l) - kPOff is the true log-sum
+            a.lse[static_cast<int64_t>(head) * a.S + lrow] = m + (__log2f(l) - kPOff);
             tc_fence_before();
         }
     }
@@ -423,11 +430,11 @@ cudaError_t launch_fwd_impl(const AttnDesc &a, const DevErr &err, int num_sms, c
                                    : C::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                   : CU_TENSOR_MAP_SWIZZLE_32B;
     CUtensorMap mq, mk, mv;
-    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2,
+    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2,
                                    C::ATOM_COLS, 128, swz);
-    ok = ok && encode_tensor_map_2d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2,
+    ok = ok && encode_tensor_map_2d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2,
                                     C::ATOM_COLS, 128, swz);
-    ok = ok && encode_tensor_map_2d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, a.S, int64_t(h) * 2,
+    ok = ok && encode_tensor_map_2d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2,
                                     C::ATOM_COLS, 128, swz);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = attn_fwd_kernel<DH>;

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <cstdio>
@@ -24,6 +25,19 @@ struct DevErr {
     unsigned int *word;       // global error word (plan-owned)
     long long wait_limit;     // cycles a single wait may spin
 };
+
+// Bits of the error word.
+constexpr unsigned int kErrTimeout = 1u;  // a bounded wait ran out
+constexpr unsigned int kErrRange = 2u;    // a value did not fit an fp16 intermediate
+
+// fp16 holds magnitudes below 65520 (RNE rounds larger ones to infinity).
+constexpr float kF16Limit = 65520.0f;
+
+// Report an fp16 overflow: `maxabs` is the largest magnitude about to be
+// stored as fp16 by this thread.
+__device__ __forceinline__ void flag_range(float maxabs, unsigned int *word) {
+    if (maxabs >= kF16Limit && word) atomicOr(word, kErrRange);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -79,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (*abort) return false;
         if (clock64() - t0 > e.wait_limit) {
             *abort = 1;
-            atomicOr(e.word, 1u);
+            atomicOr(e.word, kErrTimeout);
             printf("tsp: bounded wait gave up (block %d thread %d smem bar 0x%x parity %u)\n", blockIdx.x,
                    threadIdx.x, smem_u32(bar), parity);
             return false;
@@ -147,16 +161,24 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 // carries out of the field.
 __device__ __forceinline__ uint64_t desc_plus(uint64_t d, uint32_t off) { return d + (off >> 4); }
 
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator.
-// a_mn / b_mn select MN-major operands (else K-major).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+// Instruction descriptor of kind::f16 with fp32 accumulator (bits 4-5 = 1)
+// and A, B both fp16 (format 0) or both bf16 (format 1, bits 7-9 and 10-12):
+// one MMA never mixes the two types.  a_mn / b_mn select MN-major operands
+// (else K-major).
+__host__ __device__ constexpr uint32_t idesc_mma(int M, int N, bool a_mn, bool b_mn, bool f16) {
+    return (1u << 4) | (f16 ? 0u : ((1u << 7) | (1u << 10))) | (static_cast<uint32_t>(a_mn) << 15) |
            (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
 }
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_mma(M, N, a_mn, b_mn, false);
+}
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_mma(M, N, a_mn, b_mn, true);
+}
 
 // D[tmem] (+)= A[smem] * B[smem], issued by one thread.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -166,8 +188,8 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 // D[tmem] (+)= A[tmem] * B[smem]: A (M rows in TMEM lanes, K along columns,
-// two bf16 per 32-bit column, the lower half holding the even element).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+// two 16-bit values per 32-bit column, the lower half holding the even element).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -298,6 +320,24 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+// fp16 pairs: RNE conversion from fp32, the even element in the low half.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float f16_lo(uint32_t v) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t v) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+}
+// Largest magnitude of 32 values (for flag_range before an fp16 store).
+__device__ __forceinline__ float maxabs32(const float (&v)[32]) {
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m[i & 3] = fmaxf(m[i & 3], fabsf(v[i]));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
 
 // GELU with the tanh approximation (Hendrycks & Gimpel 2016) and its
 // derivative, in fp32 via the CUDA tanhf.

@@ -1,6 +1,8 @@
 // Persistent tcgen05 GEMM for sm_100a with the layer's fused epilogues.
 //
-//   C[m, n] = sum_k A[m, k] * B[n, k]      bf16 operands, fp32 accumulator in TMEM
+//   C[m, n] = alpha * sum_k A[m, k] * B[n, k]
+//   fp16 (or bf16) operands, fp32 accumulator in TMEM; alpha is a device
+//   scalar, the power of two that undoes an operand's conversion scale.
 //
 // A is either K-major ([M][K] rows) or MN-major ([K][M] rows, i.e. A^T stored
 // row-major); the same for B.  The projections of the forward are K-major x
@@ -50,6 +52,9 @@ struct GemmArgs {
     int hsplit;
     void *out_k;
     void *out_v;
+    const float *alpha;
+    uint32_t idesc;  // instruction descriptor (operand type, majors, 128 x BN)
+    bool f16;        // fp16 operands, and fp16 for the "h" outputs of the epilogues
     DevErr err;
 };
 
@@ -95,6 +100,29 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&
         d[j] = w;
     }
 }
+// fp16 store of 32 values; an overflow is reported, not hidden.
+__device__ __forceinline__ void store_f16x32(__half *dst, const float (&v)[32], unsigned int *err) {
+    flag_range(maxabs32(v), err);
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 w;
+        w.x = pack_f16(v[8 * j + 0], v[8 * j + 1]);
+        w.y = pack_f16(v[8 * j + 2], v[8 * j + 3]);
+        w.z = pack_f16(v[8 * j + 4], v[8 * j + 5]);
+        w.w = pack_f16(v[8 * j + 6], v[8 * j + 7]);
+        d[j] = w;
+    }
+}
+// Store in the GEMM's operand type (fp16 or bf16).
+__device__ __forceinline__ void store_hx32(bool f16, void *base, int64_t off, const float (&v)[32],
+                                           unsigned int *err) {
+    if (f16)
+        store_f16x32(static_cast<__half *>(base) + off, v, err);
+    else
+        store_bf16x32(static_cast<__nv_bfloat16 *>(base) + off, v);
+}
+
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float (&v)[32]) {
     const uint4 *s = reinterpret_cast<const uint4 *>(src);
 #pragma unroll
@@ -112,65 +140,68 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float (&v
 }
 
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs &p, int row, int col, float (&v)[32]) {
+    const int64_t r = row;
     switch (p.epi) {
         case EPI_F32: {
-            float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + row * p.ldo + col);
+            float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + r * p.ldo + col);
 #pragma unroll
             for (int j = 0; j < 8; ++j) d[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             break;
         }
         case EPI_BF16:
-            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + row * p.ldo + col, v);
+            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + r * p.ldo + col, v);
+            break;
+        case EPI_F16:
+            store_f16x32(static_cast<__half *>(p.out) + r * p.ldo + col, v, p.err.word);
             break;
         case EPI_QKV: {
             int which = col / p.hsplit;
             int c = col - which * p.hsplit;
             if (which == 0) {
-                store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + row * p.ldo + c, v);
+                store_hx32(p.f16, p.out, r * p.ldo + c, v, p.err.word);
             } else {
-                int g = p.rowmap[row];
-                void *base = (which == 1) ? p.out_k : p.out_v;
-                store_bf16x32(static_cast<__nv_bfloat16 *>(base) + static_cast<int64_t>(g) * p.ldo + c, v);
+                const int64_t g = p.rowmap[row];
+                store_hx32(p.f16, which == 1 ? p.out_k : p.out_v, g * p.ldo + c, v, p.err.word);
             }
             break;
         }
         case EPI_RESID_F32: {
-            float r[32];
-            load_bf16x32(static_cast<const __nv_bfloat16 *>(p.aux) + row * p.ldaux + col, r);
-            float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + row * p.ldo + col);
+            float rs[32];
+            load_bf16x32(static_cast<const __nv_bfloat16 *>(p.aux) + r * p.ldaux + col, rs);
+            float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + r * p.ldo + col);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                d[j] = make_float4(v[4 * j] + r[4 * j], v[4 * j + 1] + r[4 * j + 1], v[4 * j + 2] + r[4 * j + 2],
-                                   v[4 * j + 3] + r[4 * j + 3]);
+                d[j] = make_float4(v[4 * j] + rs[4 * j], v[4 * j + 1] + rs[4 * j + 1], v[4 * j + 2] + rs[4 * j + 2],
+                                   v[4 * j + 3] + rs[4 * j + 3]);
             break;
         }
         case EPI_GELU: {
-            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + row * p.ldo + col, v);
+            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + r * p.ldo + col, v);
             float g[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) g[j] = gelu_tanh(v[j]);
-            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out2) + row * p.ldo2 + col, g);
+            store_hx32(p.f16, p.out2, r * p.ldo2 + col, g, p.err.word);
             break;
         }
         case EPI_RESID_BF16: {
-            const float4 *r = reinterpret_cast<const float4 *>(static_cast<const float *>(p.aux) + row * p.ldaux + col);
+            const float4 *q4 = reinterpret_cast<const float4 *>(static_cast<const float *>(p.aux) + r * p.ldaux + col);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                float4 q = r[j];
+                float4 q = q4[j];
                 v[4 * j] += q.x;
                 v[4 * j + 1] += q.y;
                 v[4 * j + 2] += q.z;
                 v[4 * j + 3] += q.w;
             }
-            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + row * p.ldo + col, v);
+            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + r * p.ldo + col, v);
             break;
         }
         case EPI_DGELU: {
             float u[32];
-            load_bf16x32(static_cast<const __nv_bfloat16 *>(p.aux) + row * p.ldaux + col, u);
+            load_bf16x32(static_cast<const __nv_bfloat16 *>(p.aux) + r * p.ldaux + col, u);
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] *= gelu_tanh_grad(u[j]);
-            store_bf16x32(static_cast<__nv_bfloat16 *>(p.out) + row * p.ldo + col, v);
+            store_hx32(p.f16, p.out, r * p.ldo + col, v, p.err.word);
             break;
         }
         default:
@@ -275,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+            const uint32_t idesc = p.idesc;
             int stage = 0;
             uint32_t phase = 0;
             uint32_t acc_phase[2] = {0, 0};
@@ -301,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            : sdesc(a + kk * 32, 16, 1024, kSwizzle128);
                         uint64_t bd = B_MN ? sdesc(b + kk * 2048, 64 * 128, 1024, kSwizzle128)
                                            : sdesc(b + kk * 32, 16, 1024, kSwizzle128);
-                        umma_bf16(d, ad, bd, idesc, (i | kk) != 0);
+                        umma_ss(d, ad, bd, idesc, (i | kk) != 0);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == C::STAGES) {
@@ -322,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Epilogue warps 2..5; TMEM lane quarter is fixed by warp % 4.
         const int quarter = warp & 3;
         const int row_in_tile = quarter * 32 + lane;
+        const float alpha = p.alpha ? *p.alpha : 1.0f;
         uint32_t acc_phase[2] = {0, 0};
         int tile_iter = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tile_iter) {
@@ -339,6 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[32];
                 tmem_ld32(base + c * 32, v);
                 tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= alpha;
                 epilogue_chunk(p, row, n0 + c * 32, v);
             }
             tc_fence_before();
@@ -352,19 +386,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-// Host: a 2D bf16 tensor map over a row-major [rows][cols] matrix with row
-// stride `ld` elements, box {64 columns, box_rows rows}, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
-    return encode_tensor_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cols, rows, ld * 2, 64, box_rows,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
+// Host: a 2D fp16 or bf16 tensor map over a row-major [rows][cols] matrix with
+// row stride `ld` elements, box {64 columns, box_rows rows}, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_rows, bool f16) {
+    return encode_tensor_map_2d(m, base, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                cols, rows, ld * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <int BN, bool A_MN, bool B_MN>
 cudaError_t launch_impl(const GemmDesc &g, const GemmArgs &p, int num_sms, cudaStream_t st) {
     using C = Cfg<BN>;
     CUtensorMap ma, mb;
-    bool ok = A_MN ? make_map(&ma, g.A, g.K, g.M, g.lda, 64) : make_map(&ma, g.A, g.M, g.K, g.lda, BM);
-    ok = ok && (B_MN ? make_map(&mb, g.B, g.K, g.N, g.ldb, 64) : make_map(&mb, g.B, g.N, g.K, g.ldb, BN));
+    bool ok = A_MN ? make_map(&ma, g.A, g.K, g.M, g.lda, 64, g.f16) : make_map(&ma, g.A, g.M, g.K, g.lda, BM, g.f16);
+    ok = ok && (B_MN ? make_map(&mb, g.B, g.K, g.N, g.ldb, 64, g.f16) : make_map(&mb, g.B, g.N, g.K, g.ldb, BN, g.f16));
     if (!ok) return cudaErrorInvalidValue;
     auto kern = gemm_kernel<BN, A_MN, B_MN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -396,9 +430,12 @@ cudaError_t launch_gemm(const GemmDesc &g, const DevErr &err, int num_sms, cudaS
     p.hsplit = g.hsplit > 0 ? g.hsplit : g.N;
     p.out_k = g.out_k;
     p.out_v = g.out_v;
+    p.alpha = g.alpha;
+    p.f16 = g.f16;
     p.err = err;
     const bool bn256 = (g.N % 256 == 0) && (g.epi != EPI_QKV || g.hsplit % 256 == 0) && !g.force_bn128;
     if (!bn256 && g.N % 128) return cudaErrorInvalidValue;
+    p.idesc = idesc_mma(BM, bn256 ? 256 : 128, g.a_mn, g.b_mn, g.f16);
     if (!g.a_mn && !g.b_mn)
         return bn256 ? launch_impl<256, false, false>(g, p, num_sms, st) : launch_impl<128, false, false>(g, p, num_sms, st);
     if (!g.a_mn && g.b_mn)

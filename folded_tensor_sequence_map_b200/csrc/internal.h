@@ -10,21 +10,26 @@ namespace tsp {
 
 struct DevErr;
 
-// Epilogues of the GEMM (row = thread's output row, acc = fp32 accumulator):
+// Epilogues of the GEMM (row = thread's output row, acc = fp32 accumulator
+// times the descriptor's alpha; "h" = the operand type of the GEMM: fp16 when
+// GemmDesc::f16, else bf16):
 enum GemmEpilogue : int {
     EPI_F32 = 0,        // out  f32[row][col] = acc
     EPI_BF16 = 1,       // out bf16[row][col] = acc
-    EPI_QKV = 2,        // col < h: out (Q) at local row; h..2h: out_k at rowmap[row]; 2h..3h: out_v likewise
+    EPI_QKV = 2,        // col < h: out (Q) at local row; h..2h: out_k at rowmap[row]; 2h..3h: out_v likewise (h)
     EPI_RESID_F32 = 3,  // out  f32 = acc + aux bf16 (residual)
-    EPI_GELU = 4,       // out bf16 = acc (pre-activation U), out2 bf16 = gelu_tanh(acc)
+    EPI_GELU = 4,       // out bf16 = acc (pre-activation U), out2 h = gelu_tanh(acc)
     EPI_RESID_BF16 = 5, // out bf16 = acc + aux f32 (residual)
-    EPI_DGELU = 6,      // out bf16 = acc * gelu_tanh'(aux bf16)
+    EPI_DGELU = 6,      // out h = acc * gelu_tanh'(aux bf16)
+    EPI_F16 = 7,        // out fp16[row][col] = acc
 };
 
 // C[M][N] = sum_k A[m][k] B[n][k].
 //   a_mn == false: A is [M][K] with row stride lda;  true: A is stored [K][M] (row stride lda).
 //   b_mn == false: B is [N][K] with row stride ldb;  true: B is stored [K][N] (row stride ldb).
 // M % 128 == 0, K % 64 == 0, N % 128 == 0, pointers 16-byte aligned.
+// A and B are both fp16 (f16) or both bf16.  Every fp16 store of an epilogue
+// checks for overflow and sets kErrRange in the error word.
 struct GemmDesc {
     const void *A;
     int64_t lda;
@@ -49,6 +54,8 @@ struct GemmDesc {
     void *out_k;
     void *out_v;
     bool force_bn128;
+    bool f16;            // operand type: fp16 (else bf16)
+    const float *alpha;  // device scalar multiplying the accumulator, or null for 1
 };
 
 cudaError_t launch_gemm(const GemmDesc &g, const DevErr &err, int num_sms, cudaStream_t st);
@@ -58,27 +65,73 @@ bool encode_tensor_map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType 
                           int64_t inner, int64_t outer, int64_t outer_stride_bytes, int box_inner, int box_outer,
                           CUtensorMapSwizzle swz);
 
-// RMSNorm forward: out bf16 = x * rstd * g, rstd = 1/sqrt(mean(x^2)+eps).
-// x is bf16 (x_f32 == nullptr) or f32.
-cudaError_t launch_rmsnorm_fwd(const void *x_bf16, const float *x_f32, const float *g, void *out, float *rstd,
-                               int rows, int h, cudaStream_t st);
+// RMSNorm forward: out = x * rstd * g, rstd = 1/sqrt(mean(x^2)+eps); out is
+// fp16 (overflow reported in err) or bf16 (out_f16 false).  x is bf16
+// (x_f32 == nullptr) or f32.
+cudaError_t launch_rmsnorm_fwd(const void *x_bf16, const float *x_f32, const float *g, void *out, bool out_f16,
+                               float *rstd, int rows, int h, unsigned int *err, cudaStream_t st);
 
 // RMSNorm backward plus residual:
-//   n = x*rstd, dn = dout*g, dx = resid + rstd*(dn - n*mean(dn*n)).
-// dout f32; x bf16 or f32; resid bf16 or f32; outputs dx_f32 and/or dx_bf16;
-// per-block partial sums of dout*n go to dg_partial[nblocks][h], and are
-// reduced (in block order) into dg.
-cudaError_t launch_rmsnorm_bwd(const float *dout, const void *x_bf16, const float *x_f32, const float *rstd,
-                               const float *g, const void *resid_bf16, const float *resid_f32, float *dx_f32,
-                               void *dx_bf16, float *dg_partial, float *dg, int rows, int h, cudaStream_t st);
+//   n = x*rstd, dn = dout*g, dx = (resid*rm + rstd*(dn - n*mean(dn*n))) * xm,
+//   dg = (sum over rows of dout*n) * gm,
+// with rm = *resid_mul, xm = *dx_mul, gm = *dg_mul (each 1 when null).
+// dout f32; x bf16 or f32; resid bf16 or f32; outputs dx_f32 and/or dx_low
+// (bf16, or fp16 when low_f16, overflow reported in err); per-block partial
+// sums of dout*n go to dg_partial[nblocks][h] and are reduced (in block order)
+// into dg.
+struct NormBwd {
+    const float *dout;
+    const void *x_bf16;
+    const float *x_f32;
+    const float *rstd;
+    const float *g;
+    const void *resid_bf16;
+    const float *resid_f32;
+    float *dx_f32;
+    void *dx_low;
+    bool low_f16;
+    float *dg_partial;
+    float *dg;
+    const float *resid_mul, *dx_mul, *dg_mul;
+    unsigned int *err;
+    int rows, h;
+};
+cudaError_t launch_rmsnorm_bwd(const NormBwd &n, cudaStream_t st);
 int rmsnorm_bwd_partial_blocks(int rows);
 
-// Attention.
+// bf16 -> fp16 conversion with a power-of-two scale taken from the tensor's
+// largest magnitude: dst = fp16(src * 2^e), e chosen so that max|src| * 2^e
+// lies in [2^(target-1), 2^target), so every element keeps fp16's full 11-bit
+// significand far above its subnormal range.  *scale_inv = 2^-e undoes it in
+// a consumer's epilogue; *scale = 2^e.  With target == kNoScale, e = 0 and a
+// magnitude fp16 cannot hold sets kErrRange.  Two launches for up to
+// kMaxConv tensors: block partial maxima, then the conversion (every block
+// reduces the partials itself, so no atomics and no clearing).
+constexpr int kNoScale = -1000;
+constexpr int kMaxConv = 5;
+constexpr int kConvBlocks = 296;  // blocks per tensor (2 per SM)
+struct ConvTensor {
+    const void *src;   // bf16, n elements, 16-byte aligned
+    void *dst;         // fp16, n elements
+    int64_t n;         // multiple of 8
+    int target;
+    float *scale_inv;  // may be null
+    float *scale;      // may be null
+};
+struct ConvBatch {
+    ConvTensor t[kMaxConv];
+    int count;
+    float *partial;    // kMaxConv * kConvBlocks floats of scratch
+    unsigned int *err;
+};
+cudaError_t launch_convert_f16(const ConvBatch &b, cudaStream_t st);
+
+// Attention.  Q, K, V, O (and dO, dQ, dK, dV in the backward) are fp16.
 struct AttnDesc {
     int S, L, D, H, dh, chunk;  // tokens, tokens per rank, ranks, heads, head dim, zigzag chunk
-    const void *q;              // bf16 [S][h] rank-major (local) rows
-    const void *k, *v;          // bf16 [S][h] global rows
-    void *o;                    // bf16 [S][h] local rows
+    const void *q;              // fp16 [S][h] rank-major (local) rows
+    const void *k, *v;          // fp16 [S][h] global rows
+    void *o;                    // fp16 [S][h] local rows
     float *lse;                 // f32 [H][S] local rows, log2 domain (scores pre-multiplied by log2 e / sqrt(dh))
     const int *order;           // pairs (qblock * H + head, number of 128-key tiles), longest first
     int num_items;
@@ -135,8 +188,9 @@ struct AttnBwdDesc {
     const void *q, *k, *v, *o, *dout;  // q, o, dout local rows; k, v global rows
     const float *lse;                  // as written by the forward
     float *delta;                      // f32 [H][S] scratch: rowsum(dO * O) per head, local rows
-    void *dq;                          // bf16, row stride ldd, local rows
-    void *dk, *dv;                     // bf16, row stride ldd, local rows of the key's owner
+    void *dq;                          // fp16, row stride ldd, local rows
+    void *dk, *dv;                     // fp16, row stride ldd, local rows of the key's owner
+    unsigned int *err;                 // error word (fp16 overflow of dQ, dK, dV)
     int64_t ldd;
     const int *inv_map;                // global position -> local row
     const int *kv_order;               // work order of (head, 128-key block), longest first

@@ -31,6 +31,9 @@ float *g_scratch_ptr[kMaxDevices] = {};
 // Device address of the scratch array on the current device, looked up once
 // per device with that device current.  In host code the array's name is only
 // a host-side stand-in, so the kernel must be given this address instead.
+// The address is cached for the life of the process: after cudaDeviceReset
+// on a device the cached value is stale, so this entry point must not be used
+// on a device that has been reset since its first call.
 tsp_status scratch_for_current_device(float **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return TSP_ERR_CUDA;
@@ -62,7 +65,18 @@ TSP_API tsp_status tsp_rmsnorm_backward_noalloc(const float *dout, const void *x
     if (st != TSP_OK) return st;
     // Every partial-sum slot the kernel reads is written by the same call, so
     // nothing has to be cleared between calls.
-    cudaError_t e = tsp::launch_rmsnorm_bwd(dout, x, nullptr, rstd, g, nullptr, resid, nullptr, dx, scratch, dg, rows,
-                                            h, static_cast<cudaStream_t>(stream));
+    tsp::NormBwd n{};
+    n.dout = dout;
+    n.x_bf16 = x;
+    n.rstd = rstd;
+    n.g = g;
+    n.resid_f32 = resid;
+    n.dx_low = dx;
+    n.low_f16 = false;
+    n.dg_partial = scratch;
+    n.dg = dg;
+    n.rows = rows;
+    n.h = h;
+    cudaError_t e = tsp::launch_rmsnorm_bwd(n, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
 }

@@ -1,8 +1,12 @@
 // RMSNorm forward and backward (memory-bound, fp32 arithmetic).
 //
-//   forward:  rstd = 1/sqrt(mean(x^2) + 1e-5),  out = x * rstd * g   (bf16 out)
+//   forward:  rstd = 1/sqrt(mean(x^2) + 1e-5),  out = x * rstd * g   (fp16 or bf16 out)
 //   backward: n = x*rstd, dn = dout*g,
 //             dx = resid + rstd * (dn - n * mean(dn*n)),  dg = sum_rows dout*n
+//
+// The backward takes optional power-of-two multipliers for the residual, for
+// dx and for dg: the layer's backward runs in a scaled gradient domain and
+// these carry values into and out of it exactly.
 //
 // The backward adds the residual branch's gradient (resid) so that one pass
 // produces the gradient of "x + f(RMSNorm(x))" w.r.t. x.  dg is reduced in two
@@ -24,10 +28,14 @@ __device__ __forceinline__ float4 load4(const void *p, int64_t idx) {
     return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
 }
 
+__device__ __forceinline__ uint2 pack4(bool f16, float a, float b, float c, float d) {
+    return f16 ? make_uint2(pack_f16(a, b), pack_f16(c, d)) : make_uint2(pack_bf16(a, b), pack_bf16(c, d));
+}
+
 // One warp per row.
 template <bool X_F32>
-__global__ void rmsnorm_fwd_kernel(const void *x, const float *g, __nv_bfloat16 *out, float *rstd_out, int rows,
-                                   int h) {
+__global__ void rmsnorm_fwd_kernel(const void *x, const float *g, void *out, bool out_f16, float *rstd_out, int rows,
+                                   int h, unsigned int *err) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (warp >= rows) return;
@@ -41,33 +49,37 @@ __global__ void rmsnorm_fwd_kernel(const void *x, const float *g, __nv_bfloat16 
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float r = rsqrtf(ss / static_cast<float>(h) + kEps);
     if (lane == 0) rstd_out[warp] = r;
+    float mx = 0.f;
     for (int c = lane * 4; c < h; c += 128) {
         float4 v = load4<X_F32>(x, base + c);
         float4 gg = *reinterpret_cast<const float4 *>(g + c);
-        uint2 w;
-        w.x = pack_bf16(v.x * r * gg.x, v.y * r * gg.y);
-        w.y = pack_bf16(v.z * r * gg.z, v.w * r * gg.w);
-        *reinterpret_cast<uint2 *>(out + base + c) = w;
+        const float a0 = v.x * r * gg.x, a1 = v.y * r * gg.y, a2 = v.z * r * gg.z, a3 = v.w * r * gg.w;
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fabsf(a2), fabsf(a3))));
+        *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(out) + base + c) = pack4(out_f16, a0, a1, a2, a3);
     }
+    if (out_f16) flag_range(mx, err);
 }
 
 template <bool X_F32, bool R_F32>
-__global__ void rmsnorm_bwd_kernel(const float *dout, const void *x, const float *rstd, const float *g,
-                                   const void *resid, float *dx_f32, __nv_bfloat16 *dx_bf16, float *dg_partial,
-                                   int rows, int h) {
+__global__ void rmsnorm_bwd_kernel(const NormBwd n) {
     __shared__ float s_mean[kBwdRows];
+    const int rows = n.rows, h = n.h;
+    const void *x = X_F32 ? static_cast<const void *>(n.x_f32) : n.x_bf16;
+    const void *resid = R_F32 ? static_cast<const void *>(n.resid_f32) : n.resid_bf16;
+    const float rm = n.resid_mul ? *n.resid_mul : 1.0f;
+    const float xm = n.dx_mul ? *n.dx_mul : 1.0f;
     const int row0 = blockIdx.x * kBwdRows;
     const int nrows = min(kBwdRows, rows - row0);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
     // Phase 1: mean(dn * n) of every row of the block.
     for (int i = warp; i < nrows; i += nwarps) {
         const int64_t base = static_cast<int64_t>(row0 + i) * h;
-        const float r = rstd[row0 + i];
+        const float r = n.rstd[row0 + i];
         float s = 0.f;
         for (int c = lane * 4; c < h; c += 128) {
-            float4 d = *reinterpret_cast<const float4 *>(dout + base + c);
+            float4 d = *reinterpret_cast<const float4 *>(n.dout + base + c);
             float4 v = load4<X_F32>(x, base + c);
-            float4 gg = *reinterpret_cast<const float4 *>(g + c);
+            float4 gg = *reinterpret_cast<const float4 *>(n.g + c);
             s += d.x * gg.x * v.x + d.y * gg.y * v.y + d.z * gg.z * v.z + d.w * gg.w * v.w;
         }
 #pragma unroll
@@ -76,84 +88,76 @@ __global__ void rmsnorm_bwd_kernel(const float *dout, const void *x, const float
     }
     __syncthreads();
     // Phase 2: column-parallel; every thread owns 4-column groups and walks the rows.
+    float mx = 0.f;
     for (int c = threadIdx.x * 4; c < h; c += blockDim.x * 4) {
-        float4 gg = *reinterpret_cast<const float4 *>(g + c);
+        float4 gg = *reinterpret_cast<const float4 *>(n.g + c);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int i = 0; i < nrows; ++i) {
             const int64_t idx = static_cast<int64_t>(row0 + i) * h + c;
-            const float r = rstd[row0 + i];
+            const float r = n.rstd[row0 + i];
             const float m = s_mean[i];
-            float4 d = *reinterpret_cast<const float4 *>(dout + idx);
+            float4 d = *reinterpret_cast<const float4 *>(n.dout + idx);
             float4 v = load4<X_F32>(x, idx);
             float4 rs = load4<R_F32>(resid, idx);
-            float4 n = make_float4(v.x * r, v.y * r, v.z * r, v.w * r);
+            float4 nn = make_float4(v.x * r, v.y * r, v.z * r, v.w * r);
             float4 o;
-            o.x = rs.x + r * (d.x * gg.x - n.x * m);
-            o.y = rs.y + r * (d.y * gg.y - n.y * m);
-            o.z = rs.z + r * (d.z * gg.z - n.z * m);
-            o.w = rs.w + r * (d.w * gg.w - n.w * m);
-            if (dx_f32) *reinterpret_cast<float4 *>(dx_f32 + idx) = o;
-            if (dx_bf16) {
-                uint2 w;
-                w.x = pack_bf16(o.x, o.y);
-                w.y = pack_bf16(o.z, o.w);
-                *reinterpret_cast<uint2 *>(dx_bf16 + idx) = w;
+            o.x = (rs.x * rm + r * (d.x * gg.x - nn.x * m)) * xm;
+            o.y = (rs.y * rm + r * (d.y * gg.y - nn.y * m)) * xm;
+            o.z = (rs.z * rm + r * (d.z * gg.z - nn.z * m)) * xm;
+            o.w = (rs.w * rm + r * (d.w * gg.w - nn.w * m)) * xm;
+            if (n.dx_f32) *reinterpret_cast<float4 *>(n.dx_f32 + idx) = o;
+            if (n.dx_low) {
+                if (n.low_f16) mx = fmaxf(mx, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
+                *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(n.dx_low) + idx) = pack4(n.low_f16, o.x, o.y, o.z, o.w);
             }
-            acc.x += d.x * n.x;
-            acc.y += d.y * n.y;
-            acc.z += d.z * n.z;
-            acc.w += d.w * n.w;
+            acc.x += d.x * nn.x;
+            acc.y += d.y * nn.y;
+            acc.z += d.z * nn.z;
+            acc.w += d.w * nn.w;
         }
-        *reinterpret_cast<float4 *>(dg_partial + static_cast<int64_t>(blockIdx.x) * h + c) = acc;
+        *reinterpret_cast<float4 *>(n.dg_partial + static_cast<int64_t>(blockIdx.x) * h + c) = acc;
     }
+    if (n.dx_low && n.low_f16) flag_range(mx, n.err);
 }
 
-__global__ void column_sum_kernel(const float *partial, float *out, int nblocks, int h) {
+__global__ void column_sum_kernel(const float *partial, float *out, const float *mul, int nblocks, int h) {
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= h) return;
     float s = 0.f;
     for (int b = 0; b < nblocks; ++b) s += partial[static_cast<int64_t>(b) * h + c];
-    out[c] = s;
+    out[c] = mul ? s * *mul : s;
 }
 
 }  // namespace
 
 int rmsnorm_bwd_partial_blocks(int rows) { return (rows + kBwdRows - 1) / kBwdRows; }
 
-cudaError_t launch_rmsnorm_fwd(const void *x_bf16, const float *x_f32, const float *g, void *out, float *rstd,
-                               int rows, int h, cudaStream_t st) {
+cudaError_t launch_rmsnorm_fwd(const void *x_bf16, const float *x_f32, const float *g, void *out, bool out_f16,
+                               float *rstd, int rows, int h, unsigned int *err, cudaStream_t st) {
     const int threads = 256;
     const int blocks = (rows * 32 + threads - 1) / threads;
     if (x_f32)
-        rmsnorm_fwd_kernel<true><<<blocks, threads, 0, st>>>(x_f32, g, static_cast<__nv_bfloat16 *>(out), rstd,
-                                                             rows, h);
+        rmsnorm_fwd_kernel<true><<<blocks, threads, 0, st>>>(x_f32, g, out, out_f16, rstd, rows, h, err);
     else
-        rmsnorm_fwd_kernel<false><<<blocks, threads, 0, st>>>(x_bf16, g, static_cast<__nv_bfloat16 *>(out), rstd,
-                                                              rows, h);
+        rmsnorm_fwd_kernel<false><<<blocks, threads, 0, st>>>(x_bf16, g, out, out_f16, rstd, rows, h, err);
     return cudaGetLastError();
 }
 
-cudaError_t launch_rmsnorm_bwd(const float *dout, const void *x_bf16, const float *x_f32, const float *rstd,
-                               const float *g, const void *resid_bf16, const float *resid_f32, float *dx_f32,
-                               void *dx_bf16, float *dg_partial, float *dg, int rows, int h, cudaStream_t st) {
-    const int nb = rmsnorm_bwd_partial_blocks(rows);
+cudaError_t launch_rmsnorm_bwd(const NormBwd &n, cudaStream_t st) {
+    const int nb = rmsnorm_bwd_partial_blocks(n.rows);
     const int threads = 256;
-    auto *dxb = static_cast<__nv_bfloat16 *>(dx_bf16);
-    if (x_f32 && !resid_f32)
-        rmsnorm_bwd_kernel<true, false><<<nb, threads, 0, st>>>(dout, x_f32, rstd, g, resid_bf16, dx_f32, dxb,
-                                                                dg_partial, rows, h);
-    else if (!x_f32 && resid_f32)
-        rmsnorm_bwd_kernel<false, true><<<nb, threads, 0, st>>>(dout, x_bf16, rstd, g, resid_f32, dx_f32, dxb,
-                                                                dg_partial, rows, h);
-    else if (x_f32 && resid_f32)
-        rmsnorm_bwd_kernel<true, true><<<nb, threads, 0, st>>>(dout, x_f32, rstd, g, resid_f32, dx_f32, dxb,
-                                                               dg_partial, rows, h);
+    const bool xf = n.x_f32 != nullptr, rf = n.resid_f32 != nullptr;
+    if (xf && !rf)
+        rmsnorm_bwd_kernel<true, false><<<nb, threads, 0, st>>>(n);
+    else if (!xf && rf)
+        rmsnorm_bwd_kernel<false, true><<<nb, threads, 0, st>>>(n);
+    else if (xf && rf)
+        rmsnorm_bwd_kernel<true, true><<<nb, threads, 0, st>>>(n);
     else
-        rmsnorm_bwd_kernel<false, false><<<nb, threads, 0, st>>>(dout, x_bf16, rstd, g, resid_bf16, dx_f32, dxb,
-                                                                 dg_partial, rows, h);
+        rmsnorm_bwd_kernel<false, false><<<nb, threads, 0, st>>>(n);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    column_sum_kernel<<<(h + 255) / 256, 256, 0, st>>>(dg_partial, dg, nb, h);
+    column_sum_kernel<<<(n.h + 255) / 256, 256, 0, st>>>(n.dg_partial, n.dg, n.dg_mul, nb, n.h);
     return cudaGetLastError();
 }
 

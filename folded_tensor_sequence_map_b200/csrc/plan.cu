@@ -50,10 +50,17 @@ constexpr size_t kAlign = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Byte layout of the saved-activation buffer and of the backward scratch.
+// fp16: a, q, k, v, o, b, g, the weight copies, du, dyh, dO, dqkv, dy16;
+// bf16: u; fp32: the rest.  `scales` holds the weight conversion scales
+// (kScaleInv + i = 2^-e_i, kScale + i = 2^e_i for wqkv, wo, w1, w2);
+// `gscales` the gradient scale of a backward call (2^-k, 2^k).
 struct Layout {
-    size_t rstd1, a, q, k, v, o, lse, y, rstd2, b, u, g, saved_total;
-    size_t du, db, dy, dyb, dO, delta, dqkv, da, dgp, bwd_total;
+    size_t rstd1, a, q, k, v, o, lse, y, rstd2, b, u, g, wqkv_h, wo_h, w1_h, w2_h, scales, cpart, saved_total;
+    size_t du, db, dy, dyh, dO, delta, dqkv, da, dgp, dy16, gscales, gpart, bwd_total;
 };
+constexpr int kScaleInv = 0, kScale = 8;
+constexpr int kTargetWeights = 12;  // largest |w| * 2^e in [2^11, 2^12)
+constexpr int kTargetGrad = 4;      // largest |dY| * 2^k in [2^3, 2^4)
 
 Layout layout_of(const tsp_plan_s *p) {
     Layout l{};
@@ -76,17 +83,26 @@ Layout layout_of(const tsp_plan_s *p) {
     l.b = take(S * h * 2);
     l.u = take(S * F * 2);
     l.g = take(S * F * 2);
+    l.wqkv_h = take(3 * h * h * 2);
+    l.wo_h = take(h * h * 2);
+    l.w1_h = take(F * h * 2);
+    l.w2_h = take(h * F * 2);
+    l.scales = take(64 * 4);
+    l.cpart = take(static_cast<size_t>(kMaxConv) * kConvBlocks * 4);
     l.saved_total = off;
     off = 0;
     l.du = take(S * F * 2);
     l.db = take(S * h * 4);
     l.dy = take(S * h * 4);
-    l.dyb = take(S * h * 2);
+    l.dyh = take(S * h * 2);
     l.dO = take(S * h * 2);
     l.delta = take(H * S * 4);
     l.dqkv = take(S * 3 * h * 2);
     l.da = take(S * h * 4);
     l.dgp = take(static_cast<size_t>(rmsnorm_bwd_partial_blocks(static_cast<int>(S))) * h * 4);
+    l.dy16 = take(S * h * 2);
+    l.gscales = take(64 * 4);
+    l.gpart = take(static_cast<size_t>(kMaxConv) * kConvBlocks * 4);
     l.bwd_total = off;
     return l;
 }
@@ -207,7 +223,7 @@ tsp_status check_pending_error(tsp_plan_s *p) {
     if (cudaMemcpy(&e, p->d_err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return TSP_ERR_CUDA;
     if (e) {
         cudaMemset(p->d_err, 0, sizeof(unsigned int));
-        return TSP_ERR_TIMEOUT;
+        return (e & kErrTimeout) ? TSP_ERR_TIMEOUT : TSP_ERR_RANGE;
     }
     return TSP_OK;
 }
@@ -284,11 +300,13 @@ const char *kStageNames[TSP_NUM_STAGES] = {
     "fwd_rmsnorm1", "fwd_qkv_gemm", "fwd_attention", "fwd_out_proj_gemm", "fwd_rmsnorm2", "fwd_w1_gelu_gemm",
     "fwd_w2_ring_gemm", "bwd_dgelu_gemm", "bwd_dw2_gemm", "bwd_dw1_gemm", "bwd_db_ring_gemm", "bwd_rmsnorm2",
     "bwd_do_gemm", "bwd_dwo_gemm", "bwd_attn_delta", "bwd_attn_dkdv", "bwd_attn_dq", "bwd_dwqkv_gemm",
-    "bwd_da_gemm", "bwd_rmsnorm1"};
+    "bwd_da_gemm", "bwd_rmsnorm1", "fwd_convert_weights", "bwd_convert_dy"};
 
 GemmDesc gemm(const void *A, int64_t lda, bool a_mn, const void *B, int64_t ldb, bool b_mn, int M, int N, int K,
-              int epi, void *out, int64_t ldo) {
+              int epi, void *out, int64_t ldo, const float *alpha = nullptr) {
     GemmDesc g{};
+    g.f16 = true;
+    g.alpha = alpha;
     g.A = A;
     g.lda = lda;
     g.a_mn = a_mn;
@@ -417,6 +435,7 @@ TSP_API const char *tsp_status_string(tsp_status s) {
         case TSP_ERR_ALIGNMENT: return "TSP_ERR_ALIGNMENT";
         case TSP_ERR_CUDA: return "TSP_ERR_CUDA";
         case TSP_ERR_TIMEOUT: return "TSP_ERR_TIMEOUT";
+        case TSP_ERR_RANGE: return "TSP_ERR_RANGE";
     }
     return "TSP_ERR_UNKNOWN";
 }
@@ -446,15 +465,28 @@ tsp_status forward_impl(tsp_plan_s *p, const void *x, const float *g1, const voi
     auto *yres = reinterpret_cast<float *>(base + l.y);
     auto *rstd2 = reinterpret_cast<float *>(base + l.rstd2);
     void *b = base + l.b, *u = base + l.u, *g = base + l.g;
+    void *wqkv_h = base + l.wqkv_h, *wo_h = base + l.wo_h, *w1_h = base + l.w1_h, *w2_h = base + l.w2_h;
+    auto *scales = reinterpret_cast<float *>(base + l.scales);
 
 #define TSP_STAGE(id, nk, call)                                                  \
     do {                                                                         \
         if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
             return TSP_ERR_CUDA;                                                 \
     } while (0)
-    TSP_STAGE(0, 1, launch_rmsnorm_fwd(x, nullptr, g1, a, rstd1, S, h, s));
+    // fp16 copies of the weights, each with its own power-of-two scale
+    ConvBatch cb{};
+    const void *wsrc[4] = {wqkv, wo, w1, w2};
+    void *wdst[4] = {wqkv_h, wo_h, w1_h, w2_h};
+    const int64_t wn[4] = {int64_t(3) * h * h, int64_t(h) * h, int64_t(F) * h, int64_t(h) * F};
+    for (int i = 0; i < 4; ++i)
+        cb.t[i] = ConvTensor{wsrc[i], wdst[i], wn[i], kTargetWeights, scales + kScaleInv + i, scales + kScale + i};
+    cb.count = 4;
+    cb.partial = reinterpret_cast<float *>(base + l.cpart);
+    cb.err = p->d_err;
+    TSP_STAGE(20, 2, launch_convert_f16(cb, s));
+    TSP_STAGE(0, 1, launch_rmsnorm_fwd(x, nullptr, g1, a, true, rstd1, S, h, p->d_err, s));
     // QKV projection over the broadcast attention shards; K/V land at global rows.
-    GemmDesc gq = gemm(a, h, false, wqkv, h, false, S, 3 * h, h, EPI_QKV, q, h);
+    GemmDesc gq = gemm(a, h, false, wqkv_h, h, false, S, 3 * h, h, EPI_QKV, q, h, scales + kScaleInv + 0);
     gq.rowmap = p->d_zig;
     gq.hsplit = h;
     gq.out_k = k;
@@ -476,17 +508,17 @@ tsp_status forward_impl(tsp_plan_s *p, const void *x, const float *g1, const voi
     ad.num_items = p->fwd_items;
     TSP_STAGE(2, 1, launch_attn_fwd(ad, err, p->num_sms, s));
     // out-projection (head-group partial sums in broadcast order) + residual, fp32 residual stream
-    GemmDesc go = gemm(o, h, false, wo, h, false, S, h, h, EPI_RESID_F32, yres, h);
+    GemmDesc go = gemm(o, h, false, wo_h, h, false, S, h, h, EPI_RESID_F32, yres, h, scales + kScaleInv + 1);
     go.aux = x;
     go.ldaux = h;
     TSP_STAGE(3, 1, launch_gemm(go, err, p->num_sms, s));
-    TSP_STAGE(4, 1, launch_rmsnorm_fwd(nullptr, yres, g2, b, rstd2, S, h, s));
-    GemmDesc g1d = gemm(b, h, false, w1, h, false, S, F, h, EPI_GELU, u, F);
+    TSP_STAGE(4, 1, launch_rmsnorm_fwd(nullptr, yres, g2, b, true, rstd2, S, h, p->d_err, s));
+    GemmDesc g1d = gemm(b, h, false, w1_h, h, false, S, F, h, EPI_GELU, u, F, scales + kScaleInv + 2);
     g1d.out2 = g;
     g1d.ldo2 = F;
     TSP_STAGE(5, 1, launch_gemm(g1d, err, p->num_sms, s));
     // W2 with the K loop over FFN shards in ring order (r + t) mod D, + residual
-    GemmDesc g2d = gemm(g, F, false, w2, F, false, S, h, F, EPI_RESID_BF16, y, h);
+    GemmDesc g2d = gemm(g, F, false, w2_h, F, false, S, h, F, EPI_RESID_BF16, y, h, scales + kScaleInv + 3);
     g2d.aux = yres;
     g2d.ldaux = h;
     g2d.ring_rows = L;
@@ -527,14 +559,40 @@ TSP_API tsp_status tsp_layer_prefill(tsp_plan_t p, const void *x, const float *g
                         static_cast<cudaStream_t>(stream));
 }
 
+// Scratch of the standalone ring MLP: U (bf16) and G (fp16) [S][F], the fp16
+// copies of b, W1 and W2, their scales and the conversion partials.
+struct RingLayout {
+    size_t u, g, b_h, w1_h, w2_h, scales, cpart, total;
+};
+RingLayout ring_layout(const tsp_plan_s *p) {
+    RingLayout r{};
+    const size_t S = p->S, h = p->h, F = p->F;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += up(bytes);
+        return o;
+    };
+    r.u = take(S * F * 2);
+    r.g = take(S * F * 2);
+    r.b_h = take(S * h * 2);
+    r.w1_h = take(F * h * 2);
+    r.w2_h = take(h * F * 2);
+    r.scales = take(64 * 4);
+    r.cpart = take(static_cast<size_t>(kMaxConv) * kConvBlocks * 4);
+    r.total = off;
+    return r;
+}
+
 TSP_API tsp_status tsp_ring_mlp_workspace_size(tsp_plan_t p, size_t *ws_bytes) {
     if (!p || !ws_bytes) return TSP_ERR_INVALID_ARG;
-    *ws_bytes = 2 * up(static_cast<size_t>(p->S) * static_cast<size_t>(p->F) * 2);  // U and G, bf16 [S][F]
+    *ws_bytes = ring_layout(p).total;
     return TSP_OK;
 }
 
-// The layer's W1 + GELU and W2 ring steps, launched exactly as the forward
-// launches them, on caller buffers.
+// The layer's W1 + GELU and W2 ring steps, launched as the forward launches
+// them, on caller buffers: b is copied to fp16 unscaled (like the layer's own
+// RMSNorm output), the weights with their power-of-two scales.
 TSP_API tsp_status tsp_ring_mlp_forward(tsp_plan_t p, const void *b, const void *w1, const void *w2, const float *resid,
                                         void *out, void *ws, void *stream) {
     if (!p || !b || !w1 || !w2 || !resid || !out || !ws) return TSP_ERR_INVALID_ARG;
@@ -545,19 +603,29 @@ TSP_API tsp_status tsp_ring_mlp_forward(tsp_plan_t p, const void *b, const void 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int S = static_cast<int>(p->S), h = p->h, F = p->F, L = static_cast<int>(p->L);
     const DevErr err = dev_err(p);
+    const RingLayout rl = ring_layout(p);
     uint8_t *base = static_cast<uint8_t *>(ws);
-    void *u = base, *g = base + up(static_cast<size_t>(S) * F * 2);
+    void *u = base + rl.u, *g = base + rl.g, *b_h = base + rl.b_h, *w1_h = base + rl.w1_h, *w2_h = base + rl.w2_h;
+    auto *scales = reinterpret_cast<float *>(base + rl.scales);
 #define TSP_STAGE(id, nk, call)                                                  \
     do {                                                                         \
         if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
             return TSP_ERR_CUDA;                                                 \
     } while (0)
-    GemmDesc g1d = gemm(b, h, false, w1, h, false, S, F, h, EPI_GELU, u, F);
+    ConvBatch cb{};
+    cb.t[0] = ConvTensor{b, b_h, int64_t(S) * h, kNoScale, nullptr, nullptr};
+    cb.t[1] = ConvTensor{w1, w1_h, int64_t(F) * h, kTargetWeights, scales + kScaleInv + 2, scales + kScale + 2};
+    cb.t[2] = ConvTensor{w2, w2_h, int64_t(h) * F, kTargetWeights, scales + kScaleInv + 3, scales + kScale + 3};
+    cb.count = 3;
+    cb.partial = reinterpret_cast<float *>(base + rl.cpart);
+    cb.err = p->d_err;
+    TSP_STAGE(20, 2, launch_convert_f16(cb, s));
+    GemmDesc g1d = gemm(b_h, h, false, w1_h, h, false, S, F, h, EPI_GELU, u, F, scales + kScaleInv + 2);
     g1d.out2 = g;
     g1d.ldo2 = F;
     TSP_STAGE(5, 1, launch_gemm(g1d, err, p->num_sms, s));
     // K loop over FFN shards in ring order (r + t) mod D for rank r's rows, + residual
-    GemmDesc g2d = gemm(g, F, false, w2, F, false, S, h, F, EPI_RESID_BF16, out, h);
+    GemmDesc g2d = gemm(g, F, false, w2_h, F, false, S, h, F, EPI_RESID_BF16, out, h, scales + kScaleInv + 3);
     g2d.aux = resid;
     g2d.ldaux = h;
     g2d.ring_rows = L;
@@ -586,40 +654,74 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     uint8_t *w = static_cast<uint8_t *>(ws);
     const int S = static_cast<int>(p->S), h = p->h, F = p->F, L = static_cast<int>(p->L);
     const DevErr err = dev_err(p);
+    (void)wqkv;
+    (void)wo;
+    (void)w1;
+    (void)w2;
     const float *rstd1 = reinterpret_cast<const float *>(sv + l.rstd1);
     const void *a = sv + l.a, *q = sv + l.q, *k = sv + l.k, *v = sv + l.v, *o = sv + l.o;
     const float *lse = reinterpret_cast<const float *>(sv + l.lse);
     const float *yres = reinterpret_cast<const float *>(sv + l.y);
     const float *rstd2 = reinterpret_cast<const float *>(sv + l.rstd2);
     const void *b = sv + l.b, *u = sv + l.u, *g = sv + l.g;
+    const void *wqkv_h = sv + l.wqkv_h, *wo_h = sv + l.wo_h, *w1_h = sv + l.w1_h, *w2_h = sv + l.w2_h;
+    const float *winv = reinterpret_cast<const float *>(sv + l.scales) + kScaleInv;
     void *du = w + l.du;
     float *db = reinterpret_cast<float *>(w + l.db);
     float *dyf = reinterpret_cast<float *>(w + l.dy);
-    void *dyb = w + l.dyb, *dO = w + l.dO, *dqkv = w + l.dqkv;
+    void *dyh = w + l.dyh, *dO = w + l.dO, *dqkv = w + l.dqkv, *dy16 = w + l.dy16;
     float *delta = reinterpret_cast<float *>(w + l.delta);
     float *da = reinterpret_cast<float *>(w + l.da);
     float *dgp = reinterpret_cast<float *>(w + l.dgp);
+    float *gsc = reinterpret_cast<float *>(w + l.gscales);
+    const float *ginv = gsc + 0;  // 2^-k: leaves the scaled gradient domain
+    const float *gmul = gsc + 1;  // 2^k: enters it
 #define TSP_STAGE(id, nk, call)                                                  \
     do {                                                                         \
         if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
             return TSP_ERR_CUDA;                                                 \
     } while (0)
+    // The backward is linear in dY: it runs on dY * 2^k, with 2^k taken from
+    // max|dY|, so gradients of any magnitude sit well inside fp16's range;
+    // the outputs leave the scaled domain exactly (times 2^-k).
+    ConvBatch cb{};
+    cb.t[0] = ConvTensor{dy, dy16, int64_t(S) * h, kTargetGrad, gsc + 0, gsc + 1};
+    cb.count = 1;
+    cb.partial = reinterpret_cast<float *>(w + l.gpart);
+    cb.err = p->d_err;
+    TSP_STAGE(21, 2, launch_convert_f16(cb, s));
     // MLP ring backward: dU = (dY W2) * GELU'(U); dW2 = dY^T G; dW1 = dU^T b; db = dU W1 (ring K order)
-    GemmDesc gdu = gemm(dy, h, false, w2, F, true, S, F, h, EPI_DGELU, du, F);
+    GemmDesc gdu = gemm(dy16, h, false, w2_h, F, true, S, F, h, EPI_DGELU, du, F, winv + 3);
     gdu.aux = u;
     gdu.ldaux = F;
     TSP_STAGE(7, 1, launch_gemm(gdu, err, p->num_sms, s));
-    TSP_STAGE(8, 1, launch_gemm(gemm(dy, h, true, g, F, true, h, F, S, EPI_F32, dw2, F), err, p->num_sms, s));
-    TSP_STAGE(9, 1, launch_gemm(gemm(du, F, true, b, h, true, F, h, S, EPI_F32, dw1, h), err, p->num_sms, s));
-    GemmDesc gdb = gemm(du, F, false, w1, h, true, S, h, F, EPI_F32, db, h);
+    TSP_STAGE(8, 1, launch_gemm(gemm(dy16, h, true, g, F, true, h, F, S, EPI_F32, dw2, F, ginv), err, p->num_sms, s));
+    TSP_STAGE(9, 1, launch_gemm(gemm(du, F, true, b, h, true, F, h, S, EPI_F32, dw1, h, ginv), err, p->num_sms, s));
+    GemmDesc gdb = gemm(du, F, false, w1_h, h, true, S, h, F, EPI_F32, db, h, winv + 2);
     gdb.ring_rows = L;
     gdb.ring_kblocks = (F / p->D) / 64;
     TSP_STAGE(10, 1, launch_gemm(gdb, err, p->num_sms, s));
-    // RMSNorm2 backward + residual: dy = dY + RMSNorm2^T(db)
-    TSP_STAGE(11, 2, launch_rmsnorm_bwd(db, nullptr, yres, rstd2, g2, dy, nullptr, dyf, dyb, dgp, dg2, S, h, s));
+    // RMSNorm2 backward + residual: dy = dY 2^k + RMSNorm2^T(db), fp32 and fp16 copies
+    NormBwd n2{};
+    n2.dout = db;
+    n2.x_f32 = yres;
+    n2.rstd = rstd2;
+    n2.g = g2;
+    n2.resid_bf16 = dy;
+    n2.dx_f32 = dyf;
+    n2.dx_low = dyh;
+    n2.low_f16 = true;
+    n2.dg_partial = dgp;
+    n2.dg = dg2;
+    n2.resid_mul = gmul;
+    n2.dg_mul = ginv;
+    n2.err = p->d_err;
+    n2.rows = S;
+    n2.h = h;
+    TSP_STAGE(11, 2, launch_rmsnorm_bwd(n2, s));
     // out-projection backward: dO = dy Wo, dWo = dy^T O
-    TSP_STAGE(12, 1, launch_gemm(gemm(dyb, h, false, wo, h, true, S, h, h, EPI_BF16, dO, h), err, p->num_sms, s));
-    TSP_STAGE(13, 1, launch_gemm(gemm(dyb, h, true, o, h, true, h, h, S, EPI_F32, dwo, h), err, p->num_sms, s));
+    TSP_STAGE(12, 1, launch_gemm(gemm(dyh, h, false, wo_h, h, true, S, h, h, EPI_F16, dO, h, winv + 1), err, p->num_sms, s));
+    TSP_STAGE(13, 1, launch_gemm(gemm(dyh, h, true, o, h, true, h, h, S, EPI_F32, dwo, h, ginv), err, p->num_sms, s));
     // attention backward; dK/dV reduced to the keys' owners
     AttnBwdDesc ab{};
     ab.S = S;
@@ -639,6 +741,7 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     ab.dk = static_cast<uint8_t *>(dqkv) + static_cast<size_t>(h) * 2;
     ab.dv = static_cast<uint8_t *>(dqkv) + static_cast<size_t>(2 * h) * 2;
     ab.ldd = 3 * h;
+    ab.err = p->d_err;
     ab.inv_map = p->d_inv;
     ab.kv_order = p->d_kv_order;
     ab.q_order = p->d_q_order;
@@ -646,10 +749,25 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     TSP_STAGE(15, 1, launch_attn_dkdv(ab, err, p->num_sms, s, p->d_zig));
     TSP_STAGE(16, 1, launch_attn_dq(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
     // projection backward: dWqkv = [dQ|dK|dV]^T a, da = [dQ|dK|dV] Wqkv
-    TSP_STAGE(17, 1, launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h), err, p->num_sms, s));
-    TSP_STAGE(18, 1, launch_gemm(gemm(dqkv, 3 * h, false, wqkv, h, true, S, h, 3 * h, EPI_F32, da, h), err, p->num_sms, s));
-    // RMSNorm1 backward + residual: dx = dy + RMSNorm1^T(da)
-    TSP_STAGE(19, 2, launch_rmsnorm_bwd(da, x, nullptr, rstd1, g1, nullptr, dyf, nullptr, dx, dgp, dg1, S, h, s));
+    TSP_STAGE(17, 1, launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h, ginv), err, p->num_sms, s));
+    TSP_STAGE(18, 1, launch_gemm(gemm(dqkv, 3 * h, false, wqkv_h, h, true, S, h, 3 * h, EPI_F32, da, h, winv + 0), err, p->num_sms, s));
+    // RMSNorm1 backward + residual: dx = (dy + RMSNorm1^T(da)) 2^-k
+    NormBwd n1{};
+    n1.dout = da;
+    n1.x_bf16 = x;
+    n1.rstd = rstd1;
+    n1.g = g1;
+    n1.resid_f32 = dyf;
+    n1.dx_low = dx;
+    n1.low_f16 = false;
+    n1.dg_partial = dgp;
+    n1.dg = dg1;
+    n1.dx_mul = ginv;
+    n1.dg_mul = ginv;
+    n1.err = p->d_err;
+    n1.rows = S;
+    n1.h = h;
+    TSP_STAGE(19, 2, launch_rmsnorm_bwd(n1, s));
 #undef TSP_STAGE
     return TSP_OK;
 }
@@ -659,7 +777,7 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
 // ===========================================================================
 
 TSP_API tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A, int64_t lda, const void *B,
-                                 int64_t ldb, float *C, int64_t ldc, int force_bn128, void *stream) {
+                                 int64_t ldb, float *C, int64_t ldc, int force_bn128, int f16, void *stream) {
     if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0) return TSP_ERR_INVALID_ARG;
     if (M % 128 || N % 128 || K % 64) return TSP_ERR_UNSUPPORTED;
     if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return TSP_ERR_ALIGNMENT;
@@ -673,6 +791,7 @@ TSP_API tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const 
     }
     GemmDesc g = gemm(A, lda, a_mn != 0, B, ldb, b_mn != 0, M, N, K, EPI_F32, C, ldc);
     g.force_bn128 = force_bn128 != 0;
+    g.f16 = f16 != 0;
     return cuda_status(launch_gemm(g, DevErr{d_err, 4000000000LL}, sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -684,8 +803,10 @@ TSP_API tsp_status tsp_test_buffer_offset(tsp_plan_t p, const char *name, size_t
         size_t o;
     } tab[] = {{"rstd1", l.rstd1}, {"a", l.a},   {"q", l.q},         {"k", l.k},     {"v", l.v},
                {"o", l.o},         {"lse", l.lse}, {"y", l.y},       {"rstd2", l.rstd2}, {"b", l.b},
-               {"u", l.u},         {"g", l.g},   {"ws.du", l.du},    {"ws.db", l.db}, {"ws.dy", l.dy},
-               {"ws.dO", l.dO},    {"ws.delta", l.delta}, {"ws.dqkv", l.dqkv}, {"ws.da", l.da}};
+               {"u", l.u},         {"g", l.g},   {"wqkv_h", l.wqkv_h}, {"wo_h", l.wo_h}, {"w1_h", l.w1_h},
+               {"w2_h", l.w2_h},   {"scales", l.scales}, {"ws.du", l.du}, {"ws.db", l.db}, {"ws.dy", l.dy},
+               {"ws.dyh", l.dyh},  {"ws.dO", l.dO}, {"ws.delta", l.delta}, {"ws.dqkv", l.dqkv}, {"ws.da", l.da},
+               {"ws.dy16", l.dy16}, {"ws.gscales", l.gscales}};
     for (auto &t : tab)
         if (std::strcmp(t.n, name) == 0) {
             *offset = t.o;

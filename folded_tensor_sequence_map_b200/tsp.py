@@ -26,6 +26,7 @@ STATUS_NAMES = {
     4: "TSP_ERR_ALIGNMENT",
     5: "TSP_ERR_CUDA",
     6: "TSP_ERR_TIMEOUT",
+    7: "TSP_ERR_RANGE",
 }
 
 EXPORTED = (
@@ -53,7 +54,7 @@ EXPORTED = (
     "tsp_test_tables",
     "tsp_test_wait_timeout",
 )
-TSP_NUM_STAGES = 20
+TSP_NUM_STAGES = 22
 
 
 class TSPError(RuntimeError):
@@ -93,7 +94,7 @@ def _load() -> ctypes.CDLL:
     lib.tsp_status_string.restype = ctypes.c_char_p
     lib.tsp_layer_flops.argtypes = [P, I]
     lib.tsp_layer_flops.restype = ctypes.c_double
-    lib.tsp_test_gemm.argtypes = [I, I, I, I, I, V, I64, V, I64, V, I64, I, V]
+    lib.tsp_test_gemm.argtypes = [I, I, I, I, I, V, I64, V, I64, V, I64, I, I, V]
     lib.tsp_test_gemm.restype = I
     lib.tsp_test_buffer_offset.argtypes = [P, ctypes.c_char_p, ctypes.POINTER(SZ)]
     lib.tsp_test_buffer_offset.restype = I
@@ -238,8 +239,8 @@ def tsp_layer_prefill(plan: Plan, x, g1, wqkv, wo, g2, w1, w2, y, k_cache, v_cac
         _ptr(w1, "w1", bf, (F, h)),
         _ptr(w2, "w2", bf, (h, F)),
         _ptr(y, "y", bf, (S, h)),
-        _ptr(k_cache, "k_cache", bf, (S, h)),
-        _ptr(v_cache, "v_cache", bf, (S, h)),
+        _ptr(k_cache, "k_cache", torch.float16, (S, h)),
+        _ptr(v_cache, "v_cache", torch.float16, (S, h)),
         _ptr(ws, "ws"),
         _stream(stream),
     ]
@@ -335,9 +336,9 @@ def tsp_rmsnorm_backward_noalloc(dout, x, rstd, g, resid, dx, dg, rows: int, h: 
 # ---- test hooks --------------------------------------------------------------
 
 def tsp_test_gemm(a_mn: bool, b_mn: bool, M: int, N: int, K: int, A, lda: int, B, ldb: int, C, ldc: int,
-                  force_bn128: bool = False, stream=None) -> None:
+                  force_bn128: bool = False, stream=None, f16: bool = False) -> None:
     _check(_lib.tsp_test_gemm(int(a_mn), int(b_mn), M, N, K, _ptr(A, "A"), lda, _ptr(B, "B"), ldb, _ptr(C, "C"),
-                              ldc, int(force_bn128), _stream(stream)), "tsp_test_gemm")
+                              ldc, int(force_bn128), int(bool(f16)), _stream(stream)), "tsp_test_gemm")
 
 
 def tsp_test_buffer_offset(plan: Plan, name: str) -> int:

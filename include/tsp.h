@@ -36,8 +36,20 @@
  *   - Layer calls are asynchronous on `stream` (a cudaStream_t, may be 0).
  *     Argument errors are reported synchronously and enqueue nothing.
  *   - A bounded device-side wait that ran out sets a flag in the plan; it is
- *     reported as TSP_ERR_TIMEOUT by tsp_sync_status() and by the next layer
- *     call.  Kernels never spin without a limit.
+ *     reported as TSP_ERR_TIMEOUT by tsp_sync_status() (layer calls do not
+ *     read it: that would block on the device).  Kernels never spin without
+ *     a limit.
+ *   - Arithmetic: inputs and the outputs y, dx are bf16, gradients of weights
+ *     and gains fp32.  Every tensor-core operand the layer computes itself
+ *     (a, Q, K, V, P, O, b, GELU output, and the backward's dU, dy, dO, dS,
+ *     dQ, dK, dV) is stored as fp16, whose rounding is 8x finer than bf16's,
+ *     and multiplied in fp16 x fp16 MMAs at the same rate, with fp32
+ *     accumulation.  bf16 weights and dY enter as exact fp16 copies scaled by
+ *     powers of two chosen from their largest magnitudes (the scales are
+ *     undone exactly in the epilogues); the backward runs on dY times such a
+ *     power of two, so gradients of any magnitude sit inside fp16's range.  A
+ *     value too large for an fp16 intermediate sets a flag in the plan,
+ *     reported as TSP_ERR_RANGE by tsp_sync_status().
  */
 #ifndef TSP_H
 #define TSP_H
@@ -58,7 +70,8 @@ typedef enum {
     TSP_ERR_UNSUPPORTED = 3, /* shape outside the kernels' tiling, or device is not sm_100 */
     TSP_ERR_ALIGNMENT = 4,   /* a device pointer is not 16-byte aligned */
     TSP_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
-    TSP_ERR_TIMEOUT = 6      /* a bounded device-side wait expired */
+    TSP_ERR_TIMEOUT = 6,     /* a bounded device-side wait expired */
+    TSP_ERR_RANGE = 7        /* a computed value overflowed its fp16 intermediate (|v| >= 65520) */
 } tsp_status;
 
 /* Build a plan for one layer: hidden size h, `heads` attention heads (head size
@@ -114,8 +127,9 @@ tsp_status tsp_workspace_size(tsp_plan_t plan, int training, size_t *ws_bytes, s
  * out-projection with head-group partial sums in broadcast order plus the
  * residual; RMSNorm2; W1 with GELU; W2 with its K loop over FFN shards in ring
  * order (r+t) mod D, partial sums in the rank's fp32 accumulator, plus the
- * residual.  bf16 tensor-core operands, fp32 accumulation, fp32 residual
- * stream. */
+ * residual.  fp16 tensor-core operands (see Arithmetic above), fp32
+ * accumulation, fp32 residual stream.  With `saved`, the fp16 weight copies
+ * are kept there for tsp_layer_backward. */
 tsp_status tsp_layer_forward(tsp_plan_t plan, const void *x, const float *g1, const void *wqkv,
                              const void *wo, const float *g2, const void *w1, const void *w2,
                              void *y, void *saved, void *ws, void *stream);
@@ -126,7 +140,7 @@ tsp_status tsp_layer_forward(tsp_plan_t plan, const void *x, const float *g1, co
  * method's benefits to inference; this is the forward run for that use.
  * Device pointers:
  *   x, g1, wqkv, wo, g2, w1, w2, y  as for tsp_layer_forward
- *   k_cache, v_cache  bf16 [S][h] each (outputs, owned by the caller): the
+ *   k_cache, v_cache  fp16 [S][h] each (outputs, owned by the caller): the
  *       keys and values of all S tokens in GLOBAL position order (row p =
  *       token at position p, the all-gathered layout), head n in columns
  *       [n*dh, (n+1)*dh).  The attention of this call reads them there.
@@ -150,11 +164,13 @@ tsp_status tsp_layer_prefill(tsp_plan_t plan, const void *x, const float *g1, co
  *   out_r = resid_r + sum_{t=0}^{D-1} GELU_tanh(b_r W1[s_t]^T) W2[:, s_t]^T,
  *   s_t = (r + t) mod D (FFN shard s_t = units [s_t*F/D, (s_t+1)*F/D)),
  * the partial sums staying in the rank's fp32 accumulator.  Device pointers:
- *   b      bf16 [S][h], rank-major (input, the normalised activations)
- *   w1     bf16 [F][h]; w2 bf16 [h][F] (inputs)
+ *   b      bf16 [S][h], rank-major (input, the normalised activations; copied
+ *          to fp16 unscaled, so |b| must stay below 65520: TSP_ERR_RANGE)
+ *   w1     bf16 [F][h]; w2 bf16 [h][F] (inputs, copied to scaled fp16)
  *   resid  float32 [S][h], rank-major (input; pass zeros for no residual)
  *   out    bf16 [S][h], rank-major (output)
- *   ws     tsp_ring_mlp_workspace_size bytes of scratch (holds U and G)
+ *   ws     tsp_ring_mlp_workspace_size bytes of scratch (holds U, G and the
+ *          fp16 copies)
  * Errors: TSP_ERR_INVALID_ARG for a NULL pointer, TSP_ERR_ALIGNMENT unless
  * every pointer is 16-byte aligned (both before anything is enqueued),
  * TSP_ERR_UNSUPPORTED off sm_100, TSP_ERR_CUDA for a failed launch. */
@@ -168,7 +184,8 @@ tsp_status tsp_ring_mlp_forward(tsp_plan_t plan, const void *b, const void *w1, 
  * gradients are summed over every rank's queries and written back at the
  * owning rank's rows).  Device pointers:
  *   dy   bf16 [S][h] upstream gradient of the layer output, rank-major order
- *   x, g1, wqkv, wo, g2, w1, w2  the forward's inputs
+ *   x, g1, wqkv, wo, g2, w1, w2  the forward's inputs (the weights' fp16
+ *          copies that the forward kept in `saved` are what the MMAs read)
  *   saved  the buffer filled by tsp_layer_forward with the same inputs
  *   ws     ws_bytes of scratch
  * Outputs: dx bf16 [S][h] rank-major order; dg1, dg2 float32 [h];
@@ -180,16 +197,20 @@ tsp_status tsp_layer_backward(tsp_plan_t plan, const void *dy, const void *x, co
                               float *dwqkv, float *dwo, float *dg2, float *dw1, float *dw2,
                               void *stream);
 
-/* Wait for `stream`, then report TSP_ERR_CUDA for an asynchronous CUDA error
- * or TSP_ERR_TIMEOUT if a device-side wait of this plan ran out (the flag is
- * cleared by the report). */
+/* Wait for `stream`, then report TSP_ERR_CUDA for an asynchronous CUDA error,
+ * TSP_ERR_TIMEOUT if a device-side wait of this plan ran out, or TSP_ERR_RANGE
+ * if a value overflowed an fp16 intermediate (the flags are cleared by the
+ * report). */
 tsp_status tsp_sync_status(tsp_plan_t plan, void *stream);
 
 /* Static, human-readable name of a status. */
 const char *tsp_status_string(tsp_status status);
 
-/* Kernel stages of one forward + backward, in launch order (profiling ids). */
-#define TSP_NUM_STAGES 20
+/* Kernel stages of one forward + backward (profiling ids): 0-6 the forward
+ * and 7-19 the backward in launch order; 20 the forward's weight conversion
+ * (first in the forward) and 21 the backward's dY conversion (first in the
+ * backward). */
+#define TSP_NUM_STAGES 22
 
 /* Per-stage timing with CUDA events.  tsp_profile_enable(plan, 1) clears the
  * record and starts bracketing every stage of later layer calls with a pair of
@@ -202,7 +223,7 @@ tsp_status tsp_profile_read(tsp_plan_t plan, int stage, const char **name, doubl
                             int64_t *kernel_launches);
 
 /* Kernels this plan has launched since it was created (every layer call adds
- * 7 for a forward and 15 for a backward). */
+ * 9 for a forward and 17 for a backward). */
 int64_t tsp_kernel_launches(tsp_plan_t plan);
 
 /* RMSNorm backward plus residual that allocates nothing.  The TSP pages have

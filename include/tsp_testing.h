@@ -19,21 +19,28 @@ extern "C" {
 #endif
 
 /* C[M][N] (float32, row stride ldc) = sum_k A[m][k] * B[n][k] with the layer's
- * tcgen05 GEMM kernel, bf16 operands, fp32 accumulation.
- *   a_mn == 0: A is bf16 [M][K] (row stride lda); a_mn != 0: A is stored [K][M].
- *   b_mn == 0: B is bf16 [N][K] (row stride ldb); b_mn != 0: B is stored [K][N].
+ * tcgen05 GEMM kernel, fp32 accumulation; A and B are both bf16 (f16 == 0) or
+ * both fp16 (f16 != 0).
+ *   a_mn == 0: A is [M][K] (row stride lda); a_mn != 0: A is stored [K][M].
+ *   b_mn == 0: B is [N][K] (row stride ldb); b_mn != 0: B is stored [K][N].
  * M % 128 == 0, N % 128 == 0, K % 64 == 0 (TSP_ERR_UNSUPPORTED otherwise);
  * device pointers, 16-byte aligned.  force_bn128 != 0 selects the 128-column
  * tile even where the 256-column tile applies.  Asynchronous on `stream`. */
 tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A, int64_t lda, const void *B,
-                         int64_t ldb, float *C, int64_t ldc, int force_bn128, void *stream);
+                         int64_t ldb, float *C, int64_t ldc, int force_bn128, int f16, void *stream);
 
 /* Byte offset of a named intermediate inside the `saved` buffer (names: rstd1,
- * a, q, k, v, o, lse, y, rstd2, b, u, g) or, with a "ws." prefix, inside the
- * backward scratch (ws.du, ws.db, ws.dy, ws.dO, ws.delta, ws.dqkv, ws.da).
- * Layouts: a, q, o, b bf16 [S][h] local rows; k, v bf16 [S][h] global rows;
- * y f32 [S][h]; u, g bf16 [S][F]; lse f32 [H][S] in log2 units (scores times
- * log2(e)/sqrt(dh)); rstd f32 [S].  TSP_ERR_INVALID_ARG for an unknown name. */
+ * a, q, k, v, o, lse, y, rstd2, b, u, g, wqkv_h, wo_h, w1_h, w2_h, scales) or,
+ * with a "ws." prefix, inside the backward scratch (ws.du, ws.db, ws.dy,
+ * ws.dyh, ws.dO, ws.delta, ws.dqkv, ws.da, ws.dy16, ws.gscales).
+ * Layouts: a, q, o, b fp16 [S][h] local rows; k, v fp16 [S][h] global rows;
+ * y f32 [S][h]; u bf16 [S][F]; g fp16 [S][F]; lse f32 [H][S] in log2 units
+ * (scores times log2(e)/sqrt(dh)); rstd f32 [S]; the *_h weight copies fp16,
+ * each the bf16 weight times 2^e_i; scales f32: [0..3] = 2^-e_i and
+ * [8..11] = 2^e_i for wqkv, wo, w1, w2.  The backward's gradients (ws.du,
+ * ws.db, ws.dy, ws.dyh, ws.dO, ws.dqkv, ws.da, ws.dy16) are those of the
+ * layer times 2^k, with ws.gscales f32 [0] = 2^-k and [1] = 2^k.
+ * TSP_ERR_INVALID_ARG for an unknown name. */
 tsp_status tsp_test_buffer_offset(tsp_plan_t plan, const char *name, size_t *offset);
 
 /* Host evaluation of the rule the dK/dV kernel uses to walk the 64-row query

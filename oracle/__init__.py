@@ -7,3 +7,4 @@ It shares no code with the CUDA library.
 """
 
 from .tsp_oracle import *  # noqa: F401,F403
+from .long_sequence import layer_forward_backward_blocked  # noqa: F401

@@ -23,6 +23,7 @@ heads; every weight uses the ``[out, in]`` row-major layout of a linear layer.
 
 from __future__ import annotations
 
+import hashlib
 from dataclasses import dataclass
 
 import numpy as np
@@ -97,3 +98,12 @@ def sample_rows(S: int, n: int, seed: int) -> np.ndarray:
     if len(rows) > 1:
         rows[1] = S - 1
     return np.unique(rows)
+
+
+def input_hash(inp: dict) -> str:
+    """sha256 of the bf16 bit patterns of x, Wqkv, Wo, W1, W2 and dY, in that
+    order: identifies the inputs that a stored expected value belongs to."""
+    hsh = hashlib.sha256()
+    for k in ("x", "wqkv", "wo", "w1", "w2", "dy"):
+        hsh.update(np.ascontiguousarray(inp[k]).tobytes())
+    return hsh.hexdigest()

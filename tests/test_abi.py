@@ -149,10 +149,12 @@ def test_prefill_checks_arguments_before_enqueueing():
 
 
 def test_ring_mlp_workspace_and_argument_checks():
-    """Scratch for U and G (bf16 [S][F] each, 256-byte aligned pieces); NULL or
-    misaligned pointers are refused before anything is enqueued."""
+    """Scratch for U and G ([S][F] each), the fp16 copies of b [S][h], W1 and W2
+    [F][h] each, and the scales (256-byte aligned pieces); NULL or misaligned
+    pointers are refused before anything is enqueued."""
     p = T.tsp_plan(128, 4, 512, 256, 2)
-    assert T.tsp_ring_mlp_workspace_size(p) == 2 * 256 * 512 * 2
+    S, h, F = 256, 128, 512
+    assert T.tsp_ring_mlp_workspace_size(p) >= 2 * S * F * 2 + S * h * 2 + 2 * F * h * 2 + 64 * 4
     good = [0x10000 * (i + 1) for i in range(6)]
     for i in range(6):
         args = list(good)
@@ -185,9 +187,11 @@ def test_workspace_sizes_cover_the_layout():
     ws_i, saved_i = T.tsp_workspace_size(p, False)
     S, h, F, H = 256, 128, 512, 4
     assert saved_i == 0 and ws_i == saved_t
-    assert saved_t >= S * h * 2 * 6 + S * h * 4 + S * F * 2 * 2 + H * S * 4 + 2 * S * 4
-    assert ws_t >= S * F * 2 + S * h * (4 + 4 + 2 + 2 + 4) + S * 3 * h * 2
-    names = ["rstd1", "a", "q", "k", "v", "o", "lse", "y", "rstd2", "b", "u", "g"]
+    weights = (3 * h * h + h * h + 2 * F * h) * 2
+    assert saved_t >= S * h * 2 * 6 + S * h * 4 + S * F * 2 * 2 + H * S * 4 + 2 * S * 4 + weights
+    assert ws_t >= S * F * 2 + S * h * (4 + 4 + 2 + 2 + 4 + 2) + S * 3 * h * 2
+    names = ["rstd1", "a", "q", "k", "v", "o", "lse", "y", "rstd2", "b", "u", "g", "wqkv_h", "wo_h", "w1_h",
+             "w2_h", "scales"]
     offs = [T.tsp_test_buffer_offset(p, n) for n in names]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and offs[-1] < saved_t
     with pytest.raises(T.TSPError):

@@ -1,6 +1,6 @@
 """The tcgen05 GEMM kernel through its test hook: every operand-major
-combination and both tile widths against an fp64 product of the same bf16
-operands (plus fp32-accumulation rounding)."""
+combination, both tile widths and both operand types (bf16, fp16) against an
+fp64 product of the same operands (plus fp32-accumulation rounding)."""
 
 import numpy as np
 import pytest
@@ -11,22 +11,24 @@ pytestmark = pytest.mark.gpu
 import folded_tensor_sequence_map_b200 as T
 
 
-def _bf16(shape, seed):
+def _bf16(shape, seed, dtype=torch.bfloat16):
     g = torch.Generator().manual_seed(seed)
-    return torch.randn(*shape, generator=g).to(torch.bfloat16)
+    return torch.randn(*shape, generator=g).to(dtype)
 
 
+@pytest.mark.parametrize("f16", [False, True])
 @pytest.mark.parametrize("a_mn,b_mn", [(False, False), (False, True), (True, True), (True, False)])
 @pytest.mark.parametrize("M,N,K,bn128", [(128, 128, 64, False), (256, 256, 192, False), (384, 512, 1024, False),
                                          (256, 384, 320, True), (1024, 768, 512, True)])
-def test_gemm_matches_fp64(a_mn, b_mn, M, N, K, bn128):
-    A = _bf16((K, M) if a_mn else (M, K), 1)
-    B = _bf16((K, N) if b_mn else (N, K), 2)
+def test_gemm_matches_fp64(a_mn, b_mn, M, N, K, bn128, f16):
+    dt = torch.float16 if f16 else torch.bfloat16
+    A = _bf16((K, M) if a_mn else (M, K), 1, dt)
+    B = _bf16((K, N) if b_mn else (N, K), 2, dt)
     Am = A.double().T if a_mn else A.double()
     Bm = B.double() if b_mn else B.double().T
     ref = (Am @ Bm).numpy()
     C = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
-    T.tsp_test_gemm(a_mn, b_mn, M, N, K, A.cuda(), A.shape[1], B.cuda(), B.shape[1], C, N, bn128)
+    T.tsp_test_gemm(a_mn, b_mn, M, N, K, A.cuda(), A.shape[1], B.cuda(), B.shape[1], C, N, bn128, f16=f16)
     torch.cuda.synchronize()
     got = C.cpu().double().numpy()
     err = np.abs(got - ref).max() / np.abs(ref).max()

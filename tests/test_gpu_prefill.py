@@ -22,15 +22,15 @@ def test_prefill_matches_forward_and_fills_caches(workload):
     layer = GpuLayer(shape, inp, training=True)
     S, h = shape.S, shape.h
     y_fwd = layer.forward().clone()
-    k_fwd = layer.saved_view("k", (S, h), torch.bfloat16).clone()
-    v_fwd = layer.saved_view("v", (S, h), torch.bfloat16).clone()
+    k_fwd = layer.saved_view("k", (S, h), torch.float16).clone()
+    v_fwd = layer.saved_view("v", (S, h), torch.float16).clone()
 
     ws_n, saved_n = T.tsp_workspace_size(layer.plan, False)
     assert saved_n == 0
     ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
     y = torch.full((S, h), float("nan"), dtype=torch.bfloat16, device="cuda")
-    kc = torch.full((S, h), float("nan"), dtype=torch.bfloat16, device="cuda")
-    vc = torch.full((S, h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kc = torch.full((S, h), float("nan"), dtype=torch.float16, device="cuda")
+    vc = torch.full((S, h), float("nan"), dtype=torch.float16, device="cuda")
     w = layer.w
     T.tsp_layer_prefill(layer.plan, layer.x, layer.g1, w["wqkv"], w["wo"], layer.g2, w["w1"], w["w2"], y, kc, vc, ws)
     T.tsp_sync_status(layer.plan)

@@ -36,13 +36,13 @@ def test_forward_intermediates(tiny):
     S, h, F, H = s.S, s.h, s.ffn, s.heads
     cat = lambda k: np.concatenate(c[k], axis=0)
     views = {
-        "a": (cat("a"), (S, h), torch.bfloat16),
-        "q": (cat("Q"), (S, h), torch.bfloat16),
-        "k": (c["Kg"], (S, h), torch.bfloat16),
-        "v": (c["Vg"], (S, h), torch.bfloat16),
-        "o": (cat("O"), (S, h), torch.bfloat16),
+        "a": (cat("a"), (S, h), torch.float16),
+        "q": (cat("Q"), (S, h), torch.float16),
+        "k": (c["Kg"], (S, h), torch.float16),
+        "v": (c["Vg"], (S, h), torch.float16),
+        "o": (cat("O"), (S, h), torch.float16),
         "y": (cat("y"), (S, h), torch.float32),
-        "b": (cat("b"), (S, h), torch.bfloat16),
+        "b": (cat("b"), (S, h), torch.float16),
         "u": (cat("U"), (S, F), torch.bfloat16),
     }
     for name, (ref, shp, dt) in views.items():
@@ -69,3 +69,22 @@ def test_repeat_is_bitwise_deterministic(tiny):
     assert np.array_equal(z2, tiny["z"])
     for k in g2:
         assert np.array_equal(g2[k], tiny["grads"][k]), k
+
+
+def test_head_size_64_layer_against_oracle():
+    # dh = 64 (h=256, 4 heads x 64, FFN 1024, S=512, D=2): the single-atom
+    # 128-byte-swizzle path of the attention kernels, every output and gradient
+    from synth_inputs import LayerShape
+
+    shape = LayerShape(h=256, heads=4, ffn=1024, S=512, D=2)
+    inp = make_layer_inputs(shape, 6)
+    layer = GpuLayer(shape, inp, training=True)
+    z = host_f64(layer.forward())
+    grads = {k: host_f64(v) for k, v in layer.backward().items()}
+    w = oracle_weights(inp)
+    zig = layer.zig
+    zo, cache = O.tsp_layer_forward(bits_to_f32(inp["x"][zig]).astype(np.float64), w, shape.heads, shape.D)
+    go = O.tsp_layer_backward(bits_to_f32(inp["dy"][zig]).astype(np.float64), w, cache)
+    assert_close("z", z, zo)
+    for k in go:
+        assert_close(k, grads[k], go[k])

@@ -1,13 +1,15 @@
-"""Evidence for the acceptance bounds (tests/tolerances.py).
+"""Evidence for holding every tensor to the stated bounds (tests/tolerances.py).
 
-A CPU model of the CUDA path's bf16 rounding placement (tests/precision_model.py)
+A CPU model of the CUDA path's rounding placement (tests/precision_model.py)
 is compared with the fp64 oracle at the 7B width (h=4096, 32 heads x 128,
 FFN 16384) on a short sequence.  The test pins two facts:
-* the stated mean bound (2e-3) is below the floor of this arithmetic for the
-  layer output and for every gradient that passes through attention, so no
-  kernel built on bf16 operands can meet it there;
-* the floor is well inside the derived bounds (at most 60% of each), so those
-  bounds still catch real kernel errors, which show up as O(1) deviations.
+* with fp16 tensor-core operands (the CUDA path) every output and gradient
+  sits inside the stated bounds with room to spare (mean error at most 0.85
+  of 2e-3, max error at most 0.5 of 1e-2), so the GPU tests can hold the
+  kernels to them;
+* with bf16 operands the same arithmetic misses the stated mean bound for the
+  output and every gradient that passes through attention: the floor of that
+  placement, not of the method.
 """
 
 import numpy as np
@@ -16,12 +18,12 @@ import pytest
 import oracle as O
 from synth_inputs import LayerShape, bits_to_f32, make_layer_inputs
 from tests.gpu_helpers import errors
-from tests.precision_model import bf16_layer
-from tests.tolerances import DERIVED, STATED
+from tests.precision_model import layer
+from tests.tolerances import STATED
 
 
 @pytest.fixture(scope="module")
-def floor():
+def floors():
     shape = LayerShape(h=4096, heads=32, ffn=16384, S=512, D=2)
     inp = make_layer_inputs(shape, 1)
     w32 = {k: bits_to_f32(inp[k]) for k in ("wqkv", "wo", "w1", "w2")}
@@ -31,16 +33,18 @@ def floor():
     z, cache = O.layer_forward(x.astype(np.float64), w64, shape.heads)
     ref = O.layer_backward(dy.astype(np.float64), w64, shape.heads, cache)
     ref["z"] = z
-    got = bf16_layer(x, w32, dy, shape.heads)
-    return {k: errors(got[k].astype(np.float64), ref[k]) for k in ref}
+    out = {}
+    for placement in ("f16", "bf16"):
+        got = layer(x, w32, dy, shape.heads, placement)
+        out[placement] = {k: errors(got[k].astype(np.float64), ref[k]) for k in ref}
+    return out
 
 
-def test_stated_mean_bound_is_below_the_bf16_floor(floor):
+def test_fp16_placement_meets_the_stated_bounds(floors):
+    for name, (mx, mn) in floors["f16"].items():
+        assert mn <= 0.85 * STATED[1] and mx <= 0.5 * STATED[0], (name, mx, mn)
+
+
+def test_bf16_placement_misses_the_stated_mean_bound(floors):
     for name in ("z", "dx", "dg1", "dwqkv", "dwo"):
-        assert floor[name][1] > STATED[1], (name, floor[name])
-
-
-def test_floor_is_well_inside_the_derived_bounds(floor):
-    for name, (mx, mn) in floor.items():
-        bmax, bmean = DERIVED[name]
-        assert mx <= 0.8 * bmax and mn <= 0.6 * bmean, (name, mx, mn)
+        assert floors["bf16"][name][1] > STATED[1], (name, floors["bf16"][name])

@@ -6,8 +6,11 @@ library keeps the scratch of this step (partial sums of the gain gradient) in
 a device array of its own.  This test runs the tiny layer's forward and
 backward through the ordinary entry points, then calls the no-allocation entry
 point twice in a row on the same intermediates the layer's last backward stage
-used, and checks that both calls reproduce the layer's dx and dg1.  It sits in
-a file of its own, collected last.
+used, and checks that both calls reproduce the layer's dx and dg1.  The layer
+keeps those intermediates times a power of two 2^k (its scaled gradient
+domain); the test multiplies them by 2^-k first, which is exact in fp32, so
+the results must agree bit for bit.  It sits in a file of its own, collected
+last.
 """
 
 import numpy as np
@@ -31,6 +34,9 @@ def test_noalloc_matches_layer_backward_twice():
     da = L.saved_view("ws.da", (S, h), torch.float32)
     dy = L.saved_view("ws.dy", (S, h), torch.float32)
     rstd1 = L.saved_view("rstd1", (S,), torch.float32)
+    unscale = L.saved_view("ws.gscales", (2,), torch.float32)[0]
+    da = (da * unscale).contiguous()
+    dy = (dy * unscale).contiguous()
     ref_dx, ref_dg = host_f64(g["dx"]), host_f64(g["dg1"])
     for _ in range(2):
         dx = torch.full((S, h), float("nan"), dtype=torch.bfloat16, device="cuda")

@@ -4,43 +4,25 @@ Both bounds are relative to the oracle tensor:
     max|gpu - oracle|  <= B_max  * max|oracle|
     mean|gpu - oracle| <= B_mean * mean|oracle|
 
-The stated bounds are B_max = 1e-2 and B_mean = 2e-3 for every output.
+Every output and gradient is held to the stated bounds, B_max = 1e-2 and
+B_mean = 2e-3.  They are within reach because every tensor-core operand the
+layer computes itself is stored as fp16 (11-bit significand), not bf16: a CPU
+model of this rounding placement (tests/test_precision_floor.py) puts the
+error of each tensor at 0.2-0.8 of the stated mean bound at the 7B width,
+while the same model with bf16 operands misses it for every tensor.
 
-The CUDA path computes with bf16 tensor-core operands and fp32 accumulation,
-and every operand that is itself a computed activation (a, Q, K, V, P, O, b, G,
-dU, dy, dO, dS, dQKV) is rounded to bf16 once.  A bf16 rounding has a mean
-relative error of about 1.4e-3 by itself, so the bf16 layer output alone uses
-~70% of the stated mean bound, and the layer amplifies upstream roundings
-(the MLP's gain is ~2.5; attention logits feed exponentials).  A CPU model of
-exactly this rounding placement (tests/test_precision_floor.py) shows that the
-stated mean bound is out of reach of any such arithmetic for several tensors,
-whatever the kernels do.  Those tensors get a derived mean bound of about
-twice the floor that the model measures at the 7B shape; every other bound is
-the stated one.  The derivation and the measured floors are recorded in the
-design notes.
+Intermediates (test-only views of the saved buffer) are compared at a looser
+bound: U is kept in bf16 (it only feeds GELU'), and the others are single
+roundings of values whose upstream error the outputs already bound.
 """
 
 STATED = (1e-2, 2e-3)
 
-# tensor -> (B_max, B_mean)
-DERIVED = {
-    "z": (1e-2, 7e-3),
-    "dx": (1e-2, 1.1e-2),
-    "dg1": (2e-2, 1.8e-2),
-    "dwqkv": (2e-2, 1.8e-2),
-    "dwo": (2e-2, 1.6e-2),
-    "dg2": (1e-2, 7e-3),
-    "dw1": (1e-2, 8e-3),
-    "dw2": (1e-2, 7e-3),
-}
-
-# Intermediates (test-only views of the saved buffer): bf16-level agreement.
+# Intermediates (test-only views of the saved buffer).
 INTERMEDIATE = (2e-2, 1e-2)
 
 
 def bound_for(name: str):
-    if name in DERIVED:
-        return DERIVED[name]
     if name.startswith("mid."):
         return INTERMEDIATE
     return STATED
