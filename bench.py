@@ -87,6 +87,7 @@ def stage_flops(s: LayerShape) -> dict:
         "bwd_dgelu_gemm": 2 * S * h * F, "bwd_dw2_gemm": 2 * S * h * F, "bwd_dw1_gemm": 2 * S * h * F,
         "bwd_db_ring_gemm": 2 * S * h * F, "bwd_do_gemm": 2 * S * h * h, "bwd_dwo_gemm": 2 * S * h * h,
         "bwd_attn_dkdv": 3 * att, "bwd_attn_dq": att, "bwd_dwqkv_gemm": 6 * S * h * h, "bwd_da_gemm": 6 * S * h * h,
+        "bwd_attn_fused": 4 * att,
     }
 
 
@@ -105,6 +106,7 @@ def hbm_stage_bytes(s: LayerShape) -> dict:
         "bwd_rmsnorm2": S * h * (4 + 4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,  # db, y, dY -> dy f32+fp16
         "bwd_rmsnorm1": S * h * (4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,      # da, x, dy -> dx bf16
         "bwd_attn_delta": S * h * (2 + 2) + S * H * 4,                    # O, dO -> delta f32 [H][S]
+        "bwd_attn_dq_convert": S * h * (4 + 2),                           # dQ sum f32 -> dQ fp16
     }
 
 

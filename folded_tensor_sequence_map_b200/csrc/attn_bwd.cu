@@ -31,6 +31,24 @@ namespace tsp {
 namespace {
 
 constexpr float kPOff = 7.0f;                 // log2 of the factor carried by the fp16 P^T
+
+// Fractional bits of a head's fixed-point dQ sum.  With P >= 0 summing to 1
+// over a query's keys, sum_k |dS_qk| = sum_k P_qk |dP_qk - Delta_q|
+// <= 2 max_k |dP_qk| <= 2 |dO_q| max_k |V_k|, so every partial sum of
+// dQ_q = sum_k dS_qk K_k / sqrt(dh) is at most B = 2 max|dO| max|V| max|K_j| / sqrt(dh)
+// in magnitude (|.| the Euclidean norm over the head's dims, |K_j| the
+// largest element).  F is chosen so that B 2^F < 2^29: sums stay below 2^30
+// however the contributions' roundings add.  `b` holds the head's maxima of
+// |dO_q|^2, |V_k|^2 and |K_j| as float bits.  The same function gives the
+// same F in every kernel that calls it.
+__device__ __forceinline__ int dq_frac_bits(const unsigned int *b, int dh) {
+    const float bound = 2.0f * sqrtf(__uint_as_float(b[0])) * sqrtf(__uint_as_float(b[1])) * __uint_as_float(b[2]) *
+                        rsqrtf(static_cast<float>(dh));
+    if (!(bound > 0.0f) || bound > 1.0e30f) return 0;
+    int E = 0;
+    frexpf(bound, &E);  // bound < 2^E
+    return min(max(29 - E, -60), 60);
+}
 constexpr float kPOffInv = 1.0f / 128.0f;     // 2^-kPOff
 
 __device__ __forceinline__ float ex2b(float x) {
@@ -76,20 +94,65 @@ CUtensorMapSwizzle swz_of() {
 }
 
 // ---------------------------------------------------------------------------
-__global__ void attn_delta_kernel(const __half *o, const __half *dout, float *delta, int S, int H, int dh) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32, lane = threadIdx.x % 32;
-    if (warp >= S * H) return;
-    const int row = warp / H, head = warp % H;
-    const int64_t base = static_cast<int64_t>(row) * H * dh + head * dh;
-    float s = 0.f;
-    for (int c = lane * 2; c < dh; c += 64) {
-        uint32_t a = *reinterpret_cast<const uint32_t *>(o + base + c);
-        uint32_t b = *reinterpret_cast<const uint32_t *>(dout + base + c);
-        s += f16_lo(a) * f16_lo(b) + f16_hi(a) * f16_hi(b);
+// Delta[h][row] = sum_d dO * O per (row, head), one warp at a time over a
+// grid-stride loop.  For the single-pass kernel (acc non-null) it also clears
+// the (row, head) slice of the integer dQ sum and takes, per head, the
+// largest |dO_row|^2, |V_row|^2 and |K|_max that bound the sum (dq_frac_bits):
+// per block in shared memory, then one atomicMax per head and block into
+// `bound` (cleared before the launch; non-negative float bits order like
+// unsigned integers, so the maxima do not depend on the order).
+__global__ void attn_delta_kernel(const __half *o, const __half *dout, const __half *kk, const __half *vv,
+                                  float *delta, int *acc, unsigned int *bound, int S, int H, int dh) {
+    extern __shared__ unsigned int smax[];  // [H][3]
+    const bool fused = acc != nullptr;
+    if (fused) {
+        for (int i = threadIdx.x; i < 3 * H; i += blockDim.x) smax[i] = 0u;
+        __syncthreads();
     }
+    const int lane = threadIdx.x % 32;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    for (int64_t wi = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; wi < static_cast<int64_t>(S) * H;
+         wi += nwarps) {
+        const int64_t row = wi / H;
+        const int head = static_cast<int>(wi - row * H);
+        const int64_t base = row * H * dh + static_cast<int64_t>(head) * dh;
+        float s = 0.f, n2 = 0.f, v2 = 0.f, km = 0.f;
+        for (int c = lane * 2; c < dh; c += 64) {
+            const uint32_t a = *reinterpret_cast<const uint32_t *>(o + base + c);
+            const uint32_t b = *reinterpret_cast<const uint32_t *>(dout + base + c);
+            s += f16_lo(a) * f16_lo(b) + f16_hi(a) * f16_hi(b);
+            if (fused) {
+                const uint32_t kw = *reinterpret_cast<const uint32_t *>(kk + base + c);
+                const uint32_t vw = *reinterpret_cast<const uint32_t *>(vv + base + c);
+                n2 += f16_lo(b) * f16_lo(b) + f16_hi(b) * f16_hi(b);
+                v2 += f16_lo(vw) * f16_lo(vw) + f16_hi(vw) * f16_hi(vw);
+                km = fmaxf(km, fmaxf(fabsf(f16_lo(kw)), fabsf(f16_hi(kw))));
+            }
+        }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) delta[static_cast<int64_t>(head) * S + row] = s;
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) delta[static_cast<int64_t>(head) * S + row] = s;
+        if (fused) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                n2 += __shfl_xor_sync(0xffffffffu, n2, off);
+                v2 += __shfl_xor_sync(0xffffffffu, v2, off);
+                km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, off));
+            }
+            if (lane == 0) {
+                atomicMax(&smax[3 * head + 0], __float_as_uint(n2));
+                atomicMax(&smax[3 * head + 1], __float_as_uint(v2));
+                atomicMax(&smax[3 * head + 2], __float_as_uint(km));
+            }
+            int4 *z = reinterpret_cast<int4 *>(acc + base);
+            for (int c = lane; c < dh / 4; c += 32) z[c] = make_int4(0, 0, 0, 0);
+        }
+    }
+    if (fused) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < 3 * H; i += blockDim.x)
+            if (smax[i]) atomicMax(&bound[i], smax[i]);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -694,6 +757,442 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------------------
+// Single-pass backward (dh = 128).  One item = (head, 128-key tile kt); steps
+// of 64 query rows over the steps that see the tile (StepWalk, ascending).
+//   TMEM columns (128 key lanes unless noted):
+//     dV [0,128)  dK [128,256)                          accumulated per item
+//     R1: S^T [256,320)  dP^T [320,384)                 fp32, one step
+//     R2: P^T [384,416)  dS^T [416,448) packed fp16     A operands of dV, dK
+//         dQ^T [448,512): lanes = head dims, columns = the step's 64 queries
+//   Per step g the MMA warp issues S^T = K Q^T and dP^T = V dO^T into R1 and,
+//   once the element-wise warps have packed P^T / dS^T into R2 and written
+//   dS^T to shared memory, dV += P^T dO and dK += dS^T Q (A from TMEM) and
+//   dQ^T = K^T dS^T (both operands from shared memory, MN-major).  R1 is
+//   released as soon as the element-wise warps have read it, so S^T / dP^T of
+//   step g+1 run on the tensor core while step g becomes P^T and dS^T.
+//   The element-wise warps drain dQ^T of step g (once its MMAs are complete)
+//   into a shared [64][128] tile of 32-bit fixed-point integers (value times
+//   2^F_head, rounded); the reducer warp adds the tile to the step's rows of
+//   the integer dQ sum in global memory with one TMA reduce-add.  Integer
+//   addition is associative, so the sum is the same bits whatever order the
+//   CTAs' additions reach L2 in: the result is deterministic with no ordering
+//   between CTAs.  F_head comes from a bound that holds for every partial sum
+//   of the head's dQ (dq_frac_bits), so no sum can overflow.
+template <int DH>
+struct FusedCfg {
+    using C = BCfg<DH>;
+    static_assert(DH == 128, "the single-pass backward computes dQ^T with M = dh = 128");
+    static constexpr int BQ = 64;
+    static constexpr int QST = 3;
+    static constexpr int QTILE = BQ * DH * 2;
+    static constexpr int QATOM = BQ * C::SWB;
+    static constexpr int VEC_BYTES = 3 * BQ * 4;
+    static constexpr int DST_BYTES = 128 * BQ * 2;   // dS^T [128 keys][64 queries] fp16, 128-byte swizzle
+    static constexpr int DQ_BYTES = BQ * DH * 4;     // dQ tile [64 queries][dh] 32-bit fixed point
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + C::TILE_BYTES;
+    static constexpr int OFF_Q = OFF_V + C::TILE_BYTES;
+    static constexpr int OFF_DO = OFF_Q + QST * QTILE;
+    static constexpr int OFF_VEC = OFF_DO + QST * QTILE;
+    static constexpr int OFF_DST = (OFF_VEC + QST * VEC_BYTES + 1023) / 1024 * 1024;
+    static constexpr int OFF_DQ = OFF_DST + DST_BYTES;
+    static constexpr int OFF_BAR = OFF_DQ + DQ_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static_assert(SMEM <= kMaxDynSmem, "single-pass backward tiles exceed the shared-memory limit");
+    // kv_full/empty, q_full/empty[QST], s_full, r1_free, p_full, mma_done, acc_empty, stage_full, stage_empty,
+    // drain + TMEM slot + abort flag
+    static_assert(8 * (2 + 2 * QST + 8) + 8 <= 256, "single-pass backward barriers exceed their slot");
+    static constexpr uint32_t T_DV = 0, T_DK = 128, T_S = 256, T_DP = 320, T_PP = 384, T_PDS = 416, T_DQ = 448;
+    static_assert(T_DQ + BQ <= 512, "single-pass backward TMEM columns");
+};
+
+constexpr int kEwThreads = 128 * kEwGroups;
+constexpr int kFusedThreads = 64 + kEwThreads + 32;  // TMA warp, MMA warp, element-wise groups, reducer warp
+
+struct FusedParams {
+    AttnBwdDesc d;
+    const int *zig;
+    int num_items;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                          const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
+                          const __grid_constant__ CUtensorMap mDQ, const FusedParams fp, const DevErr err) {
+    using C = BCfg<DH>;
+    using F = FusedCfg<DH>;
+    const AttnBwdDesc &a = fp.d;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + F::OFF_BAR);
+    uint64_t *kv_full = bars + 0, *kv_empty = bars + 1;
+    uint64_t *q_full = bars + 2;                // [QST]
+    uint64_t *q_empty = q_full + F::QST;        // [QST]
+    uint64_t *s_full = q_empty + F::QST;        // S^T / dP^T of a step in R1
+    uint64_t *r1_free = s_full + 1;             // R1 read by every element-wise thread
+    uint64_t *p_full = r1_free + 1;             // P^T / dS^T of a step packed in R2 and dS^T in smem
+    uint64_t *mma_done = p_full + 1;            // dV / dK / dQ^T MMAs of a step complete
+    uint64_t *acc_empty = mma_done + 1;         // dV / dK of an item read out
+    uint64_t *stage_full = acc_empty + 1;       // dQ tile of a step in smem
+    uint64_t *stage_empty = stage_full + 1;     // dQ tile added to global memory
+    uint64_t *drain = stage_empty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nq64 = a.S / 64;
+    const StepVis vis{a.D, a.chunk, nq64};
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
+    const float scale = rsqrtf(static_cast<float>(DH));
+    constexpr int kReducerWarp = 2 + 4 * kEwGroups;
+    int *stage = reinterpret_cast<int *>(smem + F::OFF_DQ);
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        mbar_init(kv_empty, 1);
+        for (int s = 0; s < F::QST; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(r1_free, kEwThreads);
+        mbar_init(p_full, kEwThreads);
+        mbar_init(mma_done, 1);
+        mbar_init(acc_empty, kEwThreads);
+        mbar_init(stage_full, kEwThreads);
+        mbar_init(stage_empty, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int item_iter = 0, g = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
+                if (!mbar_wait(kv_empty, (item_iter & 1) ^ 1, abort_flag, err)) break;
+                mbar_arrive_tx(kv_full, 2 * C::TILE_BYTES);
+                for (int t = 0; t < C::NATOM; ++t) {
+                    tma_load_2d(smem + F::OFF_K + t * C::ATOM_BYTES, &mK, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
+                    tma_load_2d(smem + F::OFF_V + t * C::ATOM_BYTES, &mV, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
+                }
+                StepWalk w;
+                for (w.seek(vis, 0, kt * 128); w.q < nq64; w.next(vis, kt * 128), ++g) {
+                    const int q = w.q;
+                    const int s = g % F::QST;
+                    if (!mbar_wait(&q_empty[s], ((g / F::QST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+                    mbar_arrive_tx(&q_full[s], 2 * F::QTILE + F::VEC_BYTES);
+                    for (int t = 0; t < C::NATOM; ++t) {
+                        tma_load_2d(smem + F::OFF_Q + s * F::QTILE + t * F::QATOM, &mQ, &q_full[s],
+                                    head * DH + t * C::ATOM_COLS, q * 64);
+                        tma_load_2d(smem + F::OFF_DO + s * F::QTILE + t * F::QATOM, &mdO, &q_full[s],
+                                    head * DH + t * C::ATOM_COLS, q * 64);
+                    }
+                    float *vec = reinterpret_cast<float *>(smem + F::OFF_VEC + s * F::VEC_BYTES);
+                    bulk_load(vec, a.lse + static_cast<int64_t>(head) * a.S + q * 64, 256, &q_full[s]);
+                    bulk_load(vec + 64, a.delta + static_cast<int64_t>(head) * a.S + q * 64, 256, &q_full[s]);
+                    bulk_load(vec + 128, fp.zig + q * 64, 256, &q_full[s]);
+                }
+            }
+            if (item_iter > 0) spin_drain(kv_full, (item_iter - 1) & 1, err.wait_limit);
+            for (int s = 0; s < F::QST; ++s)
+                if (g > s) {
+                    const int last = g - 1 - ((g - 1 - s) % F::QST);
+                    spin_drain(&q_full[s], (last / F::QST) & 1, err.wait_limit);
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // The whole warp runs the loop; one elected lane polls and issues.
+        {
+            const bool leader = elect_one();
+            const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+            constexpr uint32_t idS = idesc_f16(128, 64, false, false);
+            constexpr uint32_t idG = idesc_f16(128, DH, false, true);
+            constexpr uint32_t idQ = idesc_f16(DH, 64, true, true);
+            const uint64_t dK0 = kdesc<DH>(smem_u32(smem + F::OFF_K), 0);
+            const uint64_t dV0 = kdesc<DH>(smem_u32(smem + F::OFF_V), 0);
+            // A of dQ^T = K^T: the K tile read MN-major (rows = keys, head dims
+            // contiguous in two 128-byte atoms); K steps of 16 keys advance 2 KB
+            const uint64_t dKt0 = sdesc(smem_u32(smem + F::OFF_K), C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
+            // B of dQ^T = dS^T [128 keys][64 queries]: MN-major, one atom wide
+            const uint64_t dSt0 = sdesc(smem_u32(smem + F::OFF_DST), 8192, 1024, kSwizzle128);
+            int item_iter = 0, g = 0;
+            bool ok = true;
+            auto issue_sdp = [&](int gi) -> bool {
+                const int s = gi % F::QST;
+                if (!lead_wait(leader, leader_lane, &q_full[s], (gi / F::QST) & 1, abort_flag, err)) return false;
+                if (leader) {
+                    tc_fence_after();
+                    const uint64_t dQ0 = kdesc64<DH>(smem_u32(smem + F::OFF_Q + s * F::QTILE), 0);
+                    const uint64_t dO0 = kdesc64<DH>(smem_u32(smem + F::OFF_DO + s * F::QTILE), 0);
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_ss(tmem + F::T_S, desc_plus(dK0, kdesc_off<DH>(kk)), desc_plus(dQ0, kdesc64_off<DH>(kk)),
+                                idS, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        umma_ss(tmem + F::T_DP, desc_plus(dV0, kdesc_off<DH>(kk)), desc_plus(dO0, kdesc64_off<DH>(kk)),
+                                idS, kk > 0);
+                    umma_commit(s_full);
+                }
+                return true;
+            };
+            for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kv0 = (a.kv_order[it] / a.H) * 128;
+                if (!lead_wait(leader, leader_lane, kv_full, item_iter & 1, abort_flag, err)) break;
+                if (leader) tc_fence_after();
+                StepWalk w;
+                w.seek(vis, 0, kv0);
+                if (w.q < nq64 && !issue_sdp(g)) break;
+                bool first = true;
+                while (w.q < nq64) {
+                    StepWalk wn = w;
+                    wn.next(vis, kv0);
+                    if (wn.q < nq64) {
+                        // S^T / dP^T of the next step into R1 once R1 has been read
+                        if (!lead_wait(leader, leader_lane, r1_free, g & 1, abort_flag, err) || !issue_sdp(g + 1)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!lead_wait(leader, leader_lane, p_full, g & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    // the first dV / dK MMA of an item overwrites the accumulators
+                    // that the previous item's epilogue reads
+                    if (first && item_iter > 0 &&
+                        !lead_wait(leader, leader_lane, acc_empty, (item_iter - 1) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) {
+                        tc_fence_after();
+                        const int s = g % F::QST;
+                        const uint64_t gQ0 = mndesc64<DH>(smem_u32(smem + F::OFF_Q + s * F::QTILE), 0);
+                        const uint64_t gO0 = mndesc64<DH>(smem_u32(smem + F::OFF_DO + s * F::QTILE), 0);
+                        // A operands from TMEM: queries 16 kk .. 16 kk + 15 packed at column 8 kk
+#pragma unroll
+                        for (int kk = 0; kk < F::BQ / 16; ++kk)
+                            umma_ts(tmem + F::T_DV, tmem + F::T_PP + kk * 8, desc_plus(gO0, mndesc64_off<DH>(kk)), idG,
+                                    (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int kk = 0; kk < F::BQ / 16; ++kk)
+                            umma_ts(tmem + F::T_DK, tmem + F::T_PDS + kk * 8, desc_plus(gQ0, mndesc64_off<DH>(kk)), idG,
+                                    (!first || kk > 0) ? 1u : 0u);
+                        // dQ^T [dh][64] = K^T dS^T over the 128 keys, 16 at a time
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_ss(tmem + F::T_DQ, desc_plus(dKt0, kk * 16 * C::SWB), desc_plus(dSt0, kk * 2048), idQ,
+                                    kk > 0);
+                        umma_commit(mma_done);
+                        umma_commit(&q_empty[s]);
+                    }
+                    first = false;
+                    ++g;
+                    w = wn;
+                }
+                if (leader) umma_commit(kv_empty);
+            }
+            const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
+            if (bad && leader) {
+                umma_commit(drain);
+                spin_drain(drain, 0, err.wait_limit);
+            }
+            __syncwarp();
+        }
+    } else if (warp < kReducerWarp) {
+        // ------------------------------------------------------------ element-wise groups
+        const int grp = (warp - 2) / 4;         // query columns [16 grp, 16 grp + 16) of a step
+        const int quarter = warp & 3;
+        const int trow = quarter * 32 + lane;   // key row of the tile = TMEM lane (head dim for dQ^T)
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        uint8_t *dst_tile = smem + F::OFF_DST;
+        int g = 0;
+        // dQ^T of step gd (its MMAs complete) into the shared fixed-point tile
+        // [query][dh], then handed to the reducer warp
+        float dq_scale = 1.0f;  // 2^F of the current item's head
+        auto drain_dq = [&](int gd) -> bool {
+            if (!warp_wait(mma_done, gd & 1, abort_flag, err)) return false;
+            tc_fence_after();
+            if (!warp_converged("dQ^T TMEM load")) return false;
+            float v[16];
+            tmem_ld16(tmem + lane_off + F::T_DQ + 16 * grp, v);
+            tmem_ld_wait();
+            if (gd > 0 && !warp_wait(stage_empty, (gd - 1) & 1, abort_flag, err)) return false;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) stage[(16 * grp + j) * DH + trow] = __float2int_rn(v[j] * dq_scale);
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(stage_full);
+            return true;
+        };
+        for (int it = blockIdx.x; it < fp.num_items; it += gridDim.x) {
+            const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
+            const int kv0 = kt * 128;
+            const int key = kv0 + trow;
+            bool ok = true, any = false;
+            // the previous item's last dQ tile was drained at its end, so the
+            // scale can change here
+            dq_scale = ldexpf(1.0f, dq_frac_bits(a.dq_bound + 3 * head, DH));
+            StepWalk w;
+            for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+                const int s = g % F::QST;
+                if (!warp_wait(s_full, g & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                if (!warp_converged("S^T/dP^T TMEM load")) { ok = false; break; }
+                float sv[16], dp[16];
+                tmem_ld16(tmem + lane_off + F::T_S + 16 * grp, sv);
+                tmem_ld16(tmem + lane_off + F::T_DP + 16 * grp, dp);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(r1_free);
+                const float *vec = reinterpret_cast<const float *>(smem + F::OFF_VEC + s * F::VEC_BYTES);
+                const int *pos = reinterpret_cast<const int *>(vec + 128);
+                // the 64 query rows of a step lie in one zigzag chunk, so their
+                // positions are consecutive: this key is visible to column e of
+                // the group iff e >= key - pos0
+                const int first_vis = key - pos[16 * grp];
+                const float4 *lse4 = reinterpret_cast<const float4 *>(vec + 16 * grp);
+                const float4 *dl4 = reinterpret_cast<const float4 *>(vec + 64 + 16 * grp);
+                uint32_t pk[8], dk[8];
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 l = lse4[e4], d = dl4[e4];
+                    const int e = 4 * e4;
+                    // p = 2^kPOff P (the offset rides in the exponent)
+                    float p0 = ex2b(fmaf(sv[e], sl2, kPOff - l.x)), p1 = ex2b(fmaf(sv[e + 1], sl2, kPOff - l.y));
+                    float p2 = ex2b(fmaf(sv[e + 2], sl2, kPOff - l.z)), p3 = ex2b(fmaf(sv[e + 3], sl2, kPOff - l.w));
+                    if (first_vis > 0) {
+                        p0 = e >= first_vis ? p0 : 0.f;
+                        p1 = e + 1 >= first_vis ? p1 : 0.f;
+                        p2 = e + 2 >= first_vis ? p2 : 0.f;
+                        p3 = e + 3 >= first_vis ? p3 : 0.f;
+                    }
+                    pk[2 * e4] = pack_f16(p0, p1);
+                    pk[2 * e4 + 1] = pack_f16(p2, p3);
+                    // dS = P (dP - Delta), without the offset
+                    p0 *= kPOffInv;
+                    p1 *= kPOffInv;
+                    p2 *= kPOffInv;
+                    p3 *= kPOffInv;
+                    dk[2 * e4] = pack_f16(p0 * (dp[e] - d.x), p1 * (dp[e + 1] - d.y));
+                    dk[2 * e4 + 1] = pack_f16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
+                }
+                // R2 and the dS^T tile still belong to the previous step until its
+                // MMAs complete; draining its dQ^T waits for exactly that
+                if (any && !drain_dq(g - 1)) { ok = false; break; }
+                any = true;
+                if (!warp_converged("P^T/dS^T TMEM store")) { ok = false; break; }
+                tmem_st8u(tmem + lane_off + F::T_PP + 8 * grp, pk);
+                tmem_st8u(tmem + lane_off + F::T_PDS + 8 * grp, dk);
+                // this key's row of dS^T: its 16 queries are the 16-byte chunks
+                // 2 grp and 2 grp + 1 of the 128-byte row, 128-byte swizzled
+                uint4 *row = reinterpret_cast<uint4 *>(dst_tile + trow * 128);
+                row[(2 * grp) ^ (trow & 7)] = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+                row[(2 * grp + 1) ^ (trow & 7)] = make_uint4(dk[4], dk[5], dk[6], dk[7]);
+                tmem_st_wait();
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            if (!any) continue;
+            // the item's last step: its MMAs complete means dV and dK are too
+            if (!drain_dq(g - 1)) break;
+            tc_fence_after();
+            // groups 0, 1 write dV (offset removed) and groups 2, 3 write dK
+            // (scaled), at the key owner's local row; each pair splits the
+            // 32-column chunks
+            const int lrow = a.inv_map[key];
+            const int which = grp >> 1;
+            void *dstp = which == 0 ? a.dv : a.dk;
+            const float f = which == 0 ? kPOffInv : scale;
+            __half *orow = static_cast<__half *>(dstp) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+            if (!warp_converged("dV/dK TMEM load")) break;
+#pragma unroll 1
+            for (int c = grp & 1; c < DH / 32; c += 2) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + (which == 0 ? F::T_DV : F::T_DK) + c * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= f;
+                flag_range(maxabs32(v), a.err);
+                uint4 *d4 = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+                    d4[qq] = make_uint4(pack_f16(v[8 * qq], v[8 * qq + 1]), pack_f16(v[8 * qq + 2], v[8 * qq + 3]),
+                                        pack_f16(v[8 * qq + 4], v[8 * qq + 5]), pack_f16(v[8 * qq + 6], v[8 * qq + 7]));
+            }
+            tc_fence_before();
+            mbar_arrive(acc_empty);
+        }
+    } else {
+        // ------------------------------------------------------------ reducer
+        // Adds each step's fixed-point dQ tile to the step's rows of the
+        // integer dQ sum (one TMA reduce-add); the shared tile is handed back
+        // as soon as the bulk operation has read it.
+        const bool leader = lane == 0;
+        int g = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x) {
+            const int head = a.kv_order[it] % a.H, kv0 = (a.kv_order[it] / a.H) * 128;
+            StepWalk w;
+            for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+                if (!lead_wait(leader, 0, stage_full, g & 1, abort_flag, err)) { ok = false; break; }
+                if (leader) {
+                    fence_async_global();
+                    tma_reduce_add_2d(&mDQ, stage, head * DH, w.q * 64);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                    mbar_arrive(stage_empty);
+                }
+                __syncwarp();
+            }
+        }
+        if (leader) bulk_wait_all();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// dQ = (fixed-point sum) 2^-F_head / sqrt(dh) as fp16, 8 elements per thread.
+__global__ void dq_convert_kernel(const int *acc, const unsigned int *bound, __half *dq, int64_t ldd, int S, int h,
+                                  int dh, unsigned int *err) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= static_cast<int64_t>(S) * h / 8) return;
+    const int64_t e = i * 8;
+    const int64_t row = e / h;
+    const int col = static_cast<int>(e - row * h);
+    const float f = ldexpf(rsqrtf(static_cast<float>(dh)), -dq_frac_bits(bound + 3 * (col / dh), dh));
+    const int4 t0 = *reinterpret_cast<const int4 *>(acc + e);
+    const int4 t1 = *reinterpret_cast<const int4 *>(acc + e + 4);
+    const float v[8] = {t0.x * f, t0.y * f, t0.z * f, t0.w * f, t1.x * f, t1.y * f, t1.z * f, t1.w * f};
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    flag_range(m, err);
+    *reinterpret_cast<uint4 *>(dq + row * ldd + col) =
+        make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]), pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
+}
+
 template <int DH>
 struct BwdMaps {
     CUtensorMap q, k, v, dout;
@@ -762,13 +1261,65 @@ cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms,
     return cudaGetLastError();
 }
 
+
+template <int DH>
+cudaError_t launch_fused_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig) {
+    using C = BCfg<DH>;
+    BwdMaps<DH> m;
+    if (!m.make(a)) return cudaErrorInvalidValue;
+    // Q and dO sub-tiles of 64 rows; the fp32 dQ sum in [dh x 64] boxes
+    const int h = a.H * DH;
+    const auto swz = swz_of<DH>();
+    bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    CUtensorMap mdq;
+    ok = ok && encode_tensor_map_2d(&mdq, a.dq_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, h, a.S, int64_t(h) * 4, DH, 64,
+                                    CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
+    FusedParams fp;
+    fp.d = a;
+    fp.zig = zig;
+    fp.num_items = (a.S / 128) * a.H;
+    // at most one CTA per SM, so every CTA is resident (the dQ order waits need it)
+    const int grid = fp.num_items < num_sms ? fp.num_items : num_sms;
+    auto k = attn_bwd_fused_kernel<DH>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<DH>::SMEM);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kFusedThreads, FusedCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, mdq, fp, err);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st) {
-    const int warps = a.S * a.H;
-    attn_delta_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(static_cast<const __half *>(a.o),
-                                                                 static_cast<const __half *>(a.dout), a.delta, a.S,
-                                                                 a.H, a.dh);
+bool attn_bwd_fused_supported(int dh) { return dh == 128; }
+
+cudaError_t launch_attn_bwd_fused(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
+                                  const int *zig) {
+    if (a.dh != 128 || !a.dq_acc || !a.dq_bound) return cudaErrorInvalidValue;
+    return launch_fused_impl<128>(a, err, num_sms, st, zig);
+}
+
+cudaError_t launch_dq_convert(const AttnBwdDesc &a, cudaStream_t st) {
+    const int h = a.H * a.dh;
+    const int64_t n8 = static_cast<int64_t>(a.S) * h / 8;
+    const int threads = 256;
+    const int64_t blocks = (n8 + threads - 1) / threads;
+    dq_convert_kernel<<<static_cast<unsigned int>(blocks), threads, 0, st>>>(
+        a.dq_acc, a.dq_bound, static_cast<__half *>(a.dq), a.ldd, a.S, h, a.dh, a.err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_delta(const AttnBwdDesc &a, int num_sms, cudaStream_t st) {
+    if (a.dq_acc) {
+        cudaError_t e = cudaMemsetAsync(a.dq_bound, 0, static_cast<size_t>(3) * a.H * sizeof(unsigned int), st);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t warps = static_cast<int64_t>(a.S) * a.H;
+    const int64_t want = (warps * 32 + 255) / 256;
+    const int blocks = static_cast<int>(want < 8LL * num_sms ? want : 8LL * num_sms);
+    attn_delta_kernel<<<blocks, 256, static_cast<size_t>(3) * a.H * sizeof(unsigned int), st>>>(
+        static_cast<const __half *>(a.o), static_cast<const __half *>(a.dout), static_cast<const __half *>(a.k),
+        static_cast<const __half *>(a.v), a.delta, a.dq_acc, a.dq_bound, a.S, a.H, a.dh);
     return cudaGetLastError();
 }
 

@@ -195,14 +195,24 @@ struct AttnBwdDesc {
     const int *inv_map;                // global position -> local row
     const int *kv_order;               // work order of (head, 128-key block), longest first
     const int *q_order;                // work order of (head, 128-row query block), longest first
+    int *dq_acc;                       // [S][h] scratch: dQ summed over key tiles in 32-bit fixed point
+                                       // (single-pass kernel; zeroed by the Delta kernel), or null
+    unsigned int *dq_bound;            // [H][3] scratch: per-head maxima bounding that sum (Delta kernel)
 };
 // Delta = rowsum(dO * O) per head; then dK/dV (key-tile items, 64-row query
 // steps, visibility from zz_next_visible) and dQ (query-tile items).  zig:
 // local row -> global position; qtile_maxpos: largest position of each
 // 128-row local query tile.
-cudaError_t launch_attn_delta(const AttnBwdDesc &a, cudaStream_t st);
+cudaError_t launch_attn_delta(const AttnBwdDesc &a, int num_sms, cudaStream_t st);
 cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig);
 cudaError_t launch_attn_dq(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
                            const int *qtile_maxpos);
+// Single-pass backward for dh = 128: dK, dV and the fixed-point dQ sum
+// (dq_acc, integer additions: deterministic in any order) in one kernel over
+// (head, 128-key tile) items; then dQ = dq_acc / sqrt(dh) as fp16 into a.dq.
+bool attn_bwd_fused_supported(int dh);
+cudaError_t launch_attn_bwd_fused(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
+                                  const int *zig);
+cudaError_t launch_dq_convert(const AttnBwdDesc &a, cudaStream_t st);
 
 }  // namespace tsp

@@ -56,7 +56,7 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // `gscales` the gradient scale of a backward call (2^-k, 2^k).
 struct Layout {
     size_t rstd1, a, q, k, v, o, lse, y, rstd2, b, u, g, wqkv_h, wo_h, w1_h, w2_h, scales, cpart, saved_total;
-    size_t du, db, dy, dyh, dO, delta, dqkv, da, dgp, dy16, gscales, gpart, bwd_total;
+    size_t du, db, dy, dyh, dO, delta, dqkv, da, dgp, dy16, gscales, gpart, dq_acc, dq_bound, bwd_total;
 };
 constexpr int kScaleInv = 0, kScale = 8;
 constexpr int kTargetWeights = 12;  // largest |w| * 2^e in [2^11, 2^12)
@@ -103,6 +103,8 @@ Layout layout_of(const tsp_plan_s *p) {
     l.dy16 = take(S * h * 2);
     l.gscales = take(64 * 4);
     l.gpart = take(static_cast<size_t>(kMaxConv) * kConvBlocks * 4);
+    l.dq_acc = p->dh == 128 ? take(S * h * 4) : 0;
+    l.dq_bound = take(3 * H * 4);
     l.bwd_total = off;
     return l;
 }
@@ -300,7 +302,8 @@ const char *kStageNames[TSP_NUM_STAGES] = {
     "fwd_rmsnorm1", "fwd_qkv_gemm", "fwd_attention", "fwd_out_proj_gemm", "fwd_rmsnorm2", "fwd_w1_gelu_gemm",
     "fwd_w2_ring_gemm", "bwd_dgelu_gemm", "bwd_dw2_gemm", "bwd_dw1_gemm", "bwd_db_ring_gemm", "bwd_rmsnorm2",
     "bwd_do_gemm", "bwd_dwo_gemm", "bwd_attn_delta", "bwd_attn_dkdv", "bwd_attn_dq", "bwd_dwqkv_gemm",
-    "bwd_da_gemm", "bwd_rmsnorm1", "fwd_convert_weights", "bwd_convert_dy"};
+    "bwd_da_gemm", "bwd_rmsnorm1", "fwd_convert_weights", "bwd_convert_dy", "bwd_attn_fused",
+    "bwd_attn_dq_convert"};
 
 GemmDesc gemm(const void *A, int64_t lda, bool a_mn, const void *B, int64_t ldb, bool b_mn, int M, int N, int K,
               int epi, void *out, int64_t ldo, const float *alpha = nullptr) {
@@ -745,9 +748,17 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     ab.inv_map = p->d_inv;
     ab.kv_order = p->d_kv_order;
     ab.q_order = p->d_q_order;
-    TSP_STAGE(14, 1, launch_attn_delta(ab, s));
-    TSP_STAGE(15, 1, launch_attn_dkdv(ab, err, p->num_sms, s, p->d_zig));
-    TSP_STAGE(16, 1, launch_attn_dq(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
+    ab.dq_acc = attn_bwd_fused_supported(p->dh) ? reinterpret_cast<int *>(w + l.dq_acc) : nullptr;
+    ab.dq_bound = reinterpret_cast<unsigned int *>(w + l.dq_bound);
+    TSP_STAGE(14, 1, launch_attn_delta(ab, p->num_sms, s));
+    if (attn_bwd_fused_supported(p->dh)) {
+        // one pass: dK, dV and the fixed-point dQ sum; then dQ to fp16
+        TSP_STAGE(22, 1, launch_attn_bwd_fused(ab, err, p->num_sms, s, p->d_zig));
+        TSP_STAGE(23, 1, launch_dq_convert(ab, s));
+    } else {
+        TSP_STAGE(15, 1, launch_attn_dkdv(ab, err, p->num_sms, s, p->d_zig));
+        TSP_STAGE(16, 1, launch_attn_dq(ab, err, p->num_sms, s, p->d_zig, p->d_qmax));
+    }
     // projection backward: dWqkv = [dQ|dK|dV]^T a, da = [dQ|dK|dV] Wqkv
     TSP_STAGE(17, 1, launch_gemm(gemm(dqkv, 3 * h, true, a, h, true, 3 * h, h, S, EPI_F32, dwqkv, h, ginv), err, p->num_sms, s));
     TSP_STAGE(18, 1, launch_gemm(gemm(dqkv, 3 * h, false, wqkv_h, h, true, S, h, 3 * h, EPI_F32, da, h, winv + 0), err, p->num_sms, s));

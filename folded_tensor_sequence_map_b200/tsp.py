@@ -54,7 +54,7 @@ EXPORTED = (
     "tsp_test_tables",
     "tsp_test_wait_timeout",
 )
-TSP_NUM_STAGES = 22
+TSP_NUM_STAGES = 24
 
 
 class TSPError(RuntimeError):

@@ -209,8 +209,10 @@ const char *tsp_status_string(tsp_status status);
 /* Kernel stages of one forward + backward (profiling ids): 0-6 the forward
  * and 7-19 the backward in launch order; 20 the forward's weight conversion
  * (first in the forward) and 21 the backward's dY conversion (first in the
- * backward). */
-#define TSP_NUM_STAGES 22
+ * backward).  With head size 128 the attention backward is one pass, stage
+ * 22 (dK, dV and the fp32 dQ sum) and stage 23 (dQ to fp16), in place of
+ * stages 15 and 16. */
+#define TSP_NUM_STAGES 24
 
 /* Per-stage timing with CUDA events.  tsp_profile_enable(plan, 1) clears the
  * record and starts bracketing every stage of later layer calls with a pair of

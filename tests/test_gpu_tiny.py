@@ -88,3 +88,28 @@ def test_head_size_64_layer_against_oracle():
     assert_close("z", z, zo)
     for k in go:
         assert_close(k, grads[k], go[k])
+
+
+@pytest.mark.parametrize("S,D,heads", [(512, 1, 4), (512, 4, 4), (1024, 2, 4), (1024, 8, 8)])
+def test_head_size_128_layer_against_oracle(S, D, heads):
+    # dh = 128 (heads x 128, FFN 4h): the single-pass attention backward with
+    # its ordered dQ sum, at zigzag chunks of 64 to 512 rows
+    from synth_inputs import LayerShape
+
+    shape = LayerShape(h=128 * heads, heads=heads, ffn=512 * heads, S=S, D=D)
+    inp = make_layer_inputs(shape, 7)
+    layer = GpuLayer(shape, inp, training=True)
+    z = host_f64(layer.forward())
+    grads = {k: host_f64(v) for k, v in layer.backward().items()}
+    w = oracle_weights(inp)
+    zig = layer.zig
+    zo, cache = O.tsp_layer_forward(bits_to_f32(inp["x"][zig]).astype(np.float64), w, shape.heads, shape.D)
+    go = O.tsp_layer_backward(bits_to_f32(inp["dy"][zig]).astype(np.float64), w, cache)
+    assert_close("z", z, zo)
+    for k in go:
+        assert_close(k, grads[k], go[k])
+    # the same call again gives the same bits (the dQ sum is order-fixed)
+    layer.forward()
+    g2 = {k: host_f64(v) for k, v in layer.backward().items()}
+    for k in g2:
+        assert np.array_equal(g2[k], grads[k]), k
