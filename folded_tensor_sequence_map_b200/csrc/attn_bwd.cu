@@ -771,10 +771,13 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 //   dQ^T = K^T dS^T (both operands from shared memory, MN-major).  R1 is
 //   released as soon as the element-wise warps have read it, so S^T / dP^T of
 //   step g+1 run on the tensor core while step g becomes P^T and dS^T.
-//   The element-wise warps drain dQ^T of step g (once its MMAs are complete)
-//   into a shared [64][128] tile of 32-bit fixed-point integers (value times
-//   2^F_head, rounded); the reducer warp adds the tile to the step's rows of
-//   the integer dQ sum in global memory with one TMA reduce-add.  Integer
+//   Four drain warps (one per TMEM lane quarter) take dQ^T of step g out of
+//   TMEM once its MMAs are complete, release the columns for step g+1's dQ^T
+//   and write a shared [64][128] tile of 32-bit fixed-point integers (value
+//   times 2^F_head, rounded), which one of them adds to the step's rows of the
+//   integer dQ sum in global memory with a TMA reduce-add.  The element-wise
+//   warps never wait for the drain, and the MMA warp waits for it only before
+//   the next dQ^T.  Integer
 //   addition is associative, so the sum is the same bits whatever order the
 //   CTAs' additions reach L2 in: the result is deterministic with no ordering
 //   between CTAs.  F_head comes from a bound that holds for every partial sum
@@ -800,15 +803,15 @@ struct FusedCfg {
     static constexpr int OFF_BAR = OFF_DQ + DQ_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
     static_assert(SMEM <= kMaxDynSmem, "single-pass backward tiles exceed the shared-memory limit");
-    // kv_full/empty, q_full/empty[QST], s_full, r1_free, p_full, mma_done, acc_empty, stage_full, stage_empty,
-    // drain + TMEM slot + abort flag
+    // kv_full/empty, q_full/empty[QST], s_full, r1_free, p_full, mma_done, acc_empty, dq_free, spare, drain
+    // + TMEM slot + abort flag
     static_assert(8 * (2 + 2 * QST + 8) + 8 <= 256, "single-pass backward barriers exceed their slot");
     static constexpr uint32_t T_DV = 0, T_DK = 128, T_S = 256, T_DP = 320, T_PP = 384, T_PDS = 416, T_DQ = 448;
     static_assert(T_DQ + BQ <= 512, "single-pass backward TMEM columns");
 };
 
 constexpr int kEwThreads = 128 * kEwGroups;
-constexpr int kFusedThreads = 64 + kEwThreads + 32;  // TMA warp, MMA warp, element-wise groups, reducer warp
+constexpr int kFusedThreads = 64 + kEwThreads + 128;  // TMA warp, MMA warp, element-wise groups, 4 drain warps
 
 struct FusedParams {
     AttnBwdDesc d;
@@ -836,9 +839,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     uint64_t *p_full = r1_free + 1;             // P^T / dS^T of a step packed in R2 and dS^T in smem
     uint64_t *mma_done = p_full + 1;            // dV / dK / dQ^T MMAs of a step complete
     uint64_t *acc_empty = mma_done + 1;         // dV / dK of an item read out
-    uint64_t *stage_full = acc_empty + 1;       // dQ tile of a step in smem
-    uint64_t *stage_empty = stage_full + 1;     // dQ tile added to global memory
-    uint64_t *drain = stage_empty + 1;
+    uint64_t *dq_free = acc_empty + 1;          // dQ^T of a step read out of TMEM
+    uint64_t *drain = dq_free + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -847,7 +849,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const StepVis vis{a.D, a.chunk, nq64};
     const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
     const float scale = rsqrtf(static_cast<float>(DH));
-    constexpr int kReducerWarp = 2 + 4 * kEwGroups;
+    constexpr int kDrainWarp = 2 + 4 * kEwGroups;
     int *stage = reinterpret_cast<int *>(smem + F::OFF_DQ);
 
     if (threadIdx.x == 0) {
@@ -862,8 +864,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         mbar_init(p_full, kEwThreads);
         mbar_init(mma_done, 1);
         mbar_init(acc_empty, kEwThreads);
-        mbar_init(stage_full, kEwThreads);
-        mbar_init(stage_empty, 1);
+        mbar_init(dq_free, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -981,9 +982,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         ok = false;
                         break;
                     }
+                    const int s = g % F::QST;
                     if (leader) {
                         tc_fence_after();
-                        const int s = g % F::QST;
                         const uint64_t gQ0 = mndesc64<DH>(smem_u32(smem + F::OFF_Q + s * F::QTILE), 0);
                         const uint64_t gO0 = mndesc64<DH>(smem_u32(smem + F::OFF_DO + s * F::QTILE), 0);
                         // A operands from TMEM: queries 16 kk .. 16 kk + 15 packed at column 8 kk
@@ -995,6 +996,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         for (int kk = 0; kk < F::BQ / 16; ++kk)
                             umma_ts(tmem + F::T_DK, tmem + F::T_PDS + kk * 8, desc_plus(gQ0, mndesc64_off<DH>(kk)), idG,
                                     (!first || kk > 0) ? 1u : 0u);
+                    }
+                    // the previous step's dQ^T must be out of TMEM before this one
+                    if (g > 0 && !lead_wait(leader, leader_lane, dq_free, (g - 1) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) {
+                        tc_fence_after();
                         // dQ^T [dh][64] = K^T dS^T over the 128 keys, 16 at a time
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
@@ -1016,7 +1025,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             }
             __syncwarp();
         }
-    } else if (warp < kReducerWarp) {
+    } else if (warp < kDrainWarp) {
         // ------------------------------------------------------------ element-wise groups
         const int grp = (warp - 2) / 4;         // query columns [16 grp, 16 grp + 16) of a step
         const int quarter = warp & 3;
@@ -1024,32 +1033,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         uint8_t *dst_tile = smem + F::OFF_DST;
         int g = 0;
-        // dQ^T of step gd (its MMAs complete) into the shared fixed-point tile
-        // [query][dh], then handed to the reducer warp
-        float dq_scale = 1.0f;  // 2^F of the current item's head
-        auto drain_dq = [&](int gd) -> bool {
-            if (!warp_wait(mma_done, gd & 1, abort_flag, err)) return false;
-            tc_fence_after();
-            if (!warp_converged("dQ^T TMEM load")) return false;
-            float v[16];
-            tmem_ld16(tmem + lane_off + F::T_DQ + 16 * grp, v);
-            tmem_ld_wait();
-            if (gd > 0 && !warp_wait(stage_empty, (gd - 1) & 1, abort_flag, err)) return false;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) stage[(16 * grp + j) * DH + trow] = __float2int_rn(v[j] * dq_scale);
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(stage_full);
-            return true;
-        };
         for (int it = blockIdx.x; it < fp.num_items; it += gridDim.x) {
             const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
             const int kv0 = kt * 128;
             const int key = kv0 + trow;
             bool ok = true, any = false;
-            // the previous item's last dQ tile was drained at its end, so the
-            // scale can change here
-            dq_scale = ldexpf(1.0f, dq_frac_bits(a.dq_bound + 3 * head, DH));
             StepWalk w;
             for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
                 const int s = g % F::QST;
@@ -1095,8 +1083,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     dk[2 * e4 + 1] = pack_f16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
                 }
                 // R2 and the dS^T tile still belong to the previous step until its
-                // MMAs complete; draining its dQ^T waits for exactly that
-                if (any && !drain_dq(g - 1)) { ok = false; break; }
+                // MMAs complete
+                if (g > 0 && !warp_wait(mma_done, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
                 any = true;
                 if (!warp_converged("P^T/dS^T TMEM store")) { ok = false; break; }
                 tmem_st8u(tmem + lane_off + F::T_PP + 8 * grp, pk);
@@ -1114,7 +1103,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (!ok) break;
             if (!any) continue;
             // the item's last step: its MMAs complete means dV and dK are too
-            if (!drain_dq(g - 1)) break;
+            if (!warp_wait(mma_done, (g - 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             // groups 0, 1 write dV (offset removed) and groups 2, 3 write dK
             // (scaled), at the key owner's local row; each pair splits the
@@ -1143,29 +1132,46 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             mbar_arrive(acc_empty);
         }
     } else {
-        // ------------------------------------------------------------ reducer
-        // Adds each step's fixed-point dQ tile to the step's rows of the
-        // integer dQ sum (one TMA reduce-add); the shared tile is handed back
-        // as soon as the bulk operation has read it.
-        const bool leader = lane == 0;
+        // ------------------------------------------------------------ drain warps
+        // dQ^T of every step out of TMEM (thread = head dim), into the shared
+        // fixed-point tile [query][dh], then one TMA reduce-add into the
+        // integer dQ sum.  Named barriers 1 and 2 order the four warps around
+        // the shared tile; warp kDrainWarp's first lane issues the bulk ops.
+        const int quarter = warp & 3;
+        const int d = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const bool issuer = warp == kDrainWarp && lane == 0;
         int g = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x) {
             const int head = a.kv_order[it] % a.H, kv0 = (a.kv_order[it] / a.H) * 128;
+            const float dq_scale = ldexpf(1.0f, dq_frac_bits(a.dq_bound + 3 * head, DH));
             StepWalk w;
             for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
-                if (!lead_wait(leader, 0, stage_full, g & 1, abort_flag, err)) { ok = false; break; }
-                if (leader) {
+                if (!warp_wait(mma_done, g & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                if (!warp_converged("dQ^T TMEM load")) { ok = false; break; }
+                float v[64];
+                tmem_ld32(tmem + lane_off + F::T_DQ, *reinterpret_cast<float(*)[32]>(v));
+                tmem_ld32(tmem + lane_off + F::T_DQ + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(dq_free);
+                // the previous tile has been read by its bulk operation
+                if (issuer) bulk_wait_read_all();
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+                for (int j = 0; j < 64; ++j) stage[j * DH + d] = __float2int_rn(v[j] * dq_scale);
+                fence_async_smem();
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (issuer) {
                     fence_async_global();
                     tma_reduce_add_2d(&mDQ, stage, head * DH, w.q * 64);
                     bulk_commit();
-                    bulk_wait_read_all();
-                    mbar_arrive(stage_empty);
                 }
-                __syncwarp();
             }
         }
-        if (leader) bulk_wait_all();
+        if (issuer) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -1260,6 +1266,7 @@ cudaError_t launch_dq_impl(const AttnBwdDesc &a, const DevErr &err, int num_sms,
     k2<<<grid, kBwdThreads2, Dq2Cfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, bp, err);
     return cudaGetLastError();
 }
+
 
 
 template <int DH>
