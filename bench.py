@@ -91,6 +91,13 @@ def stage_flops(s: LayerShape) -> dict:
     }
 
 
+def inactive_stages(s: LayerShape) -> set:
+    """Stages that the library does not run for this shape: head size 128
+    takes the single-pass attention backward, other head sizes the two
+    kernels."""
+    return {"bwd_attn_dkdv", "bwd_attn_dq"} if s.dh == 128 else {"bwd_attn_fused", "bwd_attn_dq_convert"}
+
+
 def hbm_stage_bytes(s: LayerShape) -> dict:
     """Algorithmic HBM bytes of one launch of each memory-bound stage: every
     tensor the stage reads or writes, once (gains and norm statistics
