@@ -4,6 +4,10 @@ and compare them with the oracle under the acceptance bounds."""
 
 from __future__ import annotations
 
+import json
+import os
+import time
+
 import numpy as np
 import torch
 
@@ -93,3 +97,25 @@ def assert_close(name: str, gpu: np.ndarray, ref: np.ndarray, report: dict | Non
     if report is not None:
         report[name] = (mx, mn)
     assert mx <= bmax and mn <= bmean, f"{name}: max-abs {mx:.3e} (bound {bmax:.1e}), mean-abs {mn:.3e} (bound {bmean:.1e})"
+
+
+class OracleTimer:
+    """Wall time of an oracle run inside a GPU test.  Printed always; appended
+    as a JSON line to the file named by TSP_ORACLE_TIMES when that is set
+    (how the oracle's host-side cost is measured on the GPU machine)."""
+
+    def __init__(self, label: str, **meta):
+        self.label, self.meta = label, meta
+
+    def __enter__(self):
+        self.t0 = time.perf_counter()
+        return self
+
+    def __exit__(self, *exc):
+        sec = time.perf_counter() - self.t0
+        rec = dict(label=self.label, seconds=round(sec, 2), cores=os.cpu_count(), **self.meta)
+        print("oracle time", json.dumps(rec))
+        path = os.environ.get("TSP_ORACLE_TIMES")
+        if path and exc[0] is None:
+            with open(path, "a") as f:
+                f.write(json.dumps(rec) + "\n")

@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 import oracle as O
 from synth_inputs import WORKLOADS, LayerShape, bits_to_f32, input_hash, make_layer_inputs, sample_rows
-from tests.gpu_helpers import GpuLayer, assert_close, errors, host_f64, oracle_weights
+from tests.gpu_helpers import GpuLayer, OracleTimer, assert_close, errors, host_f64, oracle_weights
 from tests.tolerances import bound_for
 
 GRADS = ("dx", "dg1", "dwqkv", "dwo", "dg2", "dw1", "dw2")
@@ -42,10 +42,13 @@ def _run(shape, seed, training):
 def _oracle(shape, inp, zig, training):
     w = oracle_weights(inp)
     x = bits_to_f32(inp["x"][zig]).astype(np.float64)
-    z, cache = O.tsp_layer_forward(x, w, shape.heads, shape.D)
+    meta = dict(S=shape.S, D=shape.D, h=shape.h, heads=shape.heads, ffn=shape.ffn)
+    with OracleTimer("folded forward", **meta):
+        z, cache = O.tsp_layer_forward(x, w, shape.heads, shape.D)
     g = None
     if training:
-        g = O.tsp_layer_backward(bits_to_f32(inp["dy"][zig]).astype(np.float64), w, cache)
+        with OracleTimer("folded backward", **meta):
+            g = O.tsp_layer_backward(bits_to_f32(inp["dy"][zig]).astype(np.float64), w, cache)
     del cache
     return z, g
 
