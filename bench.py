@@ -112,7 +112,9 @@ def hbm_stage_bytes(s: LayerShape) -> dict:
         "bwd_convert_dy": 3 * S * h * 2,                                  # dY read twice, fp16 copy written
         "bwd_rmsnorm2": S * h * (4 + 4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,  # db, y, dY -> dy f32+fp16
         "bwd_rmsnorm1": S * h * (4 + 2 + 4 + 2) + S * 4 + 2 * partials + h * 8,      # da, x, dy -> dx bf16
-        "bwd_attn_delta": S * h * (2 + 2) + S * H * 4,                    # O, dO -> delta f32 [H][S]
+        # O, dO -> delta f32 [H][S]; head size 128 also reads K, V for the dQ
+        # bound and clears the 32-bit dQ sum
+        "bwd_attn_delta": S * h * (2 + 2) + S * H * 4 + (S * h * (2 + 2 + 4) if s.dh == 128 else 0),
         "bwd_attn_dq_convert": S * h * (4 + 2),                           # dQ sum f32 -> dQ fp16
     }
 

@@ -94,13 +94,27 @@ CUtensorMapSwizzle swz_of() {
 }
 
 // ---------------------------------------------------------------------------
-// Delta[h][row] = sum_d dO * O per (row, head), one warp at a time over a
-// grid-stride loop.  For the single-pass kernel (acc non-null) it also clears
-// the (row, head) slice of the integer dQ sum and takes, per head, the
-// largest |dO_row|^2, |V_row|^2 and |K|_max that bound the sum (dq_frac_bits):
-// per block in shared memory, then one atomicMax per head and block into
-// `bound` (cleared before the launch; non-negative float bits order like
-// unsigned integers, so the maxima do not depend on the order).
+// Delta[h][row] = sum_d dO * O per (row, head).  A warp takes 256 contiguous
+// elements of one row per item of a grid-stride loop: dh/8 lanes per head,
+// 16-byte loads, so a warp covers 256/dh heads (lanes past the last head sit
+// out).  For the single-pass kernel (acc non-null) it also clears the
+// (row, head) slice of the integer dQ sum and takes, per head, the largest
+// |dO_row|^2, |V_row|^2 and |K|_max that bound the sum (dq_frac_bits): per
+// block in shared memory, then one atomicMax per head and block into `bound`
+// (cleared before the launch; non-negative float bits order like unsigned
+// integers, so the maxima do not depend on the order).
+__device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b) {
+    return f16_lo(a.x) * f16_lo(b.x) + f16_hi(a.x) * f16_hi(b.x) + f16_lo(a.y) * f16_lo(b.y) +
+           f16_hi(a.y) * f16_hi(b.y) + f16_lo(a.z) * f16_lo(b.z) + f16_hi(a.z) * f16_hi(b.z) +
+           f16_lo(a.w) * f16_lo(b.w) + f16_hi(a.w) * f16_hi(b.w);
+}
+__device__ __forceinline__ float absmax8(const uint4 &a) {
+    float m = fmaxf(fabsf(f16_lo(a.x)), fabsf(f16_hi(a.x)));
+    m = fmaxf(m, fmaxf(fabsf(f16_lo(a.y)), fabsf(f16_hi(a.y))));
+    m = fmaxf(m, fmaxf(fabsf(f16_lo(a.z)), fabsf(f16_hi(a.z))));
+    return fmaxf(m, fmaxf(fabsf(f16_lo(a.w)), fabsf(f16_hi(a.w))));
+}
+
 __global__ void attn_delta_kernel(const __half *o, const __half *dout, const __half *kk, const __half *vv,
                                   float *delta, int *acc, unsigned int *bound, int S, int H, int dh) {
     extern __shared__ unsigned int smax[];  // [H][3]
@@ -110,42 +124,51 @@ __global__ void attn_delta_kernel(const __half *o, const __half *dout, const __h
         __syncthreads();
     }
     const int lane = threadIdx.x % 32;
+    const int lph = dh / 8;                   // lanes per head (4, 8 or 16)
+    const int hpw = 32 / lph;                 // heads per warp item
+    const int groups = (H + hpw - 1) / hpw;   // warp items per row
+    const int head_in = lane / lph;
+    const int col = (lane % lph) * 8;
+    const int64_t h = static_cast<int64_t>(H) * dh;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
-    for (int64_t wi = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; wi < static_cast<int64_t>(S) * H;
-         wi += nwarps) {
-        const int64_t row = wi / H;
-        const int head = static_cast<int>(wi - row * H);
-        const int64_t base = row * H * dh + static_cast<int64_t>(head) * dh;
+    for (int64_t wi = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+         wi < static_cast<int64_t>(S) * groups; wi += nwarps) {
+        const int64_t row = wi / groups;
+        const int head = static_cast<int>(wi - row * groups) * hpw + head_in;
+        const bool on = head < H;
+        const int64_t at = row * h + static_cast<int64_t>(head) * dh + col;
         float s = 0.f, n2 = 0.f, v2 = 0.f, km = 0.f;
-        for (int c = lane * 2; c < dh; c += 64) {
-            const uint32_t a = *reinterpret_cast<const uint32_t *>(o + base + c);
-            const uint32_t b = *reinterpret_cast<const uint32_t *>(dout + base + c);
-            s += f16_lo(a) * f16_lo(b) + f16_hi(a) * f16_hi(b);
+        if (on) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(o + at);
+            const uint4 b = *reinterpret_cast<const uint4 *>(dout + at);
+            s = dot8(a, b);
             if (fused) {
-                const uint32_t kw = *reinterpret_cast<const uint32_t *>(kk + base + c);
-                const uint32_t vw = *reinterpret_cast<const uint32_t *>(vv + base + c);
-                n2 += f16_lo(b) * f16_lo(b) + f16_hi(b) * f16_hi(b);
-                v2 += f16_lo(vw) * f16_lo(vw) + f16_hi(vw) * f16_hi(vw);
-                km = fmaxf(km, fmaxf(fabsf(f16_lo(kw)), fabsf(f16_hi(kw))));
+                const uint4 kw = *reinterpret_cast<const uint4 *>(kk + at);
+                const uint4 vw = *reinterpret_cast<const uint4 *>(vv + at);
+                n2 = dot8(b, b);
+                v2 = dot8(vw, vw);
+                km = absmax8(kw);
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) delta[static_cast<int64_t>(head) * S + row] = s;
+        for (int off = lph / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        const bool first = on && col == 0;
+        if (first) delta[static_cast<int64_t>(head) * S + row] = s;
         if (fused) {
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
+            for (int off = lph / 2; off > 0; off >>= 1) {
                 n2 += __shfl_xor_sync(0xffffffffu, n2, off);
                 v2 += __shfl_xor_sync(0xffffffffu, v2, off);
                 km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, off));
             }
-            if (lane == 0) {
+            if (first) {
                 atomicMax(&smax[3 * head + 0], __float_as_uint(n2));
                 atomicMax(&smax[3 * head + 1], __float_as_uint(v2));
                 atomicMax(&smax[3 * head + 2], __float_as_uint(km));
             }
-            int4 *z = reinterpret_cast<int4 *>(acc + base);
-            for (int c = lane; c < dh / 4; c += 32) z[c] = make_int4(0, 0, 0, 0);
+            if (on) {
+                int4 *z = reinterpret_cast<int4 *>(acc + at);
+                z[0] = make_int4(0, 0, 0, 0);
+                z[1] = make_int4(0, 0, 0, 0);
+            }
         }
     }
     if (fused) {
@@ -761,27 +784,34 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 // Single-pass backward (dh = 128).  One item = (head, 128-key tile kt); steps
 // of 64 query rows over the steps that see the tile (StepWalk, ascending).
 //   TMEM columns (128 key lanes unless noted):
-//     dV [0,128)  dK [128,256)                          accumulated per item
-//     R1: S^T [256,320)  dP^T [320,384)                 fp32, one step
-//     R2: P^T [384,416)  dS^T [416,448) packed fp16     A operands of dV, dK
-//         dQ^T [448,512): lanes = head dims, columns = the step's 64 queries
-//   Per step g the MMA warp issues S^T = K Q^T and dP^T = V dO^T into R1 and,
-//   once the element-wise warps have packed P^T / dS^T into R2 and written
-//   dS^T to shared memory, dV += P^T dO and dK += dS^T Q (A from TMEM) and
-//   dQ^T = K^T dS^T (both operands from shared memory, MN-major).  R1 is
-//   released as soon as the element-wise warps have read it, so S^T / dP^T of
-//   step g+1 run on the tensor core while step g becomes P^T and dS^T.
+//     dV [0,128)  dK [128,256)                       accumulated per item
+//     R[0] [256,384), R[1] [384,512): the buffer of steps g with g % 2 = b.
+//     Within R[b], one step's columns are used three times over:
+//       [0,64) S^T fp32      -> [0,32) P^T and [32,64) dS^T packed fp16
+//                               (A operands of dV += P^T dO, dK += dS^T Q)
+//       [64,128) dP^T fp32   -> dQ^T: lanes = head dims, columns = the
+//                               step's 64 queries
+//   Step g: warp 1 issues S^T = K Q^T into R[g%2] once step g-2's dV / dK /
+//   dQ^T MMAs (which read P^T / dS^T there) are complete, and dP^T = V dO^T
+//   once step g-2's dQ^T has been drained (both operands from shared memory);
+//   the element-wise warps turn S^T into P^T while dP^T is computed, then
+//   read dP^T and, after the four groups of a TMEM lane quarter have all read
+//   S^T (a named barrier), write P^T and dS^T packed over S^T and dS^T also
+//   to shared memory (one tile per buffer);
+//   warp kMmaGWarp issues dV += P^T dO, dK += dS^T Q (A from TMEM) and
+//   dQ^T = K^T dS^T over dP^T's columns (both operands from shared memory,
+//   MN-major).  With two buffers the element-wise work of step g+1 overlaps
+//   the dV / dK / dQ^T MMAs of step g, and nothing waits on a previous
+//   step's MMAs except the reuse of a buffer two steps later.
 //   Four drain warps (one per TMEM lane quarter) take dQ^T of step g out of
-//   TMEM once its MMAs are complete, release the columns for step g+1's dQ^T
-//   and write a shared [64][128] tile of 32-bit fixed-point integers (value
-//   times 2^F_head, rounded), which one of them adds to the step's rows of the
-//   integer dQ sum in global memory with a TMA reduce-add.  The element-wise
-//   warps never wait for the drain, and the MMA warp waits for it only before
-//   the next dQ^T.  Integer
-//   addition is associative, so the sum is the same bits whatever order the
-//   CTAs' additions reach L2 in: the result is deterministic with no ordering
-//   between CTAs.  F_head comes from a bound that holds for every partial sum
-//   of the head's dQ (dq_frac_bits), so no sum can overflow.
+//   TMEM once its MMAs are complete, which frees the buffer, and add it to
+//   the step's rows of the integer dQ sum in global memory as 32-bit fixed
+//   point (value times 2^F_head, rounded): two [32][128] shared tiles in turn,
+//   each added with one TMA reduce-add.  Integer addition is associative, so
+//   the sum is the same bits whatever order the CTAs' additions reach L2 in:
+//   the result is deterministic with no ordering between CTAs.  F_head comes
+//   from a bound that holds for every partial sum of the head's dQ
+//   (dq_frac_bits), so no sum can overflow.
 template <int DH>
 struct FusedCfg {
     using C = BCfg<DH>;
@@ -792,26 +822,29 @@ struct FusedCfg {
     static constexpr int QATOM = BQ * C::SWB;
     static constexpr int VEC_BYTES = 3 * BQ * 4;
     static constexpr int DST_BYTES = 128 * BQ * 2;   // dS^T [128 keys][64 queries] fp16, 128-byte swizzle
-    static constexpr int DQ_BYTES = BQ * DH * 4;     // dQ tile [64 queries][dh] 32-bit fixed point
+    static constexpr int DQ_ROWS = 32;               // query rows of one fixed-point dQ tile
+    static constexpr int DQ_BYTES = DQ_ROWS * DH * 4;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + C::TILE_BYTES;
     static constexpr int OFF_Q = OFF_V + C::TILE_BYTES;
     static constexpr int OFF_DO = OFF_Q + QST * QTILE;
     static constexpr int OFF_VEC = OFF_DO + QST * QTILE;
-    static constexpr int OFF_DST = (OFF_VEC + QST * VEC_BYTES + 1023) / 1024 * 1024;
-    static constexpr int OFF_DQ = OFF_DST + DST_BYTES;
+    static constexpr int OFF_DST = (OFF_VEC + QST * VEC_BYTES + 1023) / 1024 * 1024;   // [2] tiles
+    static constexpr int OFF_DQ = OFF_DST + 2 * DST_BYTES;
     static constexpr int OFF_BAR = OFF_DQ + DQ_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
     static_assert(SMEM <= kMaxDynSmem, "single-pass backward tiles exceed the shared-memory limit");
-    // kv_full/empty, q_full/empty[QST], s_full, r1_free, p_full, mma_done, acc_empty, dq_free, spare, drain
-    // + TMEM slot + abort flag
-    static_assert(8 * (2 + 2 * QST + 8) + 8 <= 256, "single-pass backward barriers exceed their slot");
-    static constexpr uint32_t T_DV = 0, T_DK = 128, T_S = 256, T_DP = 320, T_PP = 384, T_PDS = 416, T_DQ = 448;
-    static_assert(T_DQ + BQ <= 512, "single-pass backward TMEM columns");
+    // kv_full/empty, q_full/empty[QST], s_full[2], dp_full[2], p_full[2], mma_done[2], buf_free[2],
+    // acc_empty, drain, drain2 + TMEM slot + abort flag
+    static_assert(8 * (2 + 2 * QST + 13) + 8 <= 256, "single-pass backward barriers exceed their slot");
+    static constexpr uint32_t T_DV = 0, T_DK = 128, T_R = 256, R_COLS = 128;
+    static constexpr uint32_t R_S = 0, R_PP = 0, R_PDS = 32, R_DP = 64, R_DQ = 64;
+    static_assert(T_R + 2 * R_COLS <= 512, "single-pass backward TMEM columns");
 };
 
 constexpr int kEwThreads = 128 * kEwGroups;
-constexpr int kFusedThreads = 64 + kEwThreads + 128;  // TMA warp, MMA warp, element-wise groups, 4 drain warps
+// TMA warp, S^T/dP^T MMA warp, element-wise groups, 4 drain warps, dV/dK/dQ^T MMA warp
+constexpr int kFusedThreads = 64 + kEwThreads + 128 + 32;
 
 struct FusedParams {
     AttnBwdDesc d;
@@ -834,14 +867,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     uint64_t *kv_full = bars + 0, *kv_empty = bars + 1;
     uint64_t *q_full = bars + 2;                // [QST]
     uint64_t *q_empty = q_full + F::QST;        // [QST]
-    uint64_t *s_full = q_empty + F::QST;        // S^T / dP^T of a step in R1
-    uint64_t *r1_free = s_full + 1;             // R1 read by every element-wise thread
-    uint64_t *p_full = r1_free + 1;             // P^T / dS^T of a step packed in R2 and dS^T in smem
-    uint64_t *mma_done = p_full + 1;            // dV / dK / dQ^T MMAs of a step complete
-    uint64_t *acc_empty = mma_done + 1;         // dV / dK of an item read out
-    uint64_t *dq_free = acc_empty + 1;          // dQ^T of a step read out of TMEM
-    uint64_t *drain = dq_free + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *s_full = q_empty + F::QST;        // [2] S^T of a step in R[b]
+    uint64_t *dp_full = s_full + 2;             // [2] dP^T of a step in R[b]
+    uint64_t *p_full = dp_full + 2;             // [2] P^T / dS^T of a step packed in R[b], dS^T in smem
+    uint64_t *mma_done = p_full + 2;            // [2] dV / dK / dQ^T MMAs of a step complete
+    uint64_t *buf_free = mma_done + 2;          // [2] dQ^T of a step read out of R[b]
+    uint64_t *acc_empty = buf_free + 2;         // dV / dK of an item read out
+    uint64_t *drain = acc_empty + 1;            // error path: each issuer's MMAs complete
+    uint64_t *drain2 = drain + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain2 + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -850,6 +884,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
     const float scale = rsqrtf(static_cast<float>(DH));
     constexpr int kDrainWarp = 2 + 4 * kEwGroups;
+    constexpr int kMmaGWarp = kDrainWarp + 4;
     int *stage = reinterpret_cast<int *>(smem + F::OFF_DQ);
 
     if (threadIdx.x == 0) {
@@ -859,13 +894,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(r1_free, kEwThreads);
-        mbar_init(p_full, kEwThreads);
-        mbar_init(mma_done, 1);
-        mbar_init(acc_empty, kEwThreads);
-        mbar_init(dq_free, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&dp_full[b], 1);
+            mbar_init(&p_full[b], kEwThreads / 32);
+            mbar_init(&mma_done[b], 1);
+            mbar_init(&buf_free[b], 4);
+        }
+        mbar_init(acc_empty, kEwThreads / 32);
         mbar_init(drain, 1);
+        mbar_init(drain2, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -916,62 +954,80 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     spin_drain(&q_full[s], (last / F::QST) & 1, err.wait_limit);
                 }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // The whole warp runs the loop; one elected lane polls and issues.
-        {
-            const bool leader = elect_one();
-            const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+    } else if (warp == 1 || warp == kMmaGWarp) {
+        // ------------------------------------------------------------ MMA issuers
+        // Two warps issue: warp 1 the S^T / dP^T MMAs of each step, warp
+        // kMmaGWarp the dV / dK / dQ^T MMAs.  Their MMAs are ordered by the
+        // barriers alone (S^T/dP^T of step g complete -> s_full -> element-wise
+        // -> p_full -> dV/dK/dQ^T of step g -> mma_done -> drain -> buf_free ->
+        // S^T/dP^T of step g+2), so neither issuer waits behind the other's
+        // queue.  In each warp the whole warp runs the loop; one elected lane
+        // polls and issues (a commit tracks the MMAs of the thread that issues
+        // it).
+        const bool leader = elect_one();
+        const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+        int item_iter = 0, g = 0;
+        bool ok = true;
+        if (warp == 1) {
             constexpr uint32_t idS = idesc_f16(128, 64, false, false);
-            constexpr uint32_t idG = idesc_f16(128, DH, false, true);
-            constexpr uint32_t idQ = idesc_f16(DH, 64, true, true);
             const uint64_t dK0 = kdesc<DH>(smem_u32(smem + F::OFF_K), 0);
             const uint64_t dV0 = kdesc<DH>(smem_u32(smem + F::OFF_V), 0);
-            // A of dQ^T = K^T: the K tile read MN-major (rows = keys, head dims
-            // contiguous in two 128-byte atoms); K steps of 16 keys advance 2 KB
-            const uint64_t dKt0 = sdesc(smem_u32(smem + F::OFF_K), C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
-            // B of dQ^T = dS^T [128 keys][64 queries]: MN-major, one atom wide
-            const uint64_t dSt0 = sdesc(smem_u32(smem + F::OFF_DST), 8192, 1024, kSwizzle128);
-            int item_iter = 0, g = 0;
-            bool ok = true;
-            auto issue_sdp = [&](int gi) -> bool {
-                const int s = gi % F::QST;
-                if (!lead_wait(leader, leader_lane, &q_full[s], (gi / F::QST) & 1, abort_flag, err)) return false;
-                if (leader) {
-                    tc_fence_after();
-                    const uint64_t dQ0 = kdesc64<DH>(smem_u32(smem + F::OFF_Q + s * F::QTILE), 0);
-                    const uint64_t dO0 = kdesc64<DH>(smem_u32(smem + F::OFF_DO + s * F::QTILE), 0);
-#pragma unroll
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_ss(tmem + F::T_S, desc_plus(dK0, kdesc_off<DH>(kk)), desc_plus(dQ0, kdesc64_off<DH>(kk)),
-                                idS, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        umma_ss(tmem + F::T_DP, desc_plus(dV0, kdesc_off<DH>(kk)), desc_plus(dO0, kdesc64_off<DH>(kk)),
-                                idS, kk > 0);
-                    umma_commit(s_full);
-                }
-                return true;
-            };
             for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int kv0 = (a.kv_order[it] / a.H) * 128;
                 if (!lead_wait(leader, leader_lane, kv_full, item_iter & 1, abort_flag, err)) break;
-                if (leader) tc_fence_after();
                 StepWalk w;
-                w.seek(vis, 0, kv0);
-                if (w.q < nq64 && !issue_sdp(g)) break;
-                bool first = true;
-                while (w.q < nq64) {
-                    StepWalk wn = w;
-                    wn.next(vis, kv0);
-                    if (wn.q < nq64) {
-                        // S^T / dP^T of the next step into R1 once R1 has been read
-                        if (!lead_wait(leader, leader_lane, r1_free, g & 1, abort_flag, err) || !issue_sdp(g + 1)) {
-                            ok = false;
-                            break;
-                        }
+                for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+                    const int s = g % F::QST, b = g & 1, n = g >> 1;
+                    const uint32_t rb = tmem + F::T_R + b * F::R_COLS;
+                    // S^T goes over step g-2's P^T / dS^T, free once its MMAs
+                    // are complete
+                    if (n > 0 && !lead_wait(leader, leader_lane, &mma_done[b], (n - 1) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
                     }
-                    if (!lead_wait(leader, leader_lane, p_full, g & 1, abort_flag, err)) {
+                    if (!lead_wait(leader, leader_lane, &q_full[s], (g / F::QST) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) {
+                        tc_fence_after();
+                        const uint64_t dQ0 = kdesc64<DH>(smem_u32(smem + F::OFF_Q + s * F::QTILE), 0);
+#pragma unroll
+                        for (int kk = 0; kk < DH / 16; ++kk)
+                            umma_ss(rb + F::R_S, desc_plus(dK0, kdesc_off<DH>(kk)),
+                                    desc_plus(dQ0, kdesc64_off<DH>(kk)), idS, kk > 0);
+                        umma_commit(&s_full[b]);
+                    }
+                    // dP^T goes over step g-2's dQ^T, free once drained
+                    if (n > 0 && !lead_wait(leader, leader_lane, &buf_free[b], (n - 1) & 1, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) {
+                        tc_fence_after();
+                        const uint64_t dO0 = kdesc64<DH>(smem_u32(smem + F::OFF_DO + s * F::QTILE), 0);
+#pragma unroll
+                        for (int kk = 0; kk < DH / 16; ++kk)
+                            umma_ss(rb + F::R_DP, desc_plus(dV0, kdesc_off<DH>(kk)),
+                                    desc_plus(dO0, kdesc64_off<DH>(kk)), idS, kk > 0);
+                        umma_commit(&dp_full[b]);
+                    }
+                }
+            }
+        } else {
+            constexpr uint32_t idG = idesc_f16(128, DH, false, true);
+            constexpr uint32_t idQ = idesc_f16(DH, 64, true, true);
+            // A of dQ^T = K^T: the K tile read MN-major (rows = keys, head dims
+            // contiguous in two 128-byte atoms); K steps of 16 keys advance 2 KB
+            const uint64_t dKt0 = sdesc(smem_u32(smem + F::OFF_K), C::ATOM_BYTES, 8 * C::SWB, C::LAYOUT);
+            for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x, ++item_iter) {
+                const int kv0 = (a.kv_order[it] / a.H) * 128;
+                if (!lead_wait(leader, leader_lane, kv_full, item_iter & 1, abort_flag, err)) break;
+                bool first = true;
+                StepWalk w;
+                for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+                    const int s = g % F::QST, b = g & 1, n = g >> 1;
+                    if (!lead_wait(leader, leader_lane, &p_full[b], n & 1, abort_flag, err)) {
                         ok = false;
                         break;
                     }
@@ -982,56 +1038,55 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         ok = false;
                         break;
                     }
-                    const int s = g % F::QST;
                     if (leader) {
                         tc_fence_after();
+                        const uint32_t rb = tmem + F::T_R + b * F::R_COLS;
                         const uint64_t gQ0 = mndesc64<DH>(smem_u32(smem + F::OFF_Q + s * F::QTILE), 0);
                         const uint64_t gO0 = mndesc64<DH>(smem_u32(smem + F::OFF_DO + s * F::QTILE), 0);
+                        // B of dQ^T = dS^T [128 keys][64 queries]: MN-major, one atom wide
+                        const uint64_t dSt0 = sdesc(smem_u32(smem + F::OFF_DST + b * F::DST_BYTES), 8192, 1024,
+                                                    kSwizzle128);
                         // A operands from TMEM: queries 16 kk .. 16 kk + 15 packed at column 8 kk
 #pragma unroll
                         for (int kk = 0; kk < F::BQ / 16; ++kk)
-                            umma_ts(tmem + F::T_DV, tmem + F::T_PP + kk * 8, desc_plus(gO0, mndesc64_off<DH>(kk)), idG,
+                            umma_ts(tmem + F::T_DV, rb + F::R_PP + kk * 8, desc_plus(gO0, mndesc64_off<DH>(kk)), idG,
                                     (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
                         for (int kk = 0; kk < F::BQ / 16; ++kk)
-                            umma_ts(tmem + F::T_DK, tmem + F::T_PDS + kk * 8, desc_plus(gQ0, mndesc64_off<DH>(kk)), idG,
+                            umma_ts(tmem + F::T_DK, rb + F::R_PDS + kk * 8, desc_plus(gQ0, mndesc64_off<DH>(kk)), idG,
                                     (!first || kk > 0) ? 1u : 0u);
-                    }
-                    // the previous step's dQ^T must be out of TMEM before this one
-                    if (g > 0 && !lead_wait(leader, leader_lane, dq_free, (g - 1) & 1, abort_flag, err)) {
-                        ok = false;
-                        break;
-                    }
-                    if (leader) {
-                        tc_fence_after();
-                        // dQ^T [dh][64] = K^T dS^T over the 128 keys, 16 at a time
+                        // dQ^T [dh][64] = K^T dS^T over the 128 keys, 16 at a time,
+                        // over dP^T's columns (read by every element-wise thread
+                        // before p_full)
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            umma_ss(tmem + F::T_DQ, desc_plus(dKt0, kk * 16 * C::SWB), desc_plus(dSt0, kk * 2048), idQ,
+                            umma_ss(rb + F::R_DQ, desc_plus(dKt0, kk * 16 * C::SWB), desc_plus(dSt0, kk * 2048), idQ,
                                     kk > 0);
-                        umma_commit(mma_done);
+                        // this step's S^T / dP^T completed before its p_full, so
+                        // the Q / dO stage is free once these MMAs are
+                        umma_commit(&mma_done[b]);
                         umma_commit(&q_empty[s]);
                     }
                     first = false;
-                    ++g;
-                    w = wn;
                 }
-                if (leader) umma_commit(kv_empty);
+                // likewise every S^T / dP^T of the item has read the K / V tile
+                // before the item's last p_full
+                if (leader && ok) umma_commit(kv_empty);
             }
-            const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
-            if (bad && leader) {
-                umma_commit(drain);
-                spin_drain(drain, 0, err.wait_limit);
-            }
-            __syncwarp();
         }
+        uint64_t *my_drain = warp == 1 ? drain : drain2;
+        const bool bad = __any_sync(0xffffffffu, !ok || *abort_flag);
+        if (bad && leader) {
+            umma_commit(my_drain);
+            spin_drain(my_drain, 0, err.wait_limit);
+        }
+        __syncwarp();
     } else if (warp < kDrainWarp) {
         // ------------------------------------------------------------ element-wise groups
         const int grp = (warp - 2) / 4;         // query columns [16 grp, 16 grp + 16) of a step
         const int quarter = warp & 3;
         const int trow = quarter * 32 + lane;   // key row of the tile = TMEM lane (head dim for dQ^T)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        uint8_t *dst_tile = smem + F::OFF_DST;
         int g = 0;
         for (int it = blockIdx.x; it < fp.num_items; it += gridDim.x) {
             const int kt = a.kv_order[it] / a.H, head = a.kv_order[it] % a.H;
@@ -1040,16 +1095,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             bool ok = true, any = false;
             StepWalk w;
             for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
-                const int s = g % F::QST;
-                if (!warp_wait(s_full, g & 1, abort_flag, err)) { ok = false; break; }
+                const int s = g % F::QST, b = g & 1, n = g >> 1;
+                const uint32_t rb = tmem + lane_off + F::T_R + b * F::R_COLS;
+                if (!warp_wait(&s_full[b], n & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
-                if (!warp_converged("S^T/dP^T TMEM load")) { ok = false; break; }
+                if (!warp_converged("S^T TMEM load")) { ok = false; break; }
                 float sv[16], dp[16];
-                tmem_ld16(tmem + lane_off + F::T_S + 16 * grp, sv);
-                tmem_ld16(tmem + lane_off + F::T_DP + 16 * grp, dp);
+                tmem_ld16(rb + F::R_S + 16 * grp, sv);
                 tmem_ld_wait();
                 tc_fence_before();
-                mbar_arrive(r1_free);
                 const float *vec = reinterpret_cast<const float *>(smem + F::OFF_VEC + s * F::VEC_BYTES);
                 const int *pos = reinterpret_cast<const int *>(vec + 128);
                 // the 64 query rows of a step lie in one zigzag chunk, so their
@@ -1061,7 +1115,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 uint32_t pk[8], dk[8];
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 l = lse4[e4], d = dl4[e4];
+                    const float4 l = lse4[e4];
                     const int e = 4 * e4;
                     // p = 2^kPOff P (the offset rides in the exponent)
                     float p0 = ex2b(fmaf(sv[e], sl2, kPOff - l.x)), p1 = ex2b(fmaf(sv[e + 1], sl2, kPOff - l.y));
@@ -1074,36 +1128,50 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     }
                     pk[2 * e4] = pack_f16(p0, p1);
                     pk[2 * e4 + 1] = pack_f16(p2, p3);
-                    // dS = P (dP - Delta), without the offset
-                    p0 *= kPOffInv;
-                    p1 *= kPOffInv;
-                    p2 *= kPOffInv;
-                    p3 *= kPOffInv;
-                    dk[2 * e4] = pack_f16(p0 * (dp[e] - d.x), p1 * (dp[e + 1] - d.y));
-                    dk[2 * e4 + 1] = pack_f16(p2 * (dp[e + 2] - d.z), p3 * (dp[e + 3] - d.w));
+                    // P without the offset, kept for dS
+                    sv[e] = p0 * kPOffInv;
+                    sv[e + 1] = p1 * kPOffInv;
+                    sv[e + 2] = p2 * kPOffInv;
+                    sv[e + 3] = p3 * kPOffInv;
                 }
-                // R2 and the dS^T tile still belong to the previous step until its
-                // MMAs complete
-                if (g > 0 && !warp_wait(mma_done, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+                // dP^T of the step (issued once the drain freed its columns)
+                if (!warp_wait(&dp_full[b], n & 1, abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                if (!warp_converged("dP^T TMEM load")) { ok = false; break; }
+                tmem_ld16(rb + F::R_DP + 16 * grp, dp);
+                tmem_ld_wait();
+                tc_fence_before();
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 d = dl4[e4];
+                    const int e = 4 * e4;
+                    // dS = P (dP - Delta)
+                    dk[2 * e4] = pack_f16(sv[e] * (dp[e] - d.x), sv[e + 1] * (dp[e + 1] - d.y));
+                    dk[2 * e4 + 1] = pack_f16(sv[e + 2] * (dp[e + 2] - d.z), sv[e + 3] * (dp[e + 3] - d.w));
+                }
+                // P^T / dS^T go over the S^T columns that the four groups of this
+                // lane quarter read: all four must have read them first
+                asm volatile("bar.sync %0, 128;" ::"r"(3 + quarter) : "memory");
                 tc_fence_after();
                 any = true;
                 if (!warp_converged("P^T/dS^T TMEM store")) { ok = false; break; }
-                tmem_st8u(tmem + lane_off + F::T_PP + 8 * grp, pk);
-                tmem_st8u(tmem + lane_off + F::T_PDS + 8 * grp, dk);
+                tmem_st8u(rb + F::R_PP + 8 * grp, pk);
+                tmem_st8u(rb + F::R_PDS + 8 * grp, dk);
                 // this key's row of dS^T: its 16 queries are the 16-byte chunks
                 // 2 grp and 2 grp + 1 of the 128-byte row, 128-byte swizzled
-                uint4 *row = reinterpret_cast<uint4 *>(dst_tile + trow * 128);
+                uint4 *row = reinterpret_cast<uint4 *>(smem + F::OFF_DST + b * F::DST_BYTES + trow * 128);
                 row[(2 * grp) ^ (trow & 7)] = make_uint4(dk[0], dk[1], dk[2], dk[3]);
                 row[(2 * grp + 1) ^ (trow & 7)] = make_uint4(dk[4], dk[5], dk[6], dk[7]);
                 tmem_st_wait();
                 fence_async_smem();
                 tc_fence_before();
-                mbar_arrive(p_full);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[b]);
             }
             if (!ok) break;
             if (!any) continue;
             // the item's last step: its MMAs complete means dV and dK are too
-            if (!warp_wait(mma_done, (g - 1) & 1, abort_flag, err)) break;
+            if (!warp_wait(&mma_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             // groups 0, 1 write dV (offset removed) and groups 2, 3 write dK
             // (scaled), at the key owner's local row; each pair splits the
@@ -1129,14 +1197,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                                         pack_f16(v[8 * qq + 4], v[8 * qq + 5]), pack_f16(v[8 * qq + 6], v[8 * qq + 7]));
             }
             tc_fence_before();
-            mbar_arrive(acc_empty);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
         }
-    } else {
+    } else if (warp < kMmaGWarp) {
         // ------------------------------------------------------------ drain warps
-        // dQ^T of every step out of TMEM (thread = head dim), into the shared
-        // fixed-point tile [query][dh], then one TMA reduce-add into the
-        // integer dQ sum.  Named barriers 1 and 2 order the four warps around
-        // the shared tile; warp kDrainWarp's first lane issues the bulk ops.
+        // dQ^T of every step out of TMEM (thread = head dim), then, 32 queries
+        // at a time, into the shared fixed-point tile [query][dh] and one TMA
+        // reduce-add into the integer dQ sum.  Named barriers 1 and 2 order the
+        // four warps around the shared tile; warp kDrainWarp's first lane
+        // issues the bulk operations.
         const int quarter = warp & 3;
         const int d = quarter * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -1148,26 +1218,33 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const float dq_scale = ldexpf(1.0f, dq_frac_bits(a.dq_bound + 3 * head, DH));
             StepWalk w;
             for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
-                if (!warp_wait(mma_done, g & 1, abort_flag, err)) { ok = false; break; }
+                const int b = g & 1, n = g >> 1;
+                if (!warp_wait(&mma_done[b], n & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();
                 if (!warp_converged("dQ^T TMEM load")) { ok = false; break; }
                 float v[64];
-                tmem_ld32(tmem + lane_off + F::T_DQ, *reinterpret_cast<float(*)[32]>(v));
-                tmem_ld32(tmem + lane_off + F::T_DQ + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                const uint32_t rb = tmem + lane_off + F::T_R + b * F::R_COLS;
+                tmem_ld32(rb + F::R_DQ, *reinterpret_cast<float(*)[32]>(v));
+                tmem_ld32(rb + F::R_DQ + 32, *reinterpret_cast<float(*)[32]>(v + 32));
                 tmem_ld_wait();
                 tc_fence_before();
-                mbar_arrive(dq_free);
-                // the previous tile has been read by its bulk operation
-                if (issuer) bulk_wait_read_all();
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&buf_free[b]);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) stage[j * DH + d] = __float2int_rn(v[j] * dq_scale);
-                fence_async_smem();
-                asm volatile("bar.sync 2, 128;" ::: "memory");
-                if (issuer) {
-                    fence_async_global();
-                    tma_reduce_add_2d(&mDQ, stage, head * DH, w.q * 64);
-                    bulk_commit();
+                for (int half = 0; half < 2; ++half) {
+                    // the previous tile has been read by its bulk operation
+                    if (issuer) bulk_wait_read_all();
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < F::DQ_ROWS; ++j)
+                        stage[j * DH + d] = __float2int_rn(v[half * F::DQ_ROWS + j] * dq_scale);
+                    fence_async_smem();
+                    asm volatile("bar.sync 2, 128;" ::: "memory");
+                    if (issuer) {
+                        fence_async_global();
+                        tma_reduce_add_2d(&mDQ, stage, head * DH, w.q * 64 + half * F::DQ_ROWS);
+                        bulk_commit();
+                    }
                 }
             }
         }
@@ -1274,14 +1351,14 @@ cudaError_t launch_fused_impl(const AttnBwdDesc &a, const DevErr &err, int num_s
     using C = BCfg<DH>;
     BwdMaps<DH> m;
     if (!m.make(a)) return cudaErrorInvalidValue;
-    // Q and dO sub-tiles of 64 rows; the fp32 dQ sum in [dh x 64] boxes
+    // Q and dO sub-tiles of 64 rows; the 32-bit dQ sum in [dh x 32] boxes
     const int h = a.H * DH;
     const auto swz = swz_of<DH>();
     bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
     ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
     CUtensorMap mdq;
-    ok = ok && encode_tensor_map_2d(&mdq, a.dq_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, h, a.S, int64_t(h) * 4, DH, 64,
-                                    CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && encode_tensor_map_2d(&mdq, a.dq_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, h, a.S, int64_t(h) * 4, DH,
+                                    FusedCfg<DH>::DQ_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
     FusedParams fp;
     fp.d = a;
@@ -1321,7 +1398,9 @@ cudaError_t launch_attn_delta(const AttnBwdDesc &a, int num_sms, cudaStream_t st
         cudaError_t e = cudaMemsetAsync(a.dq_bound, 0, static_cast<size_t>(3) * a.H * sizeof(unsigned int), st);
         if (e != cudaSuccess) return e;
     }
-    const int64_t warps = static_cast<int64_t>(a.S) * a.H;
+    if (a.dh % 8 || a.dh < 8 || a.dh > 256 || 32 % (a.dh / 8)) return cudaErrorInvalidValue;
+    const int hpw = 256 / a.dh;
+    const int64_t warps = static_cast<int64_t>(a.S) * ((a.H + hpw - 1) / hpw);
     const int64_t want = (warps * 32 + 255) / 256;
     const int blocks = static_cast<int>(want < 8LL * num_sms ? want : 8LL * num_sms);
     attn_delta_kernel<<<blocks, 256, static_cast<size_t>(3) * a.H * sizeof(unsigned int), st>>>(
