@@ -46,10 +46,11 @@ NOMINAL_TFLOPS = 2250.0   # dense bf16/fp16 datasheet figure
 NOMINAL_MHZ = 1965.0      # clocks.max.sm of this part
 
 # DRAM bytes (read + write) of one launch from an ncu capture of the current
-# kernel build, and the S of that capture.  The traffic is the compulsory one
-# and grows in proportion to S, so it is scaled by S to the benchmarked
-# launch.  Must be re-measured (or removed) whenever the kernel changes.
-MEASURED_TRAFFIC = {"bwd_attn_fused": (1297.982e6 + 949.780e6, 16384)}
+# kernel build (dram__bytes_read.sum + dram__bytes_write.sum, one ncu pass, at
+# the benchmark's size), and the S of that capture.  At another S the figure
+# is scaled by S, which holds only while re-reads stay in L2.  Must be
+# re-measured (or removed) whenever the kernel changes.
+MEASURED_TRAFFIC = {"bwd_attn_fused": (54.14e9 + 37.32e9, 131072)}
 
 
 def peaks():
@@ -472,8 +473,9 @@ def main():
                      "frac_of_nominal_at_run_clock": achieved / at_clock,
                      "traffic": (MEASURED_TRAFFIC[dom][0] * S / MEASURED_TRAFFIC[dom][1]) if dom in MEASURED_TRAFFIC
                      else None,
-                     "traffic_note": "ncu dram bytes of one launch at a smaller S scaled by S" if dom in MEASURED_TRAFFIC
-                     else "not measured for this kernel build",
+                     "traffic_note": ("not measured for this kernel build" if dom not in MEASURED_TRAFFIC
+                                      else "ncu dram bytes of one launch at this S" if MEASURED_TRAFFIC[dom][1] == S
+                                      else "ncu dram bytes of one launch at another S scaled by S"),
                      "peak_note": f"{src} sustained bf16 (kernel timed inside a long step)"},
         "hbm_stages": {k: {"bytes": b, "ms": stages[k][0] / max(stages[k][1], 1),
                            "achieved": b / (stages[k][0] / max(stages[k][1], 1) / 1e3) / 1e9,

@@ -782,7 +782,9 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 
 // ---------------------------------------------------------------------------
 // Single-pass backward (dh = 128).  One item = (head, 128-key tile kt); steps
-// of 64 query rows over the steps that see the tile (StepWalk, ascending).
+// of 64 query rows over the steps that see the tile, in descending order of
+// position (DescWalk): the items that run at the same time walk the same
+// query rows in step, which keeps Q, dO and the dQ sum of those rows in L2.
 //   TMEM columns (128 key lanes unless noted):
 //     dV [0,128)  dK [128,256)                       accumulated per item
 //     R[0] [256,384), R[1] [384,512): the buffer of steps g with g % 2 = b.
@@ -929,8 +931,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     tma_load_2d(smem + F::OFF_K + t * C::ATOM_BYTES, &mK, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
                     tma_load_2d(smem + F::OFF_V + t * C::ATOM_BYTES, &mV, kv_full, head * DH + t * C::ATOM_COLS, kt * 128);
                 }
-                StepWalk w;
-                for (w.seek(vis, 0, kt * 128); w.q < nq64; w.next(vis, kt * 128), ++g) {
+                DescWalk w;
+                for (w.seek(vis, kt * 128); w.q < nq64; w.next(vis, kt * 128), ++g) {
                     const int q = w.q;
                     const int s = g % F::QST;
                     if (!mbar_wait(&q_empty[s], ((g / F::QST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
@@ -975,8 +977,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x, ++item_iter) {
                 const int kv0 = (a.kv_order[it] / a.H) * 128;
                 if (!lead_wait(leader, leader_lane, kv_full, item_iter & 1, abort_flag, err)) break;
-                StepWalk w;
-                for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+                DescWalk w;
+                for (w.seek(vis, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
                     const int s = g % F::QST, b = g & 1, n = g >> 1;
                     const uint32_t rb = tmem + F::T_R + b * F::R_COLS;
                     // S^T goes over step g-2's P^T / dS^T, free once its MMAs
@@ -1024,8 +1026,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const int kv0 = (a.kv_order[it] / a.H) * 128;
                 if (!lead_wait(leader, leader_lane, kv_full, item_iter & 1, abort_flag, err)) break;
                 bool first = true;
-                StepWalk w;
-                for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+                DescWalk w;
+                for (w.seek(vis, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
                     const int s = g % F::QST, b = g & 1, n = g >> 1;
                     if (!lead_wait(leader, leader_lane, &p_full[b], n & 1, abort_flag, err)) {
                         ok = false;
@@ -1093,8 +1095,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int kv0 = kt * 128;
             const int key = kv0 + trow;
             bool ok = true, any = false;
-            StepWalk w;
-            for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+            DescWalk w;
+            for (w.seek(vis, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
                 const int s = g % F::QST, b = g & 1, n = g >> 1;
                 const uint32_t rb = tmem + lane_off + F::T_R + b * F::R_COLS;
                 if (!warp_wait(&s_full[b], n & 1, abort_flag, err)) { ok = false; break; }
@@ -1216,8 +1218,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x) {
             const int head = a.kv_order[it] % a.H, kv0 = (a.kv_order[it] / a.H) * 128;
             const float dq_scale = ldexpf(1.0f, dq_frac_bits(a.dq_bound + 3 * head, DH));
-            StepWalk w;
-            for (w.seek(vis, 0, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
+            DescWalk w;
+            for (w.seek(vis, kv0); w.q < nq64; w.next(vis, kv0), ++g) {
                 const int b = g & 1, n = g >> 1;
                 if (!warp_wait(&mma_done[b], n & 1, abort_flag, err)) { ok = false; break; }
                 tc_fence_after();

@@ -183,6 +183,47 @@ struct StepWalk {
     }
 };
 
+// Walks the query steps that can see a key tile kv0 in descending order of
+// position: position chunks from the last (2D-1) down, each chunk's steps from
+// its last down to its lowest visible one.  Every walk is then a prefix of one
+// common order (the steps of the highest positions, visible to every key tile,
+// come first), so key tiles processed at the same time touch the same query
+// rows at about the same time and those rows stay in L2.  Host-callable so
+// that tests can replay the walk.
+struct DescWalk {
+    int q;     // current local step; nq64 once the walk is over
+    int pc;    // position chunk of q: positions [pc chunk, (pc + 1) chunk)
+    int t;     // step of q within its chunk
+    int t_lo;  // lowest step of the chunk that reaches kv0
+    __host__ __device__ inline void enter(const StepVis &v, int kv0) {
+        const int spc = v.chunk >> 6;
+        // step t of chunk pc ends at position pc chunk + 64 t + 63
+        const int need = kv0 - 63 - pc * v.chunk;
+        t_lo = need <= 0 ? 0 : (need + 63) / 64;
+        if (pc < 0 || t_lo >= spc) {  // nothing here, and lower chunks lie lower still
+            q = v.nq64;
+            return;
+        }
+        t = spc - 1;
+        // local rows: rank r holds chunk r, then chunk 2D-1-r
+        const int lc = pc < v.D ? 2 * pc : 2 * (2 * v.D - 1 - pc) + 1;
+        q = lc * spc + t;
+    }
+    __host__ __device__ inline void seek(const StepVis &v, int kv0) {
+        pc = 2 * v.D - 1;
+        enter(v, kv0);
+    }
+    __host__ __device__ inline void next(const StepVis &v, int kv0) {
+        if (t > t_lo) {
+            --t;
+            --q;
+        } else {
+            --pc;
+            enter(v, kv0);
+        }
+    }
+};
+
 struct AttnBwdDesc {
     int S, L, D, H, dh, chunk;
     const void *q, *k, *v, *o, *dout;  // q, o, dout local rows; k, v global rows

@@ -189,8 +189,63 @@ HostTables host_tables(const tsp_plan_s *p) {
     return t;
 }
 
+// Pairs every head's j-th longest item with its j-th shortest and deals the
+// pairs in waves: the attention kernels hand items round-robin to G
+// persistent CTAs (CTA i takes items i, i + G, ...), so a wave of G pairs is
+// laid out as the G long items, then the G short ones in the same CTA order.
+// Under causality the two items of a pair add up to the same length for every
+// pair (key tile kt and key tile N-1-kt together see S/64 + 2 query steps),
+// so every CTA finishes a wave at about the same time and the next wave starts
+// in step, without a barrier.  Together with walks that start from a common
+// end (the backward walks query steps from the top position down, the forward
+// walks key tiles from 0 up) the rows that the CTAs touch at one time stay
+// within one wave's length differences, a few MB, instead of spreading over
+// the whole head (128 MB at S = 128K), which is more than L2 holds.
+// `order` is head-major with the longest items of a head first (host_tables);
+// `width` table entries per item.
+void pair_waves(std::vector<int32_t> &order, int width, int H, int G) {
+    const int64_t n = static_cast<int64_t>(order.size()) / width;
+    std::vector<int64_t> longs, shorts;  // item indices into `order`
+    int64_t start = 0;
+    while (start < n) {
+        const int head = order[start * width] % H;
+        int64_t end = start;
+        while (end < n && order[end * width] % H == head) ++end;
+        const int64_t m = end - start;
+        for (int64_t j = 0; j < m / 2; ++j) {
+            longs.push_back(start + j);
+            shorts.push_back(end - 1 - j);
+        }
+        if (m & 1) {  // the middle item pairs with nothing
+            longs.push_back(start + m / 2);
+            shorts.push_back(-1);
+        }
+        start = end;
+    }
+    std::vector<int32_t> out;
+    out.reserve(order.size());
+    const int64_t np = static_cast<int64_t>(longs.size());
+    auto emit = [&](int64_t idx) {
+        if (idx >= 0)
+            for (int k = 0; k < width; ++k) out.push_back(order[idx * width + k]);
+    };
+    for (int64_t w0 = 0; w0 < np; w0 += G) {
+        const int64_t w1 = std::min<int64_t>(w0 + G, np);
+        for (int64_t j = w0; j < w1; ++j) emit(longs[j]);
+        for (int64_t j = w0; j < w1; ++j) emit(shorts[j]);
+    }
+    order.swap(out);
+}
+
+// The work orders as uploaded for a device with G SMs.  The dQ kernel's
+// order (head sizes 32 and 64) keeps the host order.
+void device_orders(HostTables &t, int H, int G) {
+    pair_waves(t.forder, 2, H, G);
+    pair_waves(t.korder, 1, H, G);
+}
+
 // Device tables: map, inverse map, per-query-tile max position and the work
-// orders of the attention kernels (head-major, longest item first per head).
+// orders of the attention kernels (paired in waves, pair_waves).
 tsp_status ensure_device(tsp_plan_s *p) {
     std::lock_guard<std::mutex> g(p->mu);
     int dev = 0;
@@ -200,7 +255,8 @@ tsp_status ensure_device(tsp_plan_s *p) {
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return TSP_ERR_CUDA;
     if (prop.major != 10) return TSP_ERR_UNSUPPORTED;
     if (!get_encode()) return TSP_ERR_CUDA;
-    const HostTables t = host_tables(p);
+    HostTables t = host_tables(p);
+    device_orders(t, p->H, prop.multiProcessorCount);
 
     auto upload = [](int32_t **dst, const std::vector<int32_t> &v) {
         if (cudaMalloc(dst, v.size() * 4) != cudaSuccess) return false;
@@ -850,6 +906,36 @@ TSP_API tsp_status tsp_test_tables(tsp_plan_t p, int which, int32_t *out, int64_
     if (*count > capacity) return TSP_ERR_INVALID_ARG;
     std::copy(v->begin(), v->end(), out);
     return TSP_OK;
+}
+
+TSP_API tsp_status tsp_test_work_order(tsp_plan_t p, int which, int num_ctas, int32_t *out, int64_t capacity,
+                                       int64_t *count) {
+    if (!p || !count || capacity < 0 || (capacity > 0 && !out) || num_ctas < 1) return TSP_ERR_INVALID_ARG;
+    HostTables t = host_tables(p);
+    device_orders(t, p->H, num_ctas);
+    const std::vector<int32_t> *v = nullptr;
+    switch (which) {
+        case 2: v = &t.forder; break;
+        case 3: v = &t.korder; break;
+        case 4: v = &t.qorder; break;
+        default: return TSP_ERR_INVALID_ARG;
+    }
+    *count = static_cast<int64_t>(v->size());
+    if (*count > capacity) return TSP_ERR_INVALID_ARG;
+    std::copy(v->begin(), v->end(), out);
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_test_step_walk_desc(tsp_plan_t p, int kv0, int32_t *steps, int capacity, int *count) {
+    if (!p || !count || capacity < 0 || (capacity > 0 && !steps)) return TSP_ERR_INVALID_ARG;
+    if (kv0 < 0 || kv0 >= p->S) return TSP_ERR_INVALID_ARG;
+    const StepVis vis{p->D, static_cast<int>(p->c), static_cast<int>(p->S / 64)};
+    int n = 0;
+    DescWalk w;
+    for (w.seek(vis, kv0); w.q < vis.nq64; w.next(vis, kv0), ++n)
+        if (n < capacity) steps[n] = w.q;
+    *count = n;
+    return n <= capacity ? TSP_OK : TSP_ERR_INVALID_ARG;
 }
 
 TSP_API tsp_status tsp_test_step_walk(tsp_plan_t p, int kv0, int32_t *steps, int capacity, int *count) {

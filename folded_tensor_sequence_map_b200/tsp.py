@@ -51,7 +51,9 @@ EXPORTED = (
     "tsp_test_buffer_offset",
     "tsp_test_next_visible",
     "tsp_test_step_walk",
+    "tsp_test_step_walk_desc",
     "tsp_test_tables",
+    "tsp_test_work_order",
     "tsp_test_wait_timeout",
 )
 TSP_NUM_STAGES = 24
@@ -102,8 +104,12 @@ def _load() -> ctypes.CDLL:
     lib.tsp_test_next_visible.restype = I
     lib.tsp_test_step_walk.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I, ctypes.POINTER(I)]
     lib.tsp_test_step_walk.restype = I
+    lib.tsp_test_step_walk_desc.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I, ctypes.POINTER(I)]
+    lib.tsp_test_step_walk_desc.restype = I
     lib.tsp_test_tables.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I64, ctypes.POINTER(I64)]
     lib.tsp_test_tables.restype = I
+    lib.tsp_test_work_order.argtypes = [P, I, I, ctypes.POINTER(ctypes.c_int32), I64, ctypes.POINTER(I64)]
+    lib.tsp_test_work_order.restype = I
     lib.tsp_profile_enable.argtypes = [P, I]
     lib.tsp_profile_enable.restype = I
     lib.tsp_profile_read.argtypes = [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
@@ -353,12 +359,13 @@ def tsp_test_next_visible(plan: Plan, start: int, kv0: int) -> int:
     return out.value
 
 
-def tsp_test_step_walk(plan: Plan, kv0: int) -> np.ndarray:
+def tsp_test_step_walk(plan: Plan, kv0: int, descending: bool = False) -> np.ndarray:
     cap = plan.S // 64
     out = np.zeros(cap, dtype=np.int32)
     n = ctypes.c_int()
-    _check(_lib.tsp_test_step_walk(plan.handle, kv0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cap,
-                                   ctypes.byref(n)), "tsp_test_step_walk")
+    fn = _lib.tsp_test_step_walk_desc if descending else _lib.tsp_test_step_walk
+    name = "tsp_test_step_walk_desc" if descending else "tsp_test_step_walk"
+    _check(fn(plan.handle, kv0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cap, ctypes.byref(n)), name)
     return out[:n.value].copy()
 
 
@@ -372,6 +379,16 @@ def tsp_test_tables(plan: Plan, name: str) -> np.ndarray:
     out = np.zeros(n.value, dtype=np.int32)
     _check(_lib.tsp_test_tables(plan.handle, which, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n.value,
                                 ctypes.byref(n)), "tsp_test_tables")
+    return out
+
+
+def tsp_test_work_order(plan: Plan, name: str, num_ctas: int) -> np.ndarray:
+    n = ctypes.c_int64()
+    which = TABLES[name]
+    _lib.tsp_test_work_order(plan.handle, which, num_ctas, None, 0, ctypes.byref(n))
+    out = np.zeros(n.value, dtype=np.int32)
+    _check(_lib.tsp_test_work_order(plan.handle, which, num_ctas, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                    n.value, ctypes.byref(n)), "tsp_test_work_order")
     return out
 
 

@@ -74,6 +74,22 @@ tsp_status tsp_test_tables(tsp_plan_t plan, int which, int32_t *out, int64_t cap
  * walk longer than `capacity`. */
 tsp_status tsp_test_step_walk(tsp_plan_t plan, int kv0, int32_t *steps, int capacity, int *count);
 
+/* The same work orders (which = 2, 3, 4 as above) as the plan uploads them
+ * for a device with `num_ctas` SMs: every other round of num_ctas consecutive
+ * items reversed, so that the persistent CTAs, which take items i, i +
+ * num_ctas, ..., draw long and short items in turn and stay in step.
+ * TSP_ERR_INVALID_ARG for another `which`, num_ctas < 1, a NULL pointer or a
+ * table longer than `capacity`. */
+tsp_status tsp_test_work_order(tsp_plan_t plan, int which, int num_ctas, int32_t *out, int64_t capacity,
+                               int64_t *count);
+
+/* Host replay of the walk the single-pass attention backward makes over the
+ * 64-row query steps that can see the key tile starting at position kv0: the
+ * same steps as tsp_test_step_walk, in descending order of position (chunks
+ * from the last, each from its last step down), so that every walk is a
+ * prefix of the walk for kv0 = 0.  Output and errors as tsp_test_step_walk. */
+tsp_status tsp_test_step_walk_desc(tsp_plan_t plan, int kv0, int32_t *steps, int capacity, int *count);
+
 /* Self-test of the bounded device-side wait used by every kernel: launches one
  * CTA that waits on an mbarrier nothing ever completes, with a limit of
  * `limit_cycles` SM cycles.  The wait gives up, the kernel writes 0 to

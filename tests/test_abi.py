@@ -89,6 +89,88 @@ def test_step_walk_visits_exactly_the_visible_steps(h, H, F, S, D):
 
 
 @pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
+                                       (256, 4, 1024, 2048, 1), (4096, 32, 16384, 131072, 8)])
+def test_descending_walk_is_a_prefix_of_one_order(h, H, F, S, D):
+    """The single-pass backward's walk for a key tile at kv0 visits exactly the
+    64-row local steps holding a row at a position >= kv0 (oracle zigzag map),
+    once each, in strictly descending order of position, and is a prefix of
+    the walk for kv0 = 0 (so key tiles walked at the same time touch the same
+    query rows)."""
+    p = T.tsp_plan(h, H, F, S, D)
+    nq = S // 64
+    zig = O.zigzag_map(S, D).ravel().reshape(nq, 64)
+    step_max, step_min = zig.max(axis=1), zig.min(axis=1)
+    full = T.tsp_test_step_walk(p, 0, descending=True)
+    assert np.array_equal(np.sort(full), np.arange(nq))
+    assert np.all(np.diff(step_min[full]) < 0) and np.all(step_max[full][1:] < step_min[full][:-1])
+    rng = np.random.default_rng(S * 5 + D)
+    tiles = np.unique(np.concatenate([[0, 1, S // 256, S // 128 - 1], rng.integers(0, S // 128, 24)]))
+    for kt in tiles:
+        kv0 = int(kt) * 128
+        walk = T.tsp_test_step_walk(p, kv0, descending=True)
+        assert np.array_equal(np.sort(walk), np.nonzero(step_max >= kv0)[0]), (S, D, kv0)
+        assert np.array_equal(walk, full[:len(walk)]), (S, D, kv0)
+
+
+def _start_spread(cost, G):
+    """Largest gap, over the rounds of G items, between the first and the last
+    start time of a round's items when CTA i runs items i, i + G, ... at one
+    unit of time per unit of cost."""
+    n = len(cost)
+    t = np.zeros(G)
+    worst = 0
+    for r0 in range(0, n, G):
+        c = cost[r0:r0 + G]
+        worst = max(worst, t[:len(c)].max() - t[:len(c)].min())
+        t[:len(c)] += c
+    return worst
+
+
+@pytest.mark.parametrize("G", [1, 7, 148])
+@pytest.mark.parametrize("S", [4096, 32768, 131072])
+def test_uploaded_work_orders_pair_long_and_short_items(G, S):
+    """The orders the plan uploads for G SMs: every item once; within a head
+    the j-th longest item pairs with the j-th shortest, a wave of G pairs laid
+    out as the long items then the short ones.  So CTA i (items i, i + G, ...)
+    runs one pair per wave, every pair has the same length up to rounding, and
+    the CTAs start each round's items within one wave's length differences of
+    each other: with the head-major host order the starts drift apart by a
+    whole walk."""
+    h, H, F, D = 4096, 32, 16384, 8
+    p = T.tsp_plan(h, H, F, S, D)
+    zig = O.zigzag_map(S, D).ravel()
+    steps = np.array([(zig.reshape(S // 64, 64).max(axis=1) >= kt * 128).sum() for kt in range(S // 128)])
+    for name, width in (("fwd_order", 2), ("kv_order", 1)):
+        base = T.tsp_test_tables(p, name).reshape(-1, width)
+        up = T.tsp_test_work_order(p, name, G).reshape(-1, width)
+        assert np.array_equal(np.sort(up[:, 0]), np.sort(base[:, 0])), (name, G)
+        if width == 2:
+            assert np.array_equal(up[np.argsort(up[:, 0])], base[np.argsort(base[:, 0])])
+        cost = up[:, 1] if width == 2 else steps[up[:, 0] // H]
+        n = len(cost)
+        npairs = n // 2
+        for w0 in range(0, npairs, G):
+            w1 = min(w0 + G, npairs)
+            longs, shorts = cost[2 * w0:2 * w0 + (w1 - w0)], cost[2 * w0 + (w1 - w0):2 * w1]
+            heads_l = up[2 * w0:2 * w0 + (w1 - w0), 0] % H
+            heads_s = up[2 * w0 + (w1 - w0):2 * w1, 0] % H
+            assert np.array_equal(heads_l, heads_s)
+            assert np.all(longs >= shorts)
+            pair = longs + shorts
+            assert pair.max() - pair.min() <= 2, (name, G, w0)
+        if G == 148 and S >= 32768:
+            base_cost = base[:, 1] if width == 2 else steps[base[:, 0] // H]
+            paired, plain = _start_spread(cost, G), _start_spread(base_cost, G)
+            # a round's starts differ by at most the long items' length range
+            # of a wave; without pairing they drift by a whole walk and more
+            assert paired <= cost.max() - cost.min() and paired * 4 < plain, (name, paired, plain)
+    with pytest.raises(T.TSPError):
+        T.tsp_test_work_order(p, "kv_order", 0)
+    with pytest.raises(T.TSPError):
+        T.tsp_test_work_order(p, "inv", G)
+
+
+@pytest.mark.parametrize("h,H,F,S,D", [(128, 4, 512, 256, 2), (4096, 32, 16384, 8192, 8), (2048, 16, 4096, 4096, 16),
                                        (256, 4, 1024, 2048, 1), (4096, 32, 16384, 32768, 8)])
 def test_kernel_tables_match_the_zigzag_map(h, H, F, S, D):
     """The tables the plan uploads, rebuilt from the oracle's zigzag map: the
