@@ -808,8 +808,9 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 //   Four drain warps (one per TMEM lane quarter) take dQ^T of step g out of
 //   TMEM once its MMAs are complete, which frees the buffer, and add it to
 //   the step's rows of the integer dQ sum in global memory as 32-bit fixed
-//   point (value times 2^F_head, rounded): two [32][128] shared tiles in turn,
-//   each added with one TMA reduce-add.  Integer addition is associative, so
+//   point (value times 2^F_head, rounded), one global reduction per element
+//   (a warp's reductions for one query row cover one 128-byte line).  Integer
+//   addition is associative, so
 //   the sum is the same bits whatever order the CTAs' additions reach L2 in:
 //   the result is deterministic with no ordering between CTAs.  F_head comes
 //   from a bound that holds for every partial sum of the head's dQ
@@ -824,16 +825,13 @@ struct FusedCfg {
     static constexpr int QATOM = BQ * C::SWB;
     static constexpr int VEC_BYTES = 3 * BQ * 4;
     static constexpr int DST_BYTES = 128 * BQ * 2;   // dS^T [128 keys][64 queries] fp16, 128-byte swizzle
-    static constexpr int DQ_ROWS = 32;               // query rows of one fixed-point dQ tile
-    static constexpr int DQ_BYTES = DQ_ROWS * DH * 4;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + C::TILE_BYTES;
     static constexpr int OFF_Q = OFF_V + C::TILE_BYTES;
     static constexpr int OFF_DO = OFF_Q + QST * QTILE;
     static constexpr int OFF_VEC = OFF_DO + QST * QTILE;
     static constexpr int OFF_DST = (OFF_VEC + QST * VEC_BYTES + 1023) / 1024 * 1024;   // [2] tiles
-    static constexpr int OFF_DQ = OFF_DST + 2 * DST_BYTES;
-    static constexpr int OFF_BAR = OFF_DQ + DQ_BYTES;
+    static constexpr int OFF_BAR = OFF_DST + 2 * DST_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
     static_assert(SMEM <= kMaxDynSmem, "single-pass backward tiles exceed the shared-memory limit");
     // kv_full/empty, q_full/empty[QST], s_full[2], dp_full[2], p_full[2], mma_done[2], buf_free[2],
@@ -858,7 +856,7 @@ template <int DH>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                           const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
-                          const __grid_constant__ CUtensorMap mDQ, const FusedParams fp, const DevErr err) {
+                          const FusedParams fp, const DevErr err) {
     using C = BCfg<DH>;
     using F = FusedCfg<DH>;
     const AttnBwdDesc &a = fp.d;
@@ -887,7 +885,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const float scale = rsqrtf(static_cast<float>(DH));
     constexpr int kDrainWarp = 2 + 4 * kEwGroups;
     constexpr int kMmaGWarp = kDrainWarp + 4;
-    int *stage = reinterpret_cast<int *>(smem + F::OFF_DQ);
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -1204,15 +1201,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
     } else if (warp < kMmaGWarp) {
         // ------------------------------------------------------------ drain warps
-        // dQ^T of every step out of TMEM (thread = head dim), then, 32 queries
-        // at a time, into the shared fixed-point tile [query][dh] and one TMA
-        // reduce-add into the integer dQ sum.  Named barriers 1 and 2 order the
-        // four warps around the shared tile; warp kDrainWarp's first lane
-        // issues the bulk operations.
+        // dQ^T of every step out of TMEM (thread = head dim), which frees the
+        // buffer, then added to the integer dQ sum in global memory with one
+        // reduction per element.  Measured against staging the integers in
+        // shared memory for TMA reduce-adds, this is faster: the drain's time
+        // per step no longer delays the buffer's next use.
         const int quarter = warp & 3;
         const int d = quarter * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const bool issuer = warp == kDrainWarp && lane == 0;
+        const int hh = a.H * DH;
         int g = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < fp.num_items && ok; it += gridDim.x) {
@@ -1232,25 +1229,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&buf_free[b]);
+                // one global reduction per element: a warp's 32 head dims of one
+                // query row are one 128-byte line
+                int *col = a.dq_acc + static_cast<int64_t>(w.q) * 64 * hh + head * DH + d;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    // the previous tile has been read by its bulk operation
-                    if (issuer) bulk_wait_read_all();
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-#pragma unroll
-                    for (int j = 0; j < F::DQ_ROWS; ++j)
-                        stage[j * DH + d] = __float2int_rn(v[half * F::DQ_ROWS + j] * dq_scale);
-                    fence_async_smem();
-                    asm volatile("bar.sync 2, 128;" ::: "memory");
-                    if (issuer) {
-                        fence_async_global();
-                        tma_reduce_add_2d(&mDQ, stage, head * DH, w.q * 64 + half * F::DQ_ROWS);
-                        bulk_commit();
-                    }
-                }
+                for (int j = 0; j < 64; ++j) atomicAdd(col + j * hh, __float2int_rn(v[j] * dq_scale));
             }
         }
-        if (issuer) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -1353,14 +1338,11 @@ cudaError_t launch_fused_impl(const AttnBwdDesc &a, const DevErr &err, int num_s
     using C = BCfg<DH>;
     BwdMaps<DH> m;
     if (!m.make(a)) return cudaErrorInvalidValue;
-    // Q and dO sub-tiles of 64 rows; the 32-bit dQ sum in [dh x 32] boxes
+    // Q and dO sub-tiles of 64 rows
     const int h = a.H * DH;
     const auto swz = swz_of<DH>();
     bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
     ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
-    CUtensorMap mdq;
-    ok = ok && encode_tensor_map_2d(&mdq, a.dq_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, h, a.S, int64_t(h) * 4, DH,
-                                    FusedCfg<DH>::DQ_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
     FusedParams fp;
     fp.d = a;
@@ -1371,7 +1353,7 @@ cudaError_t launch_fused_impl(const AttnBwdDesc &a, const DevErr &err, int num_s
     auto k = attn_bwd_fused_kernel<DH>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<grid, kFusedThreads, FusedCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, mdq, fp, err);
+    k<<<grid, kFusedThreads, FusedCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, fp, err);
     return cudaGetLastError();
 }
 

@@ -136,34 +136,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// The same between the generic and the async proxy for global memory.
-__device__ __forceinline__ void fence_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-// TMA tile store and tile reduce-add (fp32 add in L2) of a shared-memory box
-// to global memory, tracked by this thread's bulk async-group.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *src, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(smem_u32(src)), "r"(x), "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *m, const void *src, int x, int y) {
-    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(smem_u32(src)), "r"(x), "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until every bulk operation this thread committed has completed (its
-// global writes performed).
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Wait until every committed bulk operation of this thread has finished
-// reading its shared-memory source (the source may then be rewritten).
-__device__ __forceinline__ void bulk_wait_read_all() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
 
 // ---- tcgen05 ------------------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100 "version 1" format):
