@@ -312,6 +312,102 @@ def run_reference(args, shape: LayerShape, seed: int):
 
 
 # ---------------------------------------------------------------------------
+# GPU run: a stack of layers (--layers)
+# ---------------------------------------------------------------------------
+
+def run_stack(args, shape: LayerShape, seed: int):
+    """One step = forward + backward of `layers` folded layers with
+    activation recompute (tsp_stack_forward / tsp_stack_backward).  For
+    timing, every layer holds its own device copy of one layer's drawn
+    weights (the values do not change the work).  Algorithmic FLOPs count
+    each layer's forward and backward once; the recomputed forwards are
+    reported apart."""
+    import torch
+
+    import folded_tensor_sequence_map_b200 as T
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    rank, world = dist_setup("nccl")
+    n, S, h, F = args.layers, shape.S, shape.h, shape.ffn
+    bf = torch.bfloat16
+    plan = T.tsp_plan(shape.h, shape.heads, shape.ffn, shape.S, shape.D)
+    zig = T.tsp_zigzag_map(plan)
+    inp = make_layer_inputs(shape, seed)
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(bf).to(dev)
+    x = torch.from_numpy(np.ascontiguousarray(inp["x"][zig]).view(np.int16)).view(bf).to(dev)
+    dz = torch.from_numpy(np.ascontiguousarray(inp["dy"][zig]).view(np.int16)).view(bf).to(dev)
+    W = {k: [to_dev(inp[k]) for _ in range(n)] for k in ("wqkv", "wo", "w1", "w2")}
+    G = {k: [torch.from_numpy(inp[k]).to(dev) for _ in range(n)] for k in ("g1", "g2")}
+    del inp
+    ws_n, saved_n, inputs_n = T.tsp_stack_workspace_size(plan, n)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+    saved = torch.empty(saved_n, dtype=torch.uint8, device=dev)
+    inputs = torch.empty(inputs_n, dtype=torch.uint8, device=dev)
+    z = torch.empty(S, h, dtype=bf, device=dev)
+    dx = torch.empty(S, h, dtype=bf, device=dev)
+    grads = {"dg1": [torch.empty(h, device=dev) for _ in range(n)],
+             "dwqkv": [torch.empty(3 * h, h, device=dev) for _ in range(n)],
+             "dwo": [torch.empty(h, h, device=dev) for _ in range(n)],
+             "dg2": [torch.empty(h, device=dev) for _ in range(n)],
+             "dw1": [torch.empty(F, h, device=dev) for _ in range(n)],
+             "dw2": [torch.empty(h, F, device=dev) for _ in range(n)]}
+    stream = torch.cuda.current_stream(dev)
+    wargs = (G["g1"], W["wqkv"], W["wo"], G["g2"], W["w1"], W["w2"])
+
+    def step():
+        T.tsp_stack_forward(plan, x, *wargs, z, inputs, saved, ws, stream)
+        T.tsp_stack_backward(plan, dz, x, *wargs, inputs, saved, ws, dx, grads["dg1"], grads["dwqkv"],
+                             grads["dwo"], grads["dg2"], grads["dw1"], grads["dw2"], stream)
+
+    for _ in range(args.warmup):
+        step()
+    T.tsp_sync_status(plan, stream)
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    launches0 = T.tsp_kernel_launches(plan)
+    with ClockSampler(gpu_id) as clk:
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+    T.tsp_sync_status(plan, stream)
+    t = reduce_max(a.elapsed_time(b) / 1e3, dev)
+    launches = T.tsp_kernel_launches(plan) - launches0
+    burst, sustained, _, src = peaks()
+    flops = n * step_flops(shape)
+    recompute = (n - 1) * layer_flops(shape, False)
+    line = {
+        "metric": f"TSP stack tokens/s (fwd+bwd, {n} layers, activation recompute) at S={S}, D={shape.D}",
+        "value": world * S * args.steps / t, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic (every layer a copy of one layer's drawn weights)",
+        "config": {"workload": f"{args.workload}_stack{n}" + (f"_seq{S}" if args.seq else ""), "layers": n, "h": h, "heads": shape.heads, "ffn": F,
+                   "seq_len": S, "D": shape.D, "global_batch": 1,
+                   "parallelism": "virtual ranks on one device; replicas across GPUs",
+                   "l2": "inputs larger than L2"},
+        "fwd_bwd_frac_of_bf16_peak": flops * args.steps / t / 1e12 / sustained,
+        "with_recompute_frac_of_bf16_peak": (flops + recompute) * args.steps / t / 1e12 / sustained,
+        "peak_source": f"{src} sustained {sustained} TFLOP/s",
+        "device_memory_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 1),
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
 # GPU run
 # ---------------------------------------------------------------------------
 
@@ -326,6 +422,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--seq", type=int, default=0, help="override S of the workload (profiling runs)")
     ap.add_argument("--ranks", type=int, default=0, help="override D of the workload (D sweep)")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="time a stack of this many layers with activation recompute instead of one layer")
     args = ap.parse_args()
     shape, seed = WORKLOADS[args.workload]
     if args.seq or args.ranks:
@@ -333,6 +431,9 @@ def main():
                            D=args.ranks or shape.D)
     if args.impl == "reference":
         run_reference(args, shape, seed)
+        return
+    if args.layers > 1:
+        run_stack(args, shape, seed)
         return
 
     import torch

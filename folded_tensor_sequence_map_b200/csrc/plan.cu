@@ -843,6 +843,106 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
 // Test hooks (tsp_testing.h)
 // ===========================================================================
 
+// ===========================================================================
+// Stack of layers with activation recompute (tsp.h)
+// ===========================================================================
+
+namespace {
+// The part of a stack's workspace that one layer call uses: the backward's
+// scratch, or the intermediates of an inference forward, whichever is larger.
+size_t stack_layer_ws(const tsp_plan_s *p) {
+    const Layout l = layout_of(p);
+    return std::max(l.bwd_total, l.saved_total);
+}
+bool all_set(int n, const void *const *v) {
+    if (!v) return false;
+    for (int i = 0; i < n; ++i)
+        if (!v[i] || !aligned16(v[i])) return false;
+    return true;
+}
+}  // namespace
+
+TSP_API tsp_status tsp_stack_workspace_size(tsp_plan_t p, int layers, size_t *ws_bytes, size_t *saved_bytes,
+                                            size_t *inputs_bytes) {
+    if (!p || layers < 1) return TSP_ERR_INVALID_ARG;
+    const size_t act = static_cast<size_t>(p->S) * p->h * 2;  // one bf16 [S][h] tensor
+    if (ws_bytes) *ws_bytes = stack_layer_ws(p) + 3 * act;
+    if (saved_bytes) *saved_bytes = layout_of(p).saved_total;
+    if (inputs_bytes) *inputs_bytes = static_cast<size_t>(layers - 1) * act;
+    return TSP_OK;
+}
+
+
+
+TSP_API tsp_status tsp_stack_forward(tsp_plan_t p, int layers, const void *x, const float *const *g1,
+                                     const void *const *wqkv, const void *const *wo, const float *const *g2,
+                                     const void *const *w1, const void *const *w2, void *z, void *inputs,
+                                     void *saved, void *ws, void *stream) {
+    if (!p || layers < 1 || !x || !z || !ws || !g1 || !wqkv || !wo || !g2 || !w1 || !w2) return TSP_ERR_INVALID_ARG;
+    if (saved && layers > 1 && !inputs) return TSP_ERR_INVALID_ARG;
+    if (!all_set(layers, reinterpret_cast<const void *const *>(g1)) || !all_set(layers, wqkv) ||
+        !all_set(layers, wo) || !all_set(layers, reinterpret_cast<const void *const *>(g2)) ||
+        !all_set(layers, w1) || !all_set(layers, w2))
+        return TSP_ERR_INVALID_ARG;
+    for (const void *q : {x, (const void *)z, (const void *)ws})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    if ((saved && !aligned16(saved)) || (inputs && !aligned16(inputs))) return TSP_ERR_ALIGNMENT;
+    const size_t act = static_cast<size_t>(p->S) * p->h * 2;
+    // inference: layer outputs alternate between two scratch tensors after the layer workspace
+    uint8_t *scratch = static_cast<uint8_t *>(ws) + stack_layer_ws(p);
+    const void *in = x;
+    for (int i = 0; i < layers; ++i) {
+        void *out = i == layers - 1 ? z
+                    : saved         ? static_cast<void *>(static_cast<uint8_t *>(inputs) + static_cast<size_t>(i) * act)
+                                    : static_cast<void *>(scratch + static_cast<size_t>(i & 1) * act);
+        const tsp_status st =
+            tsp_layer_forward(p, in, g1[i], wqkv[i], wo[i], g2[i], w1[i], w2[i], out, saved, ws, stream);
+        if (st != TSP_OK) return st;
+        in = out;
+    }
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_stack_backward(tsp_plan_t p, int layers, const void *dz, const void *x,
+                                      const float *const *g1, const void *const *wqkv, const void *const *wo,
+                                      const float *const *g2, const void *const *w1, const void *const *w2,
+                                      const void *inputs, void *saved, void *ws, void *dx, float *const *dg1,
+                                      float *const *dwqkv, float *const *dwo, float *const *dg2, float *const *dw1,
+                                      float *const *dw2, void *stream) {
+    if (!p || layers < 1 || !dz || !x || !saved || !ws || !dx || (layers > 1 && !inputs) || !g1 || !wqkv || !wo ||
+        !g2 || !w1 || !w2 || !dg1 || !dwqkv || !dwo || !dg2 || !dw1 || !dw2)
+        return TSP_ERR_INVALID_ARG;
+    auto cv = [](const auto *const *v) { return reinterpret_cast<const void *const *>(v); };
+    if (!all_set(layers, cv(g1)) || !all_set(layers, wqkv) || !all_set(layers, wo) || !all_set(layers, cv(g2)) ||
+        !all_set(layers, w1) || !all_set(layers, w2) || !all_set(layers, cv(dg1)) || !all_set(layers, cv(dwqkv)) ||
+        !all_set(layers, cv(dwo)) || !all_set(layers, cv(dg2)) || !all_set(layers, cv(dw1)) ||
+        !all_set(layers, cv(dw2)))
+        return TSP_ERR_INVALID_ARG;
+    for (const void *q : {dz, x, (const void *)saved, (const void *)ws, (const void *)dx})
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    if (inputs && !aligned16(inputs)) return TSP_ERR_ALIGNMENT;
+    const size_t act = static_cast<size_t>(p->S) * p->h * 2;
+    uint8_t *scratch = static_cast<uint8_t *>(ws) + stack_layer_ws(p);
+    void *grad[2] = {scratch, scratch + act};  // gradients between layers, in turn
+    void *znew = scratch + 2 * act;            // output of a recomputed forward (not used)
+    const void *g = dz;
+    for (int i = layers - 1; i >= 0; --i) {
+        const void *in = i == 0 ? x : static_cast<const uint8_t *>(inputs) + static_cast<size_t>(i - 1) * act;
+        // the top layer's intermediates are still in `saved` from the forward
+        if (i != layers - 1) {
+            const tsp_status st =
+                tsp_layer_forward(p, in, g1[i], wqkv[i], wo[i], g2[i], w1[i], w2[i], znew, saved, ws, stream);
+            if (st != TSP_OK) return st;
+        }
+        void *out = i == 0 ? dx : grad[i & 1];
+        const tsp_status st = tsp_layer_backward(p, g, in, g1[i], wqkv[i], wo[i], g2[i], w1[i], w2[i], saved, ws,
+                                                 out, dg1[i], dwqkv[i], dwo[i], dg2[i], dw1[i], dw2[i], stream);
+        if (st != TSP_OK) return st;
+        g = out;
+    }
+    return TSP_OK;
+}
+
 TSP_API tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A, int64_t lda, const void *B,
                                  int64_t ldb, float *C, int64_t ldc, int force_bn128, int f16, void *stream) {
     if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0) return TSP_ERR_INVALID_ARG;

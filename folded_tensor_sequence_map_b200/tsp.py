@@ -40,6 +40,9 @@ EXPORTED = (
     "tsp_ring_mlp_workspace_size",
     "tsp_ring_mlp_forward",
     "tsp_layer_backward",
+    "tsp_stack_workspace_size",
+    "tsp_stack_forward",
+    "tsp_stack_backward",
     "tsp_sync_status",
     "tsp_status_string",
     "tsp_layer_flops",
@@ -90,6 +93,12 @@ def _load() -> ctypes.CDLL:
     lib.tsp_ring_mlp_forward.restype = I
     lib.tsp_layer_backward.argtypes = [P] + [V] * 18
     lib.tsp_layer_backward.restype = I
+    lib.tsp_stack_workspace_size.argtypes = [P, I, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]
+    lib.tsp_stack_workspace_size.restype = I
+    lib.tsp_stack_forward.argtypes = [P, I] + [V] * 12
+    lib.tsp_stack_forward.restype = I
+    lib.tsp_stack_backward.argtypes = [P, I] + [V] * 19
+    lib.tsp_stack_backward.restype = I
     lib.tsp_sync_status.argtypes = [P, V]
     lib.tsp_sync_status.restype = I
     lib.tsp_status_string.argtypes = [I]
@@ -303,6 +312,57 @@ def tsp_layer_backward(plan: Plan, dy, x, g1, wqkv, wo, g2, w1, w2, saved, ws, d
         _stream(stream),
     ]
     _check(_lib.tsp_layer_backward(plan.handle, *args), "tsp_layer_backward")
+
+
+def tsp_stack_workspace_size(plan: Plan, layers: int):
+    ws, saved, inputs = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.tsp_stack_workspace_size(plan.handle, layers, ctypes.byref(ws), ctypes.byref(saved),
+                                         ctypes.byref(inputs)), "tsp_stack_workspace_size")
+    return ws.value, saved.value, inputs.value
+
+
+def _ptr_array(ts, name, dtype, shape):
+    """Host array of device pointers, one per layer (kept alive by the caller
+    of the C function through the returned object)."""
+    arr = (ctypes.c_void_p * len(ts))(*[_ptr(t, f"{name}[{i}]", dtype, shape) for i, t in enumerate(ts)])
+    return arr
+
+
+def tsp_stack_forward(plan: Plan, x, g1, wqkv, wo, g2, w1, w2, z, inputs, saved, ws, stream=None) -> None:
+    """g1, wqkv, wo, g2, w1, w2: sequences with one tensor per layer."""
+    import torch
+
+    h, F, S, n = plan.h, plan.ffn, plan.S, len(wqkv)
+    bf, f32 = torch.bfloat16, torch.float32
+    arrs = [_ptr_array(g1, "g1", f32, (h,)), _ptr_array(wqkv, "wqkv", bf, (3 * h, h)),
+            _ptr_array(wo, "wo", bf, (h, h)), _ptr_array(g2, "g2", f32, (h,)),
+            _ptr_array(w1, "w1", bf, (F, h)), _ptr_array(w2, "w2", bf, (h, F))]
+    if any(len(a) != n for a in arrs):
+        raise ValueError("one tensor per layer in every weight list")
+    _check(_lib.tsp_stack_forward(plan.handle, n, _ptr(x, "x", bf, (S, h)), *[ctypes.cast(a, ctypes.c_void_p) for a in arrs],
+                                  _ptr(z, "z", bf, (S, h)), _ptr(inputs, "inputs"), _ptr(saved, "saved"),
+                                  _ptr(ws, "ws"), _stream(stream)), "tsp_stack_forward")
+
+
+def tsp_stack_backward(plan: Plan, dz, x, g1, wqkv, wo, g2, w1, w2, inputs, saved, ws, dx, dg1, dwqkv, dwo, dg2,
+                       dw1, dw2, stream=None) -> None:
+    """Weight and gradient arguments: sequences with one tensor per layer."""
+    import torch
+
+    h, F, S, n = plan.h, plan.ffn, plan.S, len(wqkv)
+    bf, f32 = torch.bfloat16, torch.float32
+    arrs = [_ptr_array(g1, "g1", f32, (h,)), _ptr_array(wqkv, "wqkv", bf, (3 * h, h)),
+            _ptr_array(wo, "wo", bf, (h, h)), _ptr_array(g2, "g2", f32, (h,)),
+            _ptr_array(w1, "w1", bf, (F, h)), _ptr_array(w2, "w2", bf, (h, F))]
+    grads = [_ptr_array(dg1, "dg1", f32, (h,)), _ptr_array(dwqkv, "dwqkv", f32, (3 * h, h)),
+             _ptr_array(dwo, "dwo", f32, (h, h)), _ptr_array(dg2, "dg2", f32, (h,)),
+             _ptr_array(dw1, "dw1", f32, (F, h)), _ptr_array(dw2, "dw2", f32, (h, F))]
+    if any(len(a) != n for a in arrs + grads):
+        raise ValueError("one tensor per layer in every weight and gradient list")
+    _check(_lib.tsp_stack_backward(plan.handle, n, _ptr(dz, "dz", bf, (S, h)), _ptr(x, "x", bf, (S, h)),
+                                   *[ctypes.cast(a, ctypes.c_void_p) for a in arrs], _ptr(inputs, "inputs"), _ptr(saved, "saved"),
+                                   _ptr(ws, "ws"), _ptr(dx, "dx", bf, (S, h)), *[ctypes.cast(a, ctypes.c_void_p) for a in grads],
+                                   _stream(stream)), "tsp_stack_backward")
 
 
 def tsp_sync_status(plan: Plan, stream=None) -> None:

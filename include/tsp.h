@@ -197,6 +197,52 @@ tsp_status tsp_layer_backward(tsp_plan_t plan, const void *dy, const void *x, co
                               float *dwqkv, float *dwo, float *dg2, float *dw1, float *dw2,
                               void *stream);
 
+/* A stack of `layers` folded layers with activation recompute: the model the
+ * pages measure is such a stack (a 7B decoder of 32 of these layers, zubnet.ai
+ * page "Zyphra TSP folds TP+SP onto one GPU axis, 2.6x throughput on 1,024
+ * MI300Xs", paragraph 1).  Layer i has its own weights and gains; the host
+ * arrays g1[i], wqkv[i], ... hold `layers` device pointers each (layouts as
+ * for tsp_layer_forward).  Between layers the activations and gradients are
+ * bf16 [S][h] in rank-major zigzag order, as at the layer's own boundary.
+ *
+ * tsp_stack_workspace_size: bytes of
+ *   ws      scratch of one layer call plus three bf16 [S][h] tensors
+ *   saved   one layer's saved intermediates (as tsp_workspace_size)
+ *   inputs  the inputs of layers 1 .. layers-1, bf16 [layers-1][S][h]
+ * Needs no GPU.  TSP_ERR_INVALID_ARG for layers < 1. */
+tsp_status tsp_stack_workspace_size(tsp_plan_t plan, int layers, size_t *ws_bytes, size_t *saved_bytes,
+                                    size_t *inputs_bytes);
+
+/* Forward of the stack: z = layer_{L-1}( ... layer_0(x)).  With `saved`
+ * (training) every layer's input except the first is kept in `inputs` and
+ * the last layer's intermediates in `saved`, for tsp_stack_backward; with
+ * saved = NULL (inference) `inputs` is not used and the layers' outputs go
+ * through the scratch at the end of `ws`.  Device pointers x, z bf16 [S][h];
+ * ws, saved, inputs of tsp_stack_workspace_size's sizes.  Errors as for
+ * tsp_layer_forward, and TSP_ERR_INVALID_ARG for layers < 1, a NULL pointer
+ * in a weight array, or saved without inputs when layers > 1. */
+tsp_status tsp_stack_forward(tsp_plan_t plan, int layers, const void *x, const float *const *g1,
+                             const void *const *wqkv, const void *const *wo, const float *const *g2,
+                             const void *const *w1, const void *const *w2, void *z, void *inputs, void *saved,
+                             void *ws, void *stream);
+
+/* Backward of the stack after a training tsp_stack_forward with the same
+ * pointers: from the last layer down, every layer but the last is run
+ * forward again from its kept input (activation recompute, into `saved`),
+ * then backward; the gradient of a layer's input is the next lower layer's
+ * output gradient (bf16 [S][h], two scratch tensors in turn at the end of
+ * `ws`).  Device pointers: dz bf16 [S][h] (gradient of z, input); dx bf16
+ * [S][h] (output); per-layer gradient arrays dg1[i], dwqkv[i], dwo[i], dg2[i],
+ * dw1[i], dw2[i] as for tsp_layer_backward (outputs, overwritten).  `saved`
+ * is overwritten.  Errors as for tsp_layer_backward, and TSP_ERR_INVALID_ARG
+ * for layers < 1, a NULL pointer in an array, or inputs = NULL when
+ * layers > 1. */
+tsp_status tsp_stack_backward(tsp_plan_t plan, int layers, const void *dz, const void *x, const float *const *g1,
+                              const void *const *wqkv, const void *const *wo, const float *const *g2,
+                              const void *const *w1, const void *const *w2, const void *inputs, void *saved,
+                              void *ws, void *dx, float *const *dg1, float *const *dwqkv, float *const *dwo,
+                              float *const *dg2, float *const *dw1, float *const *dw2, void *stream);
+
 /* Wait for `stream`, then report TSP_ERR_CUDA for an asynchronous CUDA error,
  * TSP_ERR_TIMEOUT if a device-side wait of this plan ran out, or TSP_ERR_RANGE
  * if a value overflowed an fp16 intermediate (the flags are cleared by the

@@ -497,6 +497,50 @@ def tsp_layer_backward(dz_local, w, cache):
                 dw1=dw1, dw2=dw2)
 
 
+# ---------------------------------------------------------------------------
+# A stack of folded layers  [Z1]: the measured model is a stack of these
+# layers (a 7B decoder); between layers the tensors are bf16 (the layer's
+# boundary dtype)
+# ---------------------------------------------------------------------------
+
+def round_bf16(x):
+    """Round fp64 values to the nearest bfloat16 value (8 significand bits,
+    ties to even), returned as fp64.  The values here are finite and far from
+    bfloat16's range limits."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                    # x = m 2^e with 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def tsp_stack_forward(x_local, ws, H, D, round_interfaces=True):
+    """z = layer_{L-1}(... layer_0(x)) with every layer the folded layer of
+    ``tsp_layer_forward`` (weights ``ws[i]`` for layer i); the activation
+    between two layers is rounded to bf16 unless ``round_interfaces`` is
+    False.  Returns (z, caches), z unrounded."""
+    caches = []
+    cur = np.asarray(x_local, dtype=np.float64)
+    z = None
+    for i, w in enumerate(ws):
+        z, cache = tsp_layer_forward(cur, w, H, D)
+        caches.append(cache)
+        cur = round_bf16(z) if round_interfaces and i < len(ws) - 1 else z
+    return z, caches
+
+
+def tsp_stack_backward(dz_local, ws, caches, round_interfaces=True):
+    """Gradients of the stack: layer i's backward (``tsp_layer_backward``) on
+    the gradient of its output, from the last layer down; the gradient
+    passed to the layer below is rounded to bf16 unless ``round_interfaces``
+    is False.  Returns one gradient dict per layer; the stack's dx is
+    grads[0]["dx"]."""
+    grads = [None] * len(ws)
+    g = np.asarray(dz_local, dtype=np.float64)
+    for i in reversed(range(len(ws))):
+        grads[i] = tsp_layer_backward(g, ws[i], caches[i])
+        g = round_bf16(grads[i]["dx"]) if round_interfaces and i > 0 else grads[i]["dx"]
+    return grads
+
+
 def tsp_forward_rows(x_local, w, H, D, rows, eps=EPS):
     """Folded forward restricted to the rank-major rows ``rows``.
 

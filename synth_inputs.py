@@ -89,6 +89,32 @@ def make_layer_inputs(shape: LayerShape, seed: int, with_dy: bool = True) -> dic
     return out
 
 
+def make_layer_weights(shape: LayerShape, seed: int) -> dict:
+    """Draw one layer's weights alone: Wqkv, Wo, W1, W2 from
+    ``default_rng(seed)`` in that order (times 0.02, rounded to bf16), gains
+    ones.  Used for the layers of a stack, each with its own seed."""
+    h, F = shape.h, shape.ffn
+    rng = np.random.default_rng(seed)
+    out = {}
+    for name, shp in (("wqkv", (3 * h, h)), ("wo", (h, h)), ("w1", (F, h)), ("w2", (h, F))):
+        w = rng.standard_normal(shp, dtype=np.float32)
+        w *= np.float32(WEIGHT_STD)
+        out[name] = bf16_bits(w)
+    out["g1"] = np.ones(h, dtype=np.float32)
+    out["g2"] = np.ones(h, dtype=np.float32)
+    return out
+
+
+def make_stack_inputs(shape: LayerShape, layers: int, seed: int) -> dict:
+    """Inputs of a stack of ``layers`` layers: x and dY as make_layer_inputs
+    draws them for ``seed``, and layer i's weights from
+    make_layer_weights(shape, seed * 1000 + 1 + i).  Returns dict(x, dy,
+    layers=[weights of layer 0, ...])."""
+    inp = make_layer_inputs(shape, seed)
+    return dict(x=inp["x"], dy=inp["dy"],
+                layers=[make_layer_weights(shape, seed * 1000 + 1 + i) for i in range(layers)])
+
+
 def sample_rows(S: int, n: int, seed: int) -> np.ndarray:
     """Seeded sample of ``n`` distinct row indices in [0, S) that always
     includes the first and the last row; sorted ascending."""

@@ -212,6 +212,45 @@ def test_kernel_tables_match_the_zigzag_map(h, H, F, S, D):
     assert T.STATUS_NAMES[rc] == "TSP_ERR_INVALID_ARG"
 
 
+def test_stack_checks_arguments_before_enqueueing():
+    """tsp_stack_forward / tsp_stack_backward refuse a bad layer count, a NULL
+    in a weight or gradient array, or a misaligned pointer before anything
+    runs (the addresses are never dereferenced); the workspace sizes follow
+    the layer's: one layer's saved buffer, the layer scratch plus three
+    activations, and layers-1 kept inputs."""
+    h, H, F, S, D = 128, 4, 512, 256, 2
+    p = T.tsp_plan(h, H, F, S, D)
+    ws1, saved1 = T.tsp_workspace_size(p, True)
+    ws_inf, _ = T.tsp_workspace_size(p, False)
+    act = S * h * 2
+    for n in (1, 3, 32):
+        ws, saved, inputs = T.tsp_stack_workspace_size(p, n)
+        assert saved == saved1 and inputs == (n - 1) * act and ws == max(ws1, ws_inf) + 3 * act
+    V = ctypes.c_void_p
+    arr = lambda n, base=0x100000: (V * n)(*[base + 0x1000 * i for i in range(n)])
+    lib = TT._lib
+    st = lambda rc: T.STATUS_NAMES[rc]
+    good = dict(x=0x20000, z=0x30000, inputs=0x40000, saved=0x50000, ws=0x60000)
+    fwd = lambda n, arrs, **kw: lib.tsp_stack_forward(p.handle, n, V(kw.get("x", good["x"])),
+                                                        *[ctypes.cast(a, V) for a in arrs], V(kw.get("z", good["z"])),
+                                                        V(good["inputs"]), V(good["saved"]), V(good["ws"]), V(0))
+    six = [arr(3) for _ in range(6)]
+    assert st(fwd(0, six)) == "TSP_ERR_INVALID_ARG"
+    holey = [arr(3) for _ in range(6)]
+    holey[2][1] = None
+    assert st(fwd(3, holey)) == "TSP_ERR_INVALID_ARG"
+    assert st(fwd(3, six, x=good["x"] + 8)) == "TSP_ERR_ALIGNMENT"
+    bwd = lambda n, arrs, grads, dx=0x70000: lib.tsp_stack_backward(
+        p.handle, n, V(0x80000), V(good["x"]), *[ctypes.cast(a, V) for a in arrs], V(good["inputs"]),
+        V(good["saved"]), V(good["ws"]), V(dx), *[ctypes.cast(a, V) for a in grads], V(0))
+    grads = [arr(3, 0x900000) for _ in range(6)]
+    assert st(bwd(0, six, grads)) == "TSP_ERR_INVALID_ARG"
+    gholey = [arr(3, 0x900000) for _ in range(6)]
+    gholey[5][2] = None
+    assert st(bwd(3, six, gholey)) == "TSP_ERR_INVALID_ARG"
+    assert st(bwd(3, six, grads, dx=0x70008)) == "TSP_ERR_ALIGNMENT"
+
+
 def test_prefill_checks_arguments_before_enqueueing():
     """tsp_layer_prefill refuses a NULL or misaligned pointer before it touches
     the device (the addresses below are never dereferenced)."""
