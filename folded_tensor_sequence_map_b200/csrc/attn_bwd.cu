@@ -9,21 +9,24 @@
 // paragraph 2 gives the forward exchange; its reverse is the reading taken
 // for the backward).
 //
-// Three kernels, no atomics (deterministic):
-//   attn_delta   Delta[h][row] = sum_d dO * O (fp16 inputs, fp32 sum).
-//   attn_dkdv2   one item = (head, 128-key tile); steps of 64 query rows over
-//                the query tiles that see any of its keys.  S^T = K Q^T and
-//                dP^T = V dO^T in TMEM; P^T and dS^T go back into TMEM as
-//                packed fp16 over the columns they were read from; dV += P^T dO
-//                and dK += dS^T Q (A operand from TMEM) accumulate in TMEM.
-//   attn_dq2     one item = (head, 128-row query tile); steps of 64 keys.
-//                S = Q K^T, dP = dO V^T in TMEM; dS back into TMEM as packed
-//                fp16; dQ += dS K.
+// Kernels (every result deterministic: no floating-point atomics):
+//   attn_delta   Delta[h][row] = sum_d dO * O (fp16 inputs, fp32 sum); for the
+//                single-pass kernel it also clears the integer dQ sum and takes
+//                the per-head maxima that set its fixed-point scale.
+//   attn_bwd_fused (head size 128) one item = (head, 128-key tile); steps of 64
+//                query rows walked from the top position down.  S^T, dP^T,
+//                then P^T / dS^T and dQ^T share two TMEM step buffers; dV and
+//                dK accumulate in TMEM; dQ^T is added to a 32-bit fixed-point
+//                sum in global memory with integer reductions (the same bits in
+//                any order), which dq_convert turns into fp16 dQ.
+//   attn_dkdv2, attn_dq2 (head sizes 32, 64) the two-kernel backward: a
+//                key-tile kernel for dK, dV (P^T and dS^T go back into TMEM as
+//                packed fp16 over the columns they were read from) and a
+//                query-tile kernel for dQ (S and dP recomputed).
 // Q, K, V, O, dO and the outputs dQ, dK, dV are fp16 (gradients in the
 // backward's scaled domain).  The P^T feeding dV carries a factor 2^kPOff so
 // small probabilities stay normal fp16 numbers; the dV epilogue takes it out.
-// Warp roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2-17 element-wise (four
-// groups of four; thread = TMEM lane = row of the 128-row tile).
+// Warp roles of each kernel are described above its definition.
 #include "common.cuh"
 #include "internal.h"
 
@@ -254,6 +257,9 @@ struct KvParams {
     int num_items;
 };
 
+// Two-kernel path: warp 0 TMA, warp 1 TMEM owner and MMA issuer, warps 2-17
+// element-wise (four groups of four; thread = TMEM lane = row of the 128-row
+// tile).
 constexpr int kEwGroups = 4;                          // element-wise groups of four warps
 constexpr int kBwdThreads2 = 64 + 128 * kEwGroups;     // + TMA warp + MMA warp
 
