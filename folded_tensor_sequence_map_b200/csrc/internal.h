@@ -133,7 +133,7 @@ struct AttnDesc {
     const void *k, *v;          // fp16 [S][h] global rows
     void *o;                    // fp16 [S][h] local rows
     float *lse;                 // f32 [H][S] local rows, log2 domain (scores pre-multiplied by log2 e / sqrt(dh))
-    const int *order;           // pairs (qblock * H + head, number of 128-key tiles), longest first
+    const int *order;           // pairs (qblock * H + head, number of 128-key tiles), in paired waves
     int num_items;
 };
 cudaError_t launch_attn_fwd(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st);
@@ -234,8 +234,8 @@ struct AttnBwdDesc {
     unsigned int *err;                 // error word (fp16 overflow of dQ, dK, dV)
     int64_t ldd;
     const int *inv_map;                // global position -> local row
-    const int *kv_order;               // work order of (head, 128-key block), longest first
-    const int *q_order;                // work order of (head, 128-row query block), longest first
+    const int *kv_order;               // work order of (head, 128-key block), in paired waves
+    const int *q_order;                // work order of (head, 128-row query block), longest first per head
     int *dq_acc;                       // [S][h] scratch: dQ summed over key tiles in 32-bit fixed point
                                        // (single-pass kernel; zeroed by the Delta kernel), or null
     unsigned int *dq_bound;            // [H][3] scratch: per-head maxima bounding that sum (Delta kernel)

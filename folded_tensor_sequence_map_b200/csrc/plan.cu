@@ -132,7 +132,8 @@ tsp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSP_OK : TSP_E
 
 // Host copies of the kernels' tables: inverse map, largest position of each
 // 128-row local query tile, and the work orders of the attention kernels
-// (head-major, longest item first per head).  Needs no GPU.
+// (head-major, longest item first per head; the forward and dK/dV orders are
+// paired in waves before upload, device_orders).  Needs no GPU.
 struct HostTables {
     std::vector<int32_t> inv, qmax, forder, korder, qorder;
 };
@@ -156,9 +157,10 @@ HostTables host_tables(const tsp_plan_s *p) {
         int32_t m = std::max(qmax[2 * qb], qmax[2 * qb + 1]);
         for (int hd = 0; hd < H; ++hd) fitems.push_back({static_cast<int>(qb * H + hd), m / 128 + 1});
     }
-    // Head-major, longest first within a head: the CTAs running at the same
-    // time then share one head's K/V (64 MiB at S = 128K) in L2 instead of
-    // streaming every head's K/V from HBM.
+    // Head-major, longest first within a head (then paired in waves for the
+    // device, pair_waves): the CTAs running at the same time share one head's
+    // K/V (64 MiB at S = 128K) in L2 instead of streaming every head's K/V
+    // from HBM.
     std::stable_sort(fitems.begin(), fitems.end(), [H](auto &x, auto &y) {
         const int hx = x.first % H, hy = y.first % H;
         return hx != hy ? hx < hy : x.second > y.second;

@@ -60,7 +60,9 @@ tsp_status tsp_test_next_visible(tsp_plan_t plan, int from, int kv0, int *out);
  *      number of 128-key tiles to visit) for 256-row query blocks
  *   3  dK/dV work order: key tile * heads + head, [S/128 * heads]
  *   4  dQ work order: query tile * heads + head, [S/128 * heads]
- * Work orders are head-major with the longest items of a head first.
+ * Work orders are head-major with the longest items of a head first here;
+ * the plan uploads the forward and dK/dV orders paired in waves
+ * (tsp_test_work_order).
  * TSP_ERR_INVALID_ARG for another `which`, a NULL pointer or a table longer
  * than `capacity`. */
 tsp_status tsp_test_tables(tsp_plan_t plan, int which, int32_t *out, int64_t capacity, int64_t *count);
