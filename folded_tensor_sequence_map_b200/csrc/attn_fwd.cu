@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int w = 0; w < 2; ++w)
                     for (int t = 0; t < C::NATOM; ++t)
                         tma_load_2d(smem + C::OFF_Q + w * C::TILE_BYTES + t * C::ATOM_BYTES, &mapQ, q_full,
-                                    head * DH + t * C::ATOM_COLS, qb * 256 + w * 128);
+                                    head * DH + t * C::ATOM_COLS, qb * 256 + w * 128 - a.q_row0);
                 for (int j = 0; j < nkv; ++j) {
                     const int ks = kcount % C::KST;
                     if (!mbar_wait(&k_empty[ks], ((kcount / C::KST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!warp_wait(&o_done[w], (tcount - 1) & 1, abort_flag, err)) break;
             tc_fence_after();
             const float inv = 1.0f / l;
-            __half *orow = static_cast<__half *>(a.o) + static_cast<int64_t>(lrow) * h + head * DH;
+            __half *orow = static_cast<__half *>(a.o) + static_cast<int64_t>(lrow - a.q_row0) * h + head * DH;
 #pragma unroll 1
             for (int c = 0; c < DH / 32; ++c) {
                 float o[32];
@@ -430,7 +430,7 @@ cudaError_t launch_fwd_impl(const AttnDesc &a, const DevErr &err, int num_sms, c
                                    : C::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                   : CU_TENSOR_MAP_SWIZZLE_32B;
     CUtensorMap mq, mk, mv;
-    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2,
+    bool ok = encode_tensor_map_2d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.q_rows, int64_t(h) * 2,
                                    C::ATOM_COLS, 128, swz);
     ok = ok && encode_tensor_map_2d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2,
                                     C::ATOM_COLS, 128, swz);

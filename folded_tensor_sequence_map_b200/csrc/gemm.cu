@@ -20,7 +20,9 @@
 //
 // Folded-layer specifics live in the tile scheduler and the epilogue:
 //   * ring K order: when ring_rows > 0, the K loop of the rows of rank
-//     r = m0 / ring_rows starts at shard r's first K block and wraps around,
+//     r = ring_rank0 + m0 / ring_rows starts at shard r's first K block and
+//     wraps around (ring_rank0: the rank of row 0, for a GEMM over one
+//     rank's rows),
 //     so the partial sums over FFN shards are added in ring order (r+t) mod D
 //     inside the rank's own accumulator ("Zyphra TSP folds TP+SP onto one GPU
 //     axis", zubnet.ai, paragraph 2: the MLP ring removes the all-reduce);
@@ -40,7 +42,7 @@ constexpr int kGroupM = 16;  // rasterisation: 16 row blocks share each B column
 
 struct GemmArgs {
     int M, N, K;
-    int ring_rows, ring_kblocks;
+    int ring_rows, ring_kblocks, ring_rank0;
     int epi;
     void *out;
     int64_t ldo;
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tile_coords(t, mt, nt, mb, nb);
                 const int m0 = mb * BM, n0 = nb * BN;
                 int kstart = 0;
-                if (p.ring_rows > 0) kstart = ((m0 / p.ring_rows) * p.ring_kblocks) % nk;
+                if (p.ring_rows > 0) kstart = ((m0 / p.ring_rows + p.ring_rank0) * p.ring_kblocks) % nk;
                 for (int i = 0; i < nk; ++i) {
                     int kb = kstart + i;
                     if (kb >= nk) kb -= nk;
@@ -419,6 +421,7 @@ cudaError_t launch_gemm(const GemmDesc &g, const DevErr &err, int num_sms, cudaS
     p.K = g.K;
     p.ring_rows = g.ring_rows;
     p.ring_kblocks = g.ring_kblocks;
+    p.ring_rank0 = g.ring_rank0;
     p.epi = g.epi;
     p.out = g.out;
     p.ldo = g.ldo;

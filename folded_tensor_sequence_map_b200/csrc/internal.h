@@ -45,9 +45,11 @@ struct GemmDesc {
     int64_t ldo2;
     const void *aux;
     int64_t ldaux;
-    // ring K order: rows of rank m / ring_rows start at K block rank * ring_kblocks
+    // ring K order: rows of rank ring_rank0 + m / ring_rows start at K block
+    // rank * ring_kblocks
     int ring_rows;
     int ring_kblocks;
+    int ring_rank0;
     // EPI_QKV only
     const int *rowmap;
     int hsplit;
@@ -129,12 +131,13 @@ cudaError_t launch_convert_f16(const ConvBatch &b, cudaStream_t st);
 // Attention.  Q, K, V, O (and dO, dQ, dK, dV in the backward) are fp16.
 struct AttnDesc {
     int S, L, D, H, dh, chunk;  // tokens, tokens per rank, ranks, heads, head dim, zigzag chunk
-    const void *q;              // fp16 [S][h] rank-major (local) rows
+    const void *q;              // fp16 [q_rows][h]: local rows q_row0 .. q_row0 + q_rows - 1
     const void *k, *v;          // fp16 [S][h] global rows
-    void *o;                    // fp16 [S][h] local rows
+    void *o;                    // fp16 [q_rows][h], rows as q
     float *lse;                 // f32 [H][S] local rows, log2 domain (scores pre-multiplied by log2 e / sqrt(dh))
     const int *order;           // pairs (qblock * H + head, number of 128-key tiles), in paired waves
     int num_items;
+    int q_row0, q_rows;         // the local rows Q and O hold (0 and S for the whole layer)
 };
 cudaError_t launch_attn_fwd(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st);
 

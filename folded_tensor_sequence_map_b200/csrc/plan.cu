@@ -31,6 +31,9 @@ struct tsp_plan_s {
     int num_sms = 0;
     int32_t *d_zig = nullptr, *d_inv = nullptr, *d_qmax = nullptr;
     int32_t *d_fwd_order = nullptr, *d_kv_order = nullptr, *d_q_order = nullptr;
+    // per-rank forward orders (one rank's query blocks, paired in waves), concatenated
+    int32_t *d_rank_fwd_order = nullptr;
+    std::vector<int> rank_fwd_off, rank_fwd_items;
     unsigned int *d_err = nullptr;
     int fwd_items = 0;
     long long wait_limit = 0;
@@ -258,6 +261,28 @@ tsp_status ensure_device(tsp_plan_s *p) {
     if (prop.major != 10) return TSP_ERR_UNSUPPORTED;
     if (!get_encode()) return TSP_ERR_CUDA;
     HostTables t = host_tables(p);
+    // per-rank forward orders: the 256-row query blocks of rank r, taken from
+    // the host order before pairing, then paired in waves by themselves
+    std::vector<int32_t> rank_orders;
+    p->rank_fwd_off.assign(p->D, 0);
+    p->rank_fwd_items.assign(p->D, 0);
+    if (p->L % 256 == 0) {
+        const int64_t blocks = p->L / 256;
+        for (int r = 0; r < p->D; ++r) {
+            std::vector<int32_t> sub;
+            for (size_t i = 0; i + 1 < t.forder.size(); i += 2) {
+                const int64_t qb = t.forder[i] / p->H;
+                if (qb >= r * blocks && qb < (r + 1) * blocks) {
+                    sub.push_back(t.forder[i]);
+                    sub.push_back(t.forder[i + 1]);
+                }
+            }
+            pair_waves(sub, 2, p->H, prop.multiProcessorCount);
+            p->rank_fwd_off[r] = static_cast<int>(rank_orders.size());
+            p->rank_fwd_items[r] = static_cast<int>(sub.size() / 2);
+            rank_orders.insert(rank_orders.end(), sub.begin(), sub.end());
+        }
+    }
     device_orders(t, p->H, prop.multiProcessorCount);
 
     auto upload = [](int32_t **dst, const std::vector<int32_t> &v) {
@@ -267,6 +292,7 @@ tsp_status ensure_device(tsp_plan_s *p) {
     if (!upload(&p->d_zig, p->zig) || !upload(&p->d_inv, t.inv) || !upload(&p->d_qmax, t.qmax) ||
         !upload(&p->d_fwd_order, t.forder) || !upload(&p->d_kv_order, t.korder) || !upload(&p->d_q_order, t.qorder))
         return TSP_ERR_CUDA;
+    if (!rank_orders.empty() && !upload(&p->d_rank_fwd_order, rank_orders)) return TSP_ERR_CUDA;
     if (cudaMalloc(&p->d_err, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
     if (cudaMemset(p->d_err, 0, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
     p->fwd_items = static_cast<int>(t.forder.size() / 2);
@@ -447,6 +473,7 @@ TSP_API void tsp_plan_destroy(tsp_plan_t p) {
         cudaFree(p->d_fwd_order);
         cudaFree(p->d_kv_order);
         cudaFree(p->d_q_order);
+        cudaFree(p->d_rank_fwd_order);
         cudaFree(p->d_err);
         cudaSetDevice(cur);
     }
@@ -567,6 +594,8 @@ tsp_status forward_impl(tsp_plan_s *p, const void *x, const float *g1, const voi
     ad.lse = lse;
     ad.order = p->d_fwd_order;
     ad.num_items = p->fwd_items;
+    ad.q_row0 = 0;
+    ad.q_rows = S;
     TSP_STAGE(2, 1, launch_attn_fwd(ad, err, p->num_sms, s));
     // out-projection (head-group partial sums in broadcast order) + residual, fp32 residual stream
     GemmDesc go = gemm(o, h, false, wo_h, h, false, S, h, h, EPI_RESID_F32, yres, h, scales + kScaleInv + 1);
@@ -944,6 +973,169 @@ TSP_API tsp_status tsp_stack_backward(tsp_plan_t p, int layers, const void *dz, 
     }
     return TSP_OK;
 }
+
+// ===========================================================================
+// One rank's share of the forward, for D devices (tsp.h)
+// ===========================================================================
+
+namespace {
+// Workspace of one rank: its own L rows of every activation, the LSE of all
+// local rows (the kernel indexes it by local row; only this rank's are
+// written), and the fp16 weight copies.
+struct RankLayout {
+    size_t rstd1, a, q, o, lse, y, rstd2, b, u, g, wqkv_h, wo_h, w1_h, w2_h, scales, cpart, total;
+};
+RankLayout rank_layout_of(const tsp_plan_s *p) {
+    RankLayout l{};
+    const size_t L = p->L, S = p->S, h = p->h, F = p->F, H = p->H;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += up(bytes);
+        return o;
+    };
+    l.rstd1 = take(L * 4);
+    l.a = take(L * h * 2);
+    l.q = take(L * h * 2);
+    l.o = take(L * h * 2);
+    l.lse = take(H * S * 4);
+    l.y = take(L * h * 4);
+    l.rstd2 = take(L * 4);
+    l.b = take(L * h * 2);
+    l.u = take(L * F * 2);
+    l.g = take(L * F * 2);
+    l.wqkv_h = take(3 * h * h * 2);
+    l.wo_h = take(h * h * 2);
+    l.w1_h = take(F * h * 2);
+    l.w2_h = take(h * F * 2);
+    l.scales = take(64 * 4);
+    l.cpart = take(static_cast<size_t>(kMaxConv) * kConvBlocks * 4);
+    l.total = off;
+    return l;
+}
+
+tsp_status rank_checks(tsp_plan_s *p, int rank, std::initializer_list<const void *> ptrs) {
+    if (rank < 0 || rank >= p->D) return TSP_ERR_INVALID_ARG;
+    for (const void *q : ptrs)
+        if (!q) return TSP_ERR_INVALID_ARG;
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return TSP_ERR_ALIGNMENT;
+    if (p->L % 256) return TSP_ERR_UNSUPPORTED;  // the forward's query items are 256-row blocks
+    return ensure_device(p);
+}
+}  // namespace
+
+TSP_API tsp_status tsp_rank_workspace_size(tsp_plan_t p, size_t *ws_bytes) {
+    if (!p || !ws_bytes) return TSP_ERR_INVALID_ARG;
+    *ws_bytes = rank_layout_of(p).total;
+    return TSP_OK;
+}
+
+#define TSP_RSTAGE(id, nk, call)                                                 \
+    do {                                                                         \
+        if (stage(p, id, nk, s, [&] { return (call); }) != cudaSuccess)          \
+            return TSP_ERR_CUDA;                                                 \
+    } while (0)
+
+TSP_API tsp_status tsp_rank_forward_qkv(tsp_plan_t p, int rank, const void *x, const float *g1, const void *wqkv,
+                                        void *k, void *v, void *ws, void *stream) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    tsp_status st = rank_checks(p, rank, {x, (const void *)g1, wqkv, (const void *)k, (const void *)v,
+                                          (const void *)ws});
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const RankLayout l = rank_layout_of(p);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const int L = static_cast<int>(p->L), h = p->h;
+    const DevErr err = dev_err(p);
+    auto *scales = reinterpret_cast<float *>(w + l.scales);
+    ConvBatch cb{};
+    cb.t[0] = ConvTensor{wqkv, w + l.wqkv_h, int64_t(3) * h * h, kTargetWeights, scales + kScaleInv + 0,
+                         scales + kScale + 0};
+    cb.count = 1;
+    cb.partial = reinterpret_cast<float *>(w + l.cpart);
+    cb.err = p->d_err;
+    TSP_RSTAGE(20, 2, launch_convert_f16(cb, s));
+    TSP_RSTAGE(0, 1, launch_rmsnorm_fwd(x, nullptr, g1, w + l.a, true, reinterpret_cast<float *>(w + l.rstd1), L, h,
+                                        p->d_err, s));
+    // this rank's rows against every attention shard; K/V land at the rows'
+    // global positions, the rank's part of the all-gather
+    GemmDesc gq = gemm(w + l.a, h, false, w + l.wqkv_h, h, false, L, 3 * h, h, EPI_QKV, w + l.q, h,
+                       scales + kScaleInv + 0);
+    gq.rowmap = p->d_zig + static_cast<int64_t>(rank) * L;
+    gq.hsplit = h;
+    gq.out_k = k;
+    gq.out_v = v;
+    TSP_RSTAGE(1, 1, launch_gemm(gq, err, p->num_sms, s));
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_rank_forward_out(tsp_plan_t p, int rank, const void *x, const void *k, const void *v,
+                                        const void *wo, const float *g2, const void *w1, const void *w2, void *z,
+                                        void *ws, void *stream) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    tsp_status st = rank_checks(p, rank, {x, k, v, wo, (const void *)g2, w1, w2, (const void *)z, (const void *)ws});
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const RankLayout l = rank_layout_of(p);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const int S = static_cast<int>(p->S), L = static_cast<int>(p->L), h = p->h, F = p->F;
+    const DevErr err = dev_err(p);
+    auto *scales = reinterpret_cast<float *>(w + l.scales);
+    ConvBatch cb{};
+    const void *wsrc[3] = {wo, w1, w2};
+    void *wdst[3] = {w + l.wo_h, w + l.w1_h, w + l.w2_h};
+    const int64_t wn[3] = {int64_t(h) * h, int64_t(F) * h, int64_t(h) * F};
+    for (int i = 0; i < 3; ++i)
+        cb.t[i] = ConvTensor{wsrc[i], wdst[i], wn[i], kTargetWeights, scales + kScaleInv + 1 + i,
+                             scales + kScale + 1 + i};
+    cb.count = 3;
+    cb.partial = reinterpret_cast<float *>(w + l.cpart);
+    cb.err = p->d_err;
+    TSP_RSTAGE(20, 2, launch_convert_f16(cb, s));
+    // attention of this rank's queries over the gathered K/V
+    AttnDesc ad{};
+    ad.S = S;
+    ad.L = L;
+    ad.D = p->D;
+    ad.H = p->H;
+    ad.dh = p->dh;
+    ad.chunk = static_cast<int>(p->c);
+    ad.q = w + l.q;
+    ad.k = k;
+    ad.v = v;
+    ad.o = w + l.o;
+    ad.lse = reinterpret_cast<float *>(w + l.lse);
+    ad.order = p->d_rank_fwd_order + p->rank_fwd_off[rank];
+    ad.num_items = p->rank_fwd_items[rank];
+    ad.q_row0 = rank * L;
+    ad.q_rows = L;
+    TSP_RSTAGE(2, 1, launch_attn_fwd(ad, err, p->num_sms, s));
+    auto *yres = reinterpret_cast<float *>(w + l.y);
+    GemmDesc go = gemm(w + l.o, h, false, w + l.wo_h, h, false, L, h, h, EPI_RESID_F32, yres, h,
+                       scales + kScaleInv + 1);
+    go.aux = x;
+    go.ldaux = h;
+    TSP_RSTAGE(3, 1, launch_gemm(go, err, p->num_sms, s));
+    TSP_RSTAGE(4, 1, launch_rmsnorm_fwd(nullptr, yres, g2, w + l.b, true, reinterpret_cast<float *>(w + l.rstd2), L,
+                                        h, p->d_err, s));
+    GemmDesc g1d = gemm(w + l.b, h, false, w + l.w1_h, h, false, L, F, h, EPI_GELU, w + l.u, F,
+                        scales + kScaleInv + 2);
+    g1d.out2 = w + l.g;
+    g1d.ldo2 = F;
+    TSP_RSTAGE(5, 1, launch_gemm(g1d, err, p->num_sms, s));
+    // W2 with the K loop over FFN shards in this rank's ring order (rank + t) mod D
+    GemmDesc g2d = gemm(w + l.g, F, false, w + l.w2_h, F, false, L, h, F, EPI_RESID_BF16, z, h,
+                        scales + kScaleInv + 3);
+    g2d.aux = yres;
+    g2d.ldaux = h;
+    g2d.ring_rows = L;
+    g2d.ring_kblocks = (F / p->D) / 64;
+    g2d.ring_rank0 = rank;
+    TSP_RSTAGE(6, 1, launch_gemm(g2d, err, p->num_sms, s));
+    return TSP_OK;
+}
+#undef TSP_RSTAGE
 
 TSP_API tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A, int64_t lda, const void *B,
                                  int64_t ldb, float *C, int64_t ldc, int force_bn128, int f16, void *stream) {

@@ -43,6 +43,9 @@ EXPORTED = (
     "tsp_stack_workspace_size",
     "tsp_stack_forward",
     "tsp_stack_backward",
+    "tsp_rank_workspace_size",
+    "tsp_rank_forward_qkv",
+    "tsp_rank_forward_out",
     "tsp_sync_status",
     "tsp_status_string",
     "tsp_layer_flops",
@@ -99,6 +102,12 @@ def _load() -> ctypes.CDLL:
     lib.tsp_stack_forward.restype = I
     lib.tsp_stack_backward.argtypes = [P, I] + [V] * 19
     lib.tsp_stack_backward.restype = I
+    lib.tsp_rank_workspace_size.argtypes = [P, ctypes.POINTER(SZ)]
+    lib.tsp_rank_workspace_size.restype = I
+    lib.tsp_rank_forward_qkv.argtypes = [P, I] + [V] * 7
+    lib.tsp_rank_forward_qkv.restype = I
+    lib.tsp_rank_forward_out.argtypes = [P, I] + [V] * 10
+    lib.tsp_rank_forward_out.restype = I
     lib.tsp_sync_status.argtypes = [P, V]
     lib.tsp_sync_status.restype = I
     lib.tsp_status_string.argtypes = [I]
@@ -363,6 +372,35 @@ def tsp_stack_backward(plan: Plan, dz, x, g1, wqkv, wo, g2, w1, w2, inputs, save
                                    *[ctypes.cast(a, ctypes.c_void_p) for a in arrs], _ptr(inputs, "inputs"), _ptr(saved, "saved"),
                                    _ptr(ws, "ws"), _ptr(dx, "dx", bf, (S, h)), *[ctypes.cast(a, ctypes.c_void_p) for a in grads],
                                    _stream(stream)), "tsp_stack_backward")
+
+
+def tsp_rank_workspace_size(plan: Plan) -> int:
+    ws = ctypes.c_size_t()
+    _check(_lib.tsp_rank_workspace_size(plan.handle, ctypes.byref(ws)), "tsp_rank_workspace_size")
+    return ws.value
+
+
+def tsp_rank_forward_qkv(plan: Plan, rank: int, x, g1, wqkv, k, v, ws, stream=None) -> None:
+    import torch
+
+    h, S, L = plan.h, plan.S, plan.S // plan.D
+    bf, f32, f16 = torch.bfloat16, torch.float32, torch.float16
+    _check(_lib.tsp_rank_forward_qkv(plan.handle, rank, _ptr(x, "x", bf, (L, h)), _ptr(g1, "g1", f32, (h,)),
+                                     _ptr(wqkv, "wqkv", bf, (3 * h, h)), _ptr(k, "k", f16, (S, h)),
+                                     _ptr(v, "v", f16, (S, h)), _ptr(ws, "ws"), _stream(stream)),
+           "tsp_rank_forward_qkv")
+
+
+def tsp_rank_forward_out(plan: Plan, rank: int, x, k, v, wo, g2, w1, w2, z, ws, stream=None) -> None:
+    import torch
+
+    h, F, S, L = plan.h, plan.ffn, plan.S, plan.S // plan.D
+    bf, f32, f16 = torch.bfloat16, torch.float32, torch.float16
+    _check(_lib.tsp_rank_forward_out(plan.handle, rank, _ptr(x, "x", bf, (L, h)), _ptr(k, "k", f16, (S, h)),
+                                     _ptr(v, "v", f16, (S, h)), _ptr(wo, "wo", bf, (h, h)), _ptr(g2, "g2", f32, (h,)),
+                                     _ptr(w1, "w1", bf, (F, h)), _ptr(w2, "w2", bf, (h, F)),
+                                     _ptr(z, "z", bf, (L, h)), _ptr(ws, "ws"), _stream(stream)),
+           "tsp_rank_forward_out")
 
 
 def tsp_sync_status(plan: Plan, stream=None) -> None:

@@ -243,6 +243,46 @@ tsp_status tsp_stack_backward(tsp_plan_t plan, int layers, const void *dz, const
                               void *ws, void *dx, float *const *dg1, float *const *dwqkv, float *const *dwo,
                               float *const *dg2, float *const *dw1, float *const *dw2, void *stream);
 
+/* One rank's share of the forward, for running the folded layer on D
+ * devices, one virtual rank each ("Zyphra TSP folds TP+SP onto one GPU axis,
+ * 2.6x throughput on 1,024 MI300Xs", zubnet.ai, paragraphs 1-2).  Rank r
+ * holds its L = S/D tokens (rows [r*L, (r+1)*L) of the rank-major layout)
+ * and runs two calls, with the K/V all-gather between them:
+ *
+ * tsp_rank_workspace_size: bytes of one rank's workspace (its rows of every
+ * intermediate, the LSE of all S local rows, the fp16 weight copies).
+ *
+ * tsp_rank_forward_qkv: RMSNorm1 of the rank's tokens x (bf16 [L][h]) and
+ * their projection onto every attention shard (the whole Wqkv, bf16 [3h][h]:
+ * the shards the broadcast schedule delivers, all present on the device).  Q
+ * stays in ws; K and V are written into k, v (fp16 [S][h], global position
+ * order) at the positions of the rank's own tokens only: the rank's
+ * contribution to the all-gather.
+ *
+ * Between the calls the caller all-gathers K and V so that every rank's k, v
+ * hold all S rows.  Rank j's rows are the positions of its two zigzag chunks,
+ * [j*c, (j+1)*c) and [(2D-1-j)*c, (2D-j)*c), c = S/(2D): two all-gathers of
+ * c-row blocks per tensor put every block in place.
+ *
+ * tsp_rank_forward_out: causal attention of the rank's queries over all S
+ * keys, the out-projection + residual, RMSNorm2, W1 with GELU, and W2 with its
+ * K loop over the FFN shards in the rank's ring order (rank + t) mod D (the
+ * shards the ring delivers, all present: wo, w1, w2 whole) + residual, into z
+ * (bf16 [L][h]).  x is the same rank's tokens as in the first call.
+ *
+ * The same kernels as tsp_layer_forward on the rank's rows, so the D ranks'
+ * z rows are bit for bit the layer's.  Errors: TSP_ERR_INVALID_ARG for a rank
+ * outside [0, D) or a NULL pointer, TSP_ERR_ALIGNMENT unless every pointer is
+ * 16-byte aligned, TSP_ERR_UNSUPPORTED when L is not a multiple of 256 (the
+ * attention's query items are 256-row blocks) or off sm_100, TSP_ERR_CUDA for
+ * a failed launch; argument errors are found before anything is enqueued. */
+tsp_status tsp_rank_workspace_size(tsp_plan_t plan, size_t *ws_bytes);
+tsp_status tsp_rank_forward_qkv(tsp_plan_t plan, int rank, const void *x, const float *g1, const void *wqkv,
+                                void *k, void *v, void *ws, void *stream);
+tsp_status tsp_rank_forward_out(tsp_plan_t plan, int rank, const void *x, const void *k, const void *v,
+                                const void *wo, const float *g2, const void *w1, const void *w2, void *z, void *ws,
+                                void *stream);
+
 /* Wait for `stream`, then report TSP_ERR_CUDA for an asynchronous CUDA error,
  * TSP_ERR_TIMEOUT if a device-side wait of this plan ran out, or TSP_ERR_RANGE
  * if a value overflowed an fp16 intermediate (the flags are cleared by the

@@ -251,6 +251,30 @@ def test_stack_checks_arguments_before_enqueueing():
     assert st(bwd(3, six, grads, dx=0x70008)) == "TSP_ERR_ALIGNMENT"
 
 
+def test_rank_forward_checks_arguments_before_enqueueing():
+    """tsp_rank_forward_qkv / _out refuse a rank outside [0, D), a NULL or a
+    misaligned pointer, and a rank size L that is not a multiple of 256 (the
+    attention's query blocks), before anything runs."""
+    p = T.tsp_plan(128, 4, 512, 1024, 2)
+    V = ctypes.c_void_p
+    lib = TT._lib
+    st = lambda rc: T.STATUS_NAMES[rc]
+    good = [V(0x10000 * (i + 1)) for i in range(9)]
+    qkv = lambda rank, args: st(lib.tsp_rank_forward_qkv(p.handle, rank, *args[:6], V(0)))
+    out = lambda rank, args: st(lib.tsp_rank_forward_out(p.handle, rank, *args[:9], V(0)))
+    assert qkv(2, good) == "TSP_ERR_INVALID_ARG" and qkv(-1, good) == "TSP_ERR_INVALID_ARG"
+    assert out(2, good) == "TSP_ERR_INVALID_ARG"
+    bad = list(good)
+    bad[3] = V(0)
+    assert qkv(0, bad) == "TSP_ERR_INVALID_ARG" and out(0, bad) == "TSP_ERR_INVALID_ARG"
+    bad = list(good)
+    bad[2] = V(0x30008)
+    assert qkv(1, bad) == "TSP_ERR_ALIGNMENT" and out(1, bad) == "TSP_ERR_ALIGNMENT"
+    small = T.tsp_plan(128, 4, 512, 256, 2)  # L = 128
+    assert st(lib.tsp_rank_forward_qkv(small.handle, 0, *good[:6], V(0))) == "TSP_ERR_UNSUPPORTED"
+    assert T.tsp_rank_workspace_size(p) > 0
+
+
 def test_prefill_checks_arguments_before_enqueueing():
     """tsp_layer_prefill refuses a NULL or misaligned pointer before it touches
     the device (the addresses below are never dereferenced)."""
