@@ -93,10 +93,11 @@ def stage_flops(s: LayerShape) -> dict:
 
 
 def inactive_stages(s: LayerShape) -> set:
-    """Stages that the library does not run for this shape: head size 128
+    """Stages that the layer does not run for this shape: head size 128
     takes the single-pass attention backward, other head sizes the two
-    kernels."""
-    return {"bwd_attn_dkdv", "bwd_attn_dq"} if s.dh == 128 else {"bwd_attn_fused", "bwd_attn_dq_convert"}
+    kernels; the dK/dV conversion belongs to the per-rank backward only."""
+    attn = {"bwd_attn_dkdv", "bwd_attn_dq"} if s.dh == 128 else {"bwd_attn_fused", "bwd_attn_dq_convert"}
+    return attn | {"bwd_convert_dkdv"}
 
 
 def hbm_stage_bytes(s: LayerShape) -> dict:
@@ -117,6 +118,7 @@ def hbm_stage_bytes(s: LayerShape) -> dict:
         # bound and clears the 32-bit dQ sum
         "bwd_attn_delta": S * h * (2 + 2) + S * H * 4 + (S * h * (2 + 2 + 4) if s.dh == 128 else 0),
         "bwd_attn_dq_convert": S * h * (4 + 2),                           # dQ sum f32 -> dQ fp16
+        "bwd_convert_dkdv": 2 * S / s.D * h * (4 + 2),                    # one rank's dK, dV f32 -> fp16
     }
 
 

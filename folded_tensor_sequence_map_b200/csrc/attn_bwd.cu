@@ -105,7 +105,9 @@ CUtensorMapSwizzle swz_of() {
 // |dO_row|^2, |V_row|^2 and |K|_max that bound the sum (dq_frac_bits): per
 // block in shared memory, then one atomicMax per head and block into `bound`
 // (cleared before the launch; non-negative float bits order like unsigned
-// integers, so the maxima do not depend on the order).
+// integers, so the maxima do not depend on the order).  The O / dO rows
+// (q_rows of them, local rows from q_row0) and the K / V rows (all S, read
+// only for the bounds) are separate ranges of the same loop.
 __device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b) {
     return f16_lo(a.x) * f16_lo(b.x) + f16_hi(a.x) * f16_hi(b.x) + f16_lo(a.y) * f16_lo(b.y) +
            f16_hi(a.y) * f16_hi(b.y) + f16_lo(a.z) * f16_lo(b.z) + f16_hi(a.z) * f16_hi(b.z) +
@@ -119,7 +121,8 @@ __device__ __forceinline__ float absmax8(const uint4 &a) {
 }
 
 __global__ void attn_delta_kernel(const __half *o, const __half *dout, const __half *kk, const __half *vv,
-                                  float *delta, int *acc, unsigned int *bound, int S, int H, int dh) {
+                                  float *delta, int *acc, unsigned int *bound, int S, int H, int dh, int q_row0,
+                                  int q_rows, int kv_rows) {
     extern __shared__ unsigned int smax[];  // [H][3]
     const bool fused = acc != nullptr;
     if (fused) {
@@ -134,28 +137,31 @@ __global__ void attn_delta_kernel(const __half *o, const __half *dout, const __h
     const int col = (lane % lph) * 8;
     const int64_t h = static_cast<int64_t>(H) * dh;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    // rows [0, q_rows) of O and dO (local rows q_row0 + row), rows [0, kv_rows) of K and V
+    const int64_t nrows = q_rows > kv_rows ? q_rows : kv_rows;
     for (int64_t wi = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-         wi < static_cast<int64_t>(S) * groups; wi += nwarps) {
+         wi < nrows * groups; wi += nwarps) {
         const int64_t row = wi / groups;
         const int head = static_cast<int>(wi - row * groups) * hpw + head_in;
         const bool on = head < H;
+        const bool qrow = on && row < q_rows;
         const int64_t at = row * h + static_cast<int64_t>(head) * dh + col;
         float s = 0.f, n2 = 0.f, v2 = 0.f, km = 0.f;
-        if (on) {
+        if (qrow) {
             const uint4 a = *reinterpret_cast<const uint4 *>(o + at);
             const uint4 b = *reinterpret_cast<const uint4 *>(dout + at);
             s = dot8(a, b);
-            if (fused) {
-                const uint4 kw = *reinterpret_cast<const uint4 *>(kk + at);
-                const uint4 vw = *reinterpret_cast<const uint4 *>(vv + at);
-                n2 = dot8(b, b);
-                v2 = dot8(vw, vw);
-                km = absmax8(kw);
-            }
+            if (fused) n2 = dot8(b, b);
+        }
+        if (fused && on && row < kv_rows) {
+            const uint4 kw = *reinterpret_cast<const uint4 *>(kk + at);
+            const uint4 vw = *reinterpret_cast<const uint4 *>(vv + at);
+            v2 = dot8(vw, vw);
+            km = absmax8(kw);
         }
         for (int off = lph / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         const bool first = on && col == 0;
-        if (first) delta[static_cast<int64_t>(head) * S + row] = s;
+        if (first && row < q_rows) delta[static_cast<int64_t>(head) * S + q_row0 + row] = s;
         if (fused) {
             for (int off = lph / 2; off > 0; off >>= 1) {
                 n2 += __shfl_xor_sync(0xffffffffu, n2, off);
@@ -167,7 +173,7 @@ __global__ void attn_delta_kernel(const __half *o, const __half *dout, const __h
                 atomicMax(&smax[3 * head + 1], __float_as_uint(v2));
                 atomicMax(&smax[3 * head + 2], __float_as_uint(km));
             }
-            if (on) {
+            if (qrow) {
                 int4 *z = reinterpret_cast<int4 *>(acc + at);
                 z[0] = make_int4(0, 0, 0, 0);
                 z[1] = make_int4(0, 0, 0, 0);
@@ -858,7 +864,9 @@ struct FusedParams {
     int num_items;
 };
 
-template <int DH>
+// PART: one rank's share (AttnBwdDesc::rank >= 0), a separate instance so
+// that the whole-layer instance carries none of its code.
+template <int DH, bool PART>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                           const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdO,
@@ -886,7 +894,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nq64 = a.S / 64;
-    const StepVis vis{a.D, a.chunk, nq64};
+    const StepVis vis{a.D, a.chunk, nq64, PART ? a.rank : -1};
+    const int q_row0 = PART ? a.q_row0 : 0;
     const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
     const float scale = rsqrtf(static_cast<float>(DH));
     constexpr int kDrainWarp = 2 + 4 * kEwGroups;
@@ -942,9 +951,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     mbar_arrive_tx(&q_full[s], 2 * F::QTILE + F::VEC_BYTES);
                     for (int t = 0; t < C::NATOM; ++t) {
                         tma_load_2d(smem + F::OFF_Q + s * F::QTILE + t * F::QATOM, &mQ, &q_full[s],
-                                    head * DH + t * C::ATOM_COLS, q * 64);
+                                    head * DH + t * C::ATOM_COLS, q * 64 - q_row0);
                         tma_load_2d(smem + F::OFF_DO + s * F::QTILE + t * F::QATOM, &mdO, &q_full[s],
-                                    head * DH + t * C::ATOM_COLS, q * 64);
+                                    head * DH + t * C::ATOM_COLS, q * 64 - q_row0);
                     }
                     float *vec = reinterpret_cast<float *>(smem + F::OFF_VEC + s * F::VEC_BYTES);
                     bulk_load(vec, a.lse + static_cast<int64_t>(head) * a.S + q * 64, 256, &q_full[s]);
@@ -1180,12 +1189,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             tc_fence_after();
             // groups 0, 1 write dV (offset removed) and groups 2, 3 write dK
             // (scaled), at the key owner's local row; each pair splits the
-            // 32-column chunks
+            // 32-column chunks.  One rank's share goes out as fp32 partial
+            // sums, also times *dkv_mul.
             const int lrow = a.inv_map[key];
             const int which = grp >> 1;
+            const float f = (which == 0 ? kPOffInv : scale) * (PART ? *a.dkv_mul : 1.0f);
             void *dstp = which == 0 ? a.dv : a.dk;
-            const float f = which == 0 ? kPOffInv : scale;
-            __half *orow = static_cast<__half *>(dstp) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+            __half *orow = PART ? nullptr : static_cast<__half *>(dstp) + static_cast<int64_t>(lrow) * a.ldd + head * DH;
+            float *frow = PART ? (which == 0 ? a.dv_part : a.dk_part) + static_cast<int64_t>(lrow) * (a.H * DH) + head * DH
+                               : nullptr;
             if (!warp_converged("dV/dK TMEM load")) break;
 #pragma unroll 1
             for (int c = grp & 1; c < DH / 32; c += 2) {
@@ -1194,6 +1206,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] *= f;
+                if (PART) {
+                    float4 *d4 = reinterpret_cast<float4 *>(frow + c * 32);
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq)
+                        d4[qq] = make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]);
+                    continue;
+                }
                 flag_range(maxabs32(v), a.err);
                 uint4 *d4 = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
@@ -1237,7 +1256,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 if (lane == 0) mbar_arrive(&buf_free[b]);
                 // one global reduction per element: a warp's 32 head dims of one
                 // query row are one 128-byte line
-                int *col = a.dq_acc + static_cast<int64_t>(w.q) * 64 * hh + head * DH + d;
+                int *col = a.dq_acc + (static_cast<int64_t>(w.q) * 64 - q_row0) * hh + head * DH + d;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) atomicAdd(col + j * hh, __float2int_rn(v[j] * dq_scale));
             }
@@ -1276,10 +1295,10 @@ struct BwdMaps {
         using C = BCfg<DH>;
         const int h = a.H * DH;
         const auto swz = swz_of<DH>();
-        bool ok = encode_tensor_map_2d(&q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        bool ok = encode_tensor_map_2d(&q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.q_rows, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
         ok = ok && encode_tensor_map_2d(&k, a.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
         ok = ok && encode_tensor_map_2d(&v, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
-        ok = ok && encode_tensor_map_2d(&dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
+        ok = ok && encode_tensor_map_2d(&dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.q_rows, int64_t(h) * 2, C::ATOM_COLS, 128, swz);
         return ok;
     }
 };
@@ -1347,16 +1366,17 @@ cudaError_t launch_fused_impl(const AttnBwdDesc &a, const DevErr &err, int num_s
     // Q and dO sub-tiles of 64 rows
     const int h = a.H * DH;
     const auto swz = swz_of<DH>();
-    bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
-    ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.S, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    bool ok = encode_tensor_map_2d(&m.q, a.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.q_rows, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
+    ok = ok && encode_tensor_map_2d(&m.dout, a.dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h, a.q_rows, int64_t(h) * 2, C::ATOM_COLS, 64, swz);
     if (!ok) return cudaErrorInvalidValue;
     FusedParams fp;
     fp.d = a;
     fp.zig = zig;
-    fp.num_items = (a.S / 128) * a.H;
+    fp.num_items = a.rank < 0 ? (a.S / 128) * a.H : a.kv_items;
+    if (fp.num_items <= 0) return cudaSuccess;
     // at most one CTA per SM, so every CTA is resident (the dQ order waits need it)
     const int grid = fp.num_items < num_sms ? fp.num_items : num_sms;
-    auto k = attn_bwd_fused_kernel<DH>;
+    auto k = a.rank < 0 ? attn_bwd_fused_kernel<DH, false> : attn_bwd_fused_kernel<DH, true>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<DH>::SMEM);
     if (e != cudaSuccess) return e;
     k<<<grid, kFusedThreads, FusedCfg<DH>::SMEM, st>>>(m.q, m.k, m.v, m.dout, fp, err);
@@ -1370,16 +1390,25 @@ bool attn_bwd_fused_supported(int dh) { return dh == 128; }
 cudaError_t launch_attn_bwd_fused(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st,
                                   const int *zig) {
     if (a.dh != 128 || !a.dq_acc || !a.dq_bound) return cudaErrorInvalidValue;
+    if (a.q_row0 < 0 || a.q_row0 % 64 || a.q_rows % 64 || a.q_row0 + a.q_rows > a.S) return cudaErrorInvalidValue;
+    if (a.rank >= 0) {
+        const size_t bytes = static_cast<size_t>(a.S) * a.H * a.dh * sizeof(float);
+        if (a.rank >= a.D || !a.dk_part || !a.dv_part || !a.dkv_mul) return cudaErrorInvalidValue;
+        cudaError_t e = cudaMemsetAsync(a.dk_part, 0, bytes, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a.dv_part, 0, bytes, st);
+        if (e != cudaSuccess) return e;
+    }
     return launch_fused_impl<128>(a, err, num_sms, st, zig);
 }
 
 cudaError_t launch_dq_convert(const AttnBwdDesc &a, cudaStream_t st) {
     const int h = a.H * a.dh;
-    const int64_t n8 = static_cast<int64_t>(a.S) * h / 8;
+    const int64_t n8 = static_cast<int64_t>(a.q_rows) * h / 8;
+    if (n8 == 0) return cudaSuccess;
     const int threads = 256;
     const int64_t blocks = (n8 + threads - 1) / threads;
     dq_convert_kernel<<<static_cast<unsigned int>(blocks), threads, 0, st>>>(
-        a.dq_acc, a.dq_bound, static_cast<__half *>(a.dq), a.ldd, a.S, h, a.dh, a.err);
+        a.dq_acc, a.dq_bound, static_cast<__half *>(a.dq), a.ldd, a.q_rows, h, a.dh, a.err);
     return cudaGetLastError();
 }
 
@@ -1389,17 +1418,23 @@ cudaError_t launch_attn_delta(const AttnBwdDesc &a, int num_sms, cudaStream_t st
         if (e != cudaSuccess) return e;
     }
     if (a.dh % 8 || a.dh < 8 || a.dh > 256 || 32 % (a.dh / 8)) return cudaErrorInvalidValue;
+    if (a.q_row0 < 0 || a.q_rows < 0 || a.q_row0 + a.q_rows > a.S) return cudaErrorInvalidValue;
+    // without the fused kernel's sums only the O / dO rows are read
+    const int64_t rows = a.dq_acc ? (a.q_rows > a.S ? a.q_rows : a.S) : a.q_rows;
+    if (rows == 0) return cudaSuccess;
     const int hpw = 256 / a.dh;
-    const int64_t warps = static_cast<int64_t>(a.S) * ((a.H + hpw - 1) / hpw);
+    const int64_t warps = rows * ((a.H + hpw - 1) / hpw);
     const int64_t want = (warps * 32 + 255) / 256;
     const int blocks = static_cast<int>(want < 8LL * num_sms ? want : 8LL * num_sms);
     attn_delta_kernel<<<blocks, 256, static_cast<size_t>(3) * a.H * sizeof(unsigned int), st>>>(
         static_cast<const __half *>(a.o), static_cast<const __half *>(a.dout), static_cast<const __half *>(a.k),
-        static_cast<const __half *>(a.v), a.delta, a.dq_acc, a.dq_bound, a.S, a.H, a.dh);
+        static_cast<const __half *>(a.v), a.delta, a.dq_acc, a.dq_bound, a.S, a.H, a.dh, a.q_row0, a.q_rows,
+        a.dq_acc ? a.S : 0);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig) {
+    if (a.rank >= 0 || a.q_row0 != 0 || a.q_rows != a.S) return cudaErrorInvalidValue;
     switch (a.dh) {
         case 32: return launch_dkdv_impl<32>(a, err, num_sms, st, zig);
         case 64: return launch_dkdv_impl<64>(a, err, num_sms, st, zig);
@@ -1410,6 +1445,7 @@ cudaError_t launch_attn_dkdv(const AttnBwdDesc &a, const DevErr &err, int num_sm
 
 cudaError_t launch_attn_dq(const AttnBwdDesc &a, const DevErr &err, int num_sms, cudaStream_t st, const int *zig,
                            const int *qtile_maxpos) {
+    if (a.rank >= 0 || a.q_row0 != 0 || a.q_rows != a.S) return cudaErrorInvalidValue;
     switch (a.dh) {
         case 32: return launch_dq_impl<32>(a, err, num_sms, st, zig, qtile_maxpos);
         case 64: return launch_dq_impl<64>(a, err, num_sms, st, zig, qtile_maxpos);

@@ -91,7 +91,39 @@ __global__ void __launch_bounds__(kThreads) convert_kernel(const ConvBatch b) {
     }
 }
 
+// fp32 rows of `cols` values -> fp16 times *mul into rows of stride ldd,
+// 8 elements per thread; values past fp16's range set the range error bit.
+__global__ void __launch_bounds__(kThreads) scale_to_f16_kernel(const float *src, int64_t n8, int cols, __half *dst,
+                                                                int64_t ldd, const float *mul, unsigned int *err) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    if (i >= n8) return;
+    const int64_t e = i * 8;
+    const int64_t row = e / cols;
+    const int col = static_cast<int>(e - row * cols);
+    const float m = *mul;
+    const float4 a = *reinterpret_cast<const float4 *>(src + e);
+    const float4 b = *reinterpret_cast<const float4 *>(src + e + 4);
+    const float v[8] = {a.x * m, a.y * m, a.z * m, a.w * m, b.x * m, b.y * m, b.z * m, b.w * m};
+    float mx = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(v[j]));
+    flag_range(mx, err);
+    *reinterpret_cast<uint4 *>(dst + row * ldd + col) =
+        make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]), pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
+}
+
 }  // namespace
+
+cudaError_t launch_scale_to_f16(const float *src, int64_t rows, int cols, void *dst, int64_t ldd, const float *mul,
+                                unsigned int *err, cudaStream_t st) {
+    if (cols % 8 || ldd % 8 || (reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(dst) & 15u))
+        return cudaErrorInvalidValue;
+    const int64_t n8 = rows * cols / 8;
+    if (n8 == 0) return cudaSuccess;
+    scale_to_f16_kernel<<<static_cast<unsigned int>((n8 + kThreads - 1) / kThreads), kThreads, 0, st>>>(
+        src, n8, cols, static_cast<__half *>(dst), ldd, mul, err);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_convert_f16(const ConvBatch &b, cudaStream_t st) {
     if (b.count <= 0 || b.count > kMaxConv) return cudaErrorInvalidValue;

@@ -127,6 +127,10 @@ struct ConvBatch {
     unsigned int *err;
 };
 cudaError_t launch_convert_f16(const ConvBatch &b, cudaStream_t st);
+// fp32 [rows][cols] -> fp16 times *mul (device scalar) into rows of stride
+// ldd elements (cols, ldd multiples of 8; both pointers 16-byte aligned).
+cudaError_t launch_scale_to_f16(const float *src, int64_t rows, int cols, void *dst, int64_t ldd, const float *mul,
+                                unsigned int *err, cudaStream_t st);
 
 // Attention.  Q, K, V, O (and dO, dQ, dK, dV in the backward) are fp16.
 struct AttnDesc {
@@ -165,6 +169,7 @@ __host__ __device__ inline int zz_next_visible(int from, int kv0, int D, int chu
 // Visibility of 64-row query steps to a key tile, from the zigzag layout.
 struct StepVis {
     int D, chunk, nq64;
+    int rank = -1;  // >= 0: only the steps of rank `rank` (chunks rank and 2D-1-rank); DescWalk only
 };
 
 // Walks the query steps that can see a key tile kv0, in ascending order.
@@ -213,7 +218,7 @@ struct DescWalk {
         q = lc * spc + t;
     }
     __host__ __device__ inline void seek(const StepVis &v, int kv0) {
-        pc = 2 * v.D - 1;
+        pc = 2 * v.D - 1 - (v.rank < 0 ? 0 : v.rank);
         enter(v, kv0);
     }
     __host__ __device__ inline void next(const StepVis &v, int kv0) {
@@ -221,7 +226,7 @@ struct DescWalk {
             --t;
             --q;
         } else {
-            --pc;
+            pc = v.rank < 0 ? pc - 1 : (pc == 2 * v.D - 1 - v.rank ? v.rank : -1);
             enter(v, kv0);
         }
     }
@@ -242,6 +247,19 @@ struct AttnBwdDesc {
     int *dq_acc;                       // [S][h] scratch: dQ summed over key tiles in 32-bit fixed point
                                        // (single-pass kernel; zeroed by the Delta kernel), or null
     unsigned int *dq_bound;            // [H][3] scratch: per-head maxima bounding that sum (Delta kernel)
+    // Query-row window: q, o, dout, dq and dq_acc hold the q_rows local rows
+    // starting at local row q_row0 (the whole layer: 0 and S).  lse and delta
+    // stay [H][S], indexed by local row.
+    int q_row0, q_rows;
+    // One rank's share (single-pass kernel only): rank >= 0 walks only the
+    // query steps of that rank's rows, kv_order holds only the key tiles
+    // those rows see, and dK / dV go out as fp32 partial sums times *dkv_mul
+    // into dk_part / dv_part ([S][h], local rows of the key's owner, zeroed
+    // by the launcher) instead of dk / dv.
+    int rank;
+    int kv_items;                      // entries of kv_order
+    float *dk_part, *dv_part;
+    const float *dkv_mul;
 };
 // Delta = rowsum(dO * O) per head; then dK/dV (key-tile items, 64-row query
 // steps, visibility from zz_next_visible) and dQ (query-tile items).  zig:

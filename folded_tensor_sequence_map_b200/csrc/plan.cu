@@ -34,6 +34,9 @@ struct tsp_plan_s {
     // per-rank forward orders (one rank's query blocks, paired in waves), concatenated
     int32_t *d_rank_fwd_order = nullptr;
     std::vector<int> rank_fwd_off, rank_fwd_items;
+    // per-rank backward orders (the key tiles one rank's rows see, paired in waves), concatenated
+    int32_t *d_rank_bwd_order = nullptr;
+    std::vector<int> rank_bwd_off, rank_bwd_items;
     unsigned int *d_err = nullptr;
     int fwd_items = 0;
     long long wait_limit = 0;
@@ -249,6 +252,19 @@ void device_orders(HostTables &t, int H, int G) {
     pair_waves(t.korder, 1, H, G);
 }
 
+// The backward work order of rank r for G SMs: the key tiles that its rows
+// see (its highest chunk, 2D-1-r, ends at position (2D-r) c - 1), taken from
+// the host order before pairing (a head's tiles in ascending order there, so
+// also longest first for one rank's rows), then paired in waves.
+std::vector<int32_t> rank_kv_order(const tsp_plan_s *p, const HostTables &t, int r, int G) {
+    const int64_t last = (2 * p->D - r) * p->c - 1;
+    std::vector<int32_t> sub;
+    for (int32_t it : t.korder)
+        if (static_cast<int64_t>(it / p->H) * 128 <= last) sub.push_back(it);
+    pair_waves(sub, 1, p->H, G);
+    return sub;
+}
+
 // Device tables: map, inverse map, per-query-tile max position and the work
 // orders of the attention kernels (paired in waves, pair_waves).
 tsp_status ensure_device(tsp_plan_s *p) {
@@ -283,6 +299,16 @@ tsp_status ensure_device(tsp_plan_s *p) {
             rank_orders.insert(rank_orders.end(), sub.begin(), sub.end());
         }
     }
+    // per-rank backward orders (rank_kv_order)
+    std::vector<int32_t> rank_korders;
+    p->rank_bwd_off.assign(p->D, 0);
+    p->rank_bwd_items.assign(p->D, 0);
+    for (int r = 0; r < p->D; ++r) {
+        const std::vector<int32_t> sub = rank_kv_order(p, t, r, prop.multiProcessorCount);
+        p->rank_bwd_off[r] = static_cast<int>(rank_korders.size());
+        p->rank_bwd_items[r] = static_cast<int>(sub.size());
+        rank_korders.insert(rank_korders.end(), sub.begin(), sub.end());
+    }
     device_orders(t, p->H, prop.multiProcessorCount);
 
     auto upload = [](int32_t **dst, const std::vector<int32_t> &v) {
@@ -293,6 +319,7 @@ tsp_status ensure_device(tsp_plan_s *p) {
         !upload(&p->d_fwd_order, t.forder) || !upload(&p->d_kv_order, t.korder) || !upload(&p->d_q_order, t.qorder))
         return TSP_ERR_CUDA;
     if (!rank_orders.empty() && !upload(&p->d_rank_fwd_order, rank_orders)) return TSP_ERR_CUDA;
+    if (!upload(&p->d_rank_bwd_order, rank_korders)) return TSP_ERR_CUDA;
     if (cudaMalloc(&p->d_err, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
     if (cudaMemset(p->d_err, 0, sizeof(unsigned int)) != cudaSuccess) return TSP_ERR_CUDA;
     p->fwd_items = static_cast<int>(t.forder.size() / 2);
@@ -387,7 +414,7 @@ const char *kStageNames[TSP_NUM_STAGES] = {
     "fwd_w2_ring_gemm", "bwd_dgelu_gemm", "bwd_dw2_gemm", "bwd_dw1_gemm", "bwd_db_ring_gemm", "bwd_rmsnorm2",
     "bwd_do_gemm", "bwd_dwo_gemm", "bwd_attn_delta", "bwd_attn_dkdv", "bwd_attn_dq", "bwd_dwqkv_gemm",
     "bwd_da_gemm", "bwd_rmsnorm1", "fwd_convert_weights", "bwd_convert_dy", "bwd_attn_fused",
-    "bwd_attn_dq_convert"};
+    "bwd_attn_dq_convert", "bwd_convert_dkdv"};
 
 GemmDesc gemm(const void *A, int64_t lda, bool a_mn, const void *B, int64_t ldb, bool b_mn, int M, int N, int K,
               int epi, void *out, int64_t ldo, const float *alpha = nullptr) {
@@ -474,6 +501,7 @@ TSP_API void tsp_plan_destroy(tsp_plan_t p) {
         cudaFree(p->d_kv_order);
         cudaFree(p->d_q_order);
         cudaFree(p->d_rank_fwd_order);
+        cudaFree(p->d_rank_bwd_order);
         cudaFree(p->d_err);
         cudaSetDevice(cur);
     }
@@ -837,6 +865,9 @@ TSP_API tsp_status tsp_layer_backward(tsp_plan_t p, const void *dy, const void *
     ab.q_order = p->d_q_order;
     ab.dq_acc = attn_bwd_fused_supported(p->dh) ? reinterpret_cast<int *>(w + l.dq_acc) : nullptr;
     ab.dq_bound = reinterpret_cast<unsigned int *>(w + l.dq_bound);
+    ab.q_row0 = 0;
+    ab.q_rows = S;
+    ab.rank = -1;
     TSP_STAGE(14, 1, launch_attn_delta(ab, p->num_sms, s));
     if (attn_bwd_fused_supported(p->dh)) {
         // one pass: dK, dV and the fixed-point dQ sum; then dQ to fp16
@@ -1135,6 +1166,191 @@ TSP_API tsp_status tsp_rank_forward_out(tsp_plan_t p, int rank, const void *x, c
     TSP_RSTAGE(6, 1, launch_gemm(g2d, err, p->num_sms, s));
     return TSP_OK;
 }
+
+namespace {
+// Byte layout of one rank's backward scratch: the layer backward's buffers
+// over the rank's L rows (delta stays [H][S], indexed by local row like lse).
+struct RankBwdLayout {
+    size_t dy16, du, db, dy, dyh, dO, delta, dqkv, da, dgp, gscales, gpart, dq_acc, dq_bound, total;
+};
+RankBwdLayout rank_bwd_layout_of(const tsp_plan_s *p) {
+    RankBwdLayout l{};
+    const size_t L = p->L, S = p->S, h = p->h, F = p->F, H = p->H;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += up(bytes);
+        return o;
+    };
+    l.dy16 = take(L * h * 2);
+    l.du = take(L * F * 2);
+    l.db = take(L * h * 4);
+    l.dy = take(L * h * 4);
+    l.dyh = take(L * h * 2);
+    l.dO = take(L * h * 2);
+    l.delta = take(H * S * 4);
+    l.dqkv = take(L * 3 * h * 2);
+    l.da = take(L * h * 4);
+    l.dgp = take(static_cast<size_t>(rmsnorm_bwd_partial_blocks(static_cast<int>(L))) * h * 4);
+    l.gscales = take(64 * 4);
+    l.gpart = take(static_cast<size_t>(kMaxConv) * kConvBlocks * 4);
+    l.dq_acc = take(L * h * 4);
+    l.dq_bound = take(3 * H * 4);
+    l.total = off;
+    return l;
+}
+}  // namespace
+
+TSP_API tsp_status tsp_rank_backward_workspace_size(tsp_plan_t p, size_t *bws_bytes) {
+    if (!p || !bws_bytes) return TSP_ERR_INVALID_ARG;
+    *bws_bytes = rank_bwd_layout_of(p).total;
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_rank_backward_attn(tsp_plan_t p, int rank, const void *dz, const void *k, const void *v,
+                                          const float *g2, void *ws, void *bws, float *dk_part, float *dv_part,
+                                          float *dwo, float *dg2, float *dw1, float *dw2, void *stream) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    if (!attn_bwd_fused_supported(p->dh)) return TSP_ERR_UNSUPPORTED;  // the single-pass kernel's rank mode
+    tsp_status st = rank_checks(p, rank, {dz, k, v, (const void *)g2, (const void *)ws, (const void *)bws,
+                                          (const void *)dk_part, (const void *)dv_part, (const void *)dwo,
+                                          (const void *)dg2, (const void *)dw1, (const void *)dw2});
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const RankLayout fl = rank_layout_of(p);
+    const RankBwdLayout l = rank_bwd_layout_of(p);
+    const uint8_t *sv = static_cast<const uint8_t *>(ws);
+    uint8_t *w = static_cast<uint8_t *>(bws);
+    const int S = static_cast<int>(p->S), L = static_cast<int>(p->L), h = p->h, F = p->F;
+    const DevErr err = dev_err(p);
+    const float *winv = reinterpret_cast<const float *>(sv + fl.scales) + kScaleInv;
+    const void *u = sv + fl.u, *g = sv + fl.g, *b = sv + fl.b, *o = sv + fl.o;
+    void *dy16 = w + l.dy16, *du = w + l.du, *dyh = w + l.dyh, *dO = w + l.dO, *dqkv = w + l.dqkv;
+    float *db = reinterpret_cast<float *>(w + l.db);
+    float *gsc = reinterpret_cast<float *>(w + l.gscales);
+    const float *ginv = gsc + 0, *gmul = gsc + 1;
+    // dZ of this rank's rows into the scaled fp16 domain (2^k from this rank's max|dZ|)
+    ConvBatch cb{};
+    cb.t[0] = ConvTensor{dz, dy16, int64_t(L) * h, kTargetGrad, gsc + 0, gsc + 1};
+    cb.count = 1;
+    cb.partial = reinterpret_cast<float *>(w + l.gpart);
+    cb.err = p->d_err;
+    TSP_RSTAGE(21, 2, launch_convert_f16(cb, s));
+    // MLP backward over the rank's rows; dW2, dW1 are this rank's partial sums
+    GemmDesc gdu = gemm(dy16, h, false, sv + fl.w2_h, F, true, L, F, h, EPI_DGELU, du, F, winv + 3);
+    gdu.aux = u;
+    gdu.ldaux = F;
+    TSP_RSTAGE(7, 1, launch_gemm(gdu, err, p->num_sms, s));
+    TSP_RSTAGE(8, 1, launch_gemm(gemm(dy16, h, true, g, F, true, h, F, L, EPI_F32, dw2, F, ginv), err, p->num_sms, s));
+    TSP_RSTAGE(9, 1, launch_gemm(gemm(du, F, true, b, h, true, F, h, L, EPI_F32, dw1, h, ginv), err, p->num_sms, s));
+    GemmDesc gdb = gemm(du, F, false, sv + fl.w1_h, h, true, L, h, F, EPI_F32, db, h, winv + 2);
+    gdb.ring_rows = L;
+    gdb.ring_kblocks = (F / p->D) / 64;
+    gdb.ring_rank0 = rank;
+    TSP_RSTAGE(10, 1, launch_gemm(gdb, err, p->num_sms, s));
+    NormBwd n2{};
+    n2.dout = db;
+    n2.x_f32 = reinterpret_cast<const float *>(sv + fl.y);
+    n2.rstd = reinterpret_cast<const float *>(sv + fl.rstd2);
+    n2.g = g2;
+    n2.resid_bf16 = dz;
+    n2.dx_f32 = reinterpret_cast<float *>(w + l.dy);
+    n2.dx_low = dyh;
+    n2.low_f16 = true;
+    n2.dg_partial = reinterpret_cast<float *>(w + l.dgp);
+    n2.dg = dg2;
+    n2.resid_mul = gmul;
+    n2.dg_mul = ginv;
+    n2.err = p->d_err;
+    n2.rows = L;
+    n2.h = h;
+    TSP_RSTAGE(11, 2, launch_rmsnorm_bwd(n2, s));
+    TSP_RSTAGE(12, 1, launch_gemm(gemm(dyh, h, false, sv + fl.wo_h, h, true, L, h, h, EPI_F16, dO, h, winv + 1), err,
+                                  p->num_sms, s));
+    TSP_RSTAGE(13, 1, launch_gemm(gemm(dyh, h, true, o, h, true, h, h, L, EPI_F32, dwo, h, ginv), err, p->num_sms, s));
+    // attention backward of the rank's query rows over the gathered K / V:
+    // dQ of its rows, and its share of every visible key's dK / dV (fp32,
+    // out of the scaled domain) for the caller to reduce to the keys' owners
+    AttnBwdDesc ab{};
+    ab.S = S;
+    ab.L = L;
+    ab.D = p->D;
+    ab.H = p->H;
+    ab.dh = p->dh;
+    ab.chunk = static_cast<int>(p->c);
+    ab.q = sv + fl.q;
+    ab.k = k;
+    ab.v = v;
+    ab.o = o;
+    ab.dout = dO;
+    ab.lse = reinterpret_cast<const float *>(sv + fl.lse);
+    ab.delta = reinterpret_cast<float *>(w + l.delta);
+    ab.dq = dqkv;
+    ab.ldd = 3 * h;
+    ab.err = p->d_err;
+    ab.inv_map = p->d_inv;
+    ab.kv_order = p->d_rank_bwd_order + p->rank_bwd_off[rank];
+    ab.kv_items = p->rank_bwd_items[rank];
+    ab.dq_acc = reinterpret_cast<int *>(w + l.dq_acc);
+    ab.dq_bound = reinterpret_cast<unsigned int *>(w + l.dq_bound);
+    ab.q_row0 = rank * L;
+    ab.q_rows = L;
+    ab.rank = rank;
+    ab.dk_part = dk_part;
+    ab.dv_part = dv_part;
+    ab.dkv_mul = ginv;
+    TSP_RSTAGE(14, 1, launch_attn_delta(ab, p->num_sms, s));
+    TSP_RSTAGE(22, 1, launch_attn_bwd_fused(ab, err, p->num_sms, s, p->d_zig));
+    TSP_RSTAGE(23, 1, launch_dq_convert(ab, s));
+    return TSP_OK;
+}
+
+TSP_API tsp_status tsp_rank_backward_qkv(tsp_plan_t p, int rank, const void *x, const float *g1, const float *dk,
+                                         const float *dv, void *ws, void *bws, void *dx, float *dg1, float *dwqkv,
+                                         void *stream) {
+    if (!p) return TSP_ERR_INVALID_ARG;
+    if (!attn_bwd_fused_supported(p->dh)) return TSP_ERR_UNSUPPORTED;  // the single-pass kernel's rank mode
+    tsp_status st = rank_checks(p, rank, {x, (const void *)g1, (const void *)dk, (const void *)dv,
+                                          (const void *)ws, (const void *)bws, dx, (const void *)dg1,
+                                          (const void *)dwqkv});
+    if (st != TSP_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const RankLayout fl = rank_layout_of(p);
+    const RankBwdLayout l = rank_bwd_layout_of(p);
+    const uint8_t *sv = static_cast<const uint8_t *>(ws);
+    uint8_t *w = static_cast<uint8_t *>(bws);
+    const int L = static_cast<int>(p->L), h = p->h;
+    const DevErr err = dev_err(p);
+    const float *winv = reinterpret_cast<const float *>(sv + fl.scales) + kScaleInv;
+    uint8_t *dqkv = w + l.dqkv;
+    const float *gsc = reinterpret_cast<const float *>(w + l.gscales);
+    const float *ginv = gsc + 0, *gmul = gsc + 1;
+    float *da = reinterpret_cast<float *>(w + l.da);
+    // the reduced dK / dV of this rank's rows back into its scaled fp16 domain
+    TSP_RSTAGE(24, 1, launch_scale_to_f16(dk, L, h, dqkv + static_cast<size_t>(h) * 2, 3 * h, gmul, p->d_err, s));
+    TSP_RSTAGE(24, 1, launch_scale_to_f16(dv, L, h, dqkv + static_cast<size_t>(2 * h) * 2, 3 * h, gmul, p->d_err, s));
+    TSP_RSTAGE(17, 1, launch_gemm(gemm(dqkv, 3 * h, true, sv + fl.a, h, true, 3 * h, h, L, EPI_F32, dwqkv, h, ginv),
+                                  err, p->num_sms, s));
+    TSP_RSTAGE(18, 1, launch_gemm(gemm(dqkv, 3 * h, false, sv + fl.wqkv_h, h, true, L, h, 3 * h, EPI_F32, da, h,
+                                       winv + 0), err, p->num_sms, s));
+    NormBwd n1{};
+    n1.dout = da;
+    n1.x_bf16 = x;
+    n1.rstd = reinterpret_cast<const float *>(sv + fl.rstd1);
+    n1.g = g1;
+    n1.resid_f32 = reinterpret_cast<const float *>(w + l.dy);
+    n1.dx_low = dx;
+    n1.low_f16 = false;
+    n1.dg_partial = reinterpret_cast<float *>(w + l.dgp);
+    n1.dg = dg1;
+    n1.dx_mul = ginv;
+    n1.dg_mul = ginv;
+    n1.err = p->d_err;
+    n1.rows = L;
+    n1.h = h;
+    TSP_RSTAGE(19, 2, launch_rmsnorm_bwd(n1, s));
+    return TSP_OK;
+}
 #undef TSP_RSTAGE
 
 TSP_API tsp_status tsp_test_gemm(int a_mn, int b_mn, int M, int N, int K, const void *A, int64_t lda, const void *B,
@@ -1230,6 +1446,30 @@ TSP_API tsp_status tsp_test_step_walk_desc(tsp_plan_t p, int kv0, int32_t *steps
         if (n < capacity) steps[n] = w.q;
     *count = n;
     return n <= capacity ? TSP_OK : TSP_ERR_INVALID_ARG;
+}
+
+TSP_API tsp_status tsp_test_step_walk_rank(tsp_plan_t p, int rank, int kv0, int32_t *steps, int capacity,
+                                           int *count) {
+    if (!p || !count || capacity < 0 || (capacity > 0 && !steps)) return TSP_ERR_INVALID_ARG;
+    if (kv0 < 0 || kv0 >= p->S || rank < 0 || rank >= p->D) return TSP_ERR_INVALID_ARG;
+    const StepVis vis{p->D, static_cast<int>(p->c), static_cast<int>(p->S / 64), rank};
+    int n = 0;
+    DescWalk w;
+    for (w.seek(vis, kv0); w.q < vis.nq64; w.next(vis, kv0), ++n)
+        if (n < capacity) steps[n] = w.q;
+    *count = n;
+    return n <= capacity ? TSP_OK : TSP_ERR_INVALID_ARG;
+}
+
+TSP_API tsp_status tsp_test_rank_kv_order(tsp_plan_t p, int rank, int num_ctas, int32_t *out, int64_t capacity,
+                                          int64_t *count) {
+    if (!p || !count || capacity < 0 || (capacity > 0 && !out) || num_ctas < 1) return TSP_ERR_INVALID_ARG;
+    if (rank < 0 || rank >= p->D) return TSP_ERR_INVALID_ARG;
+    const std::vector<int32_t> v = rank_kv_order(p, host_tables(p), rank, num_ctas);
+    *count = static_cast<int64_t>(v.size());
+    if (*count > capacity) return TSP_ERR_INVALID_ARG;
+    std::copy(v.begin(), v.end(), out);
+    return TSP_OK;
 }
 
 TSP_API tsp_status tsp_test_step_walk(tsp_plan_t p, int kv0, int32_t *steps, int capacity, int *count) {

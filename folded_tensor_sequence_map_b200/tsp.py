@@ -46,6 +46,9 @@ EXPORTED = (
     "tsp_rank_workspace_size",
     "tsp_rank_forward_qkv",
     "tsp_rank_forward_out",
+    "tsp_rank_backward_workspace_size",
+    "tsp_rank_backward_attn",
+    "tsp_rank_backward_qkv",
     "tsp_sync_status",
     "tsp_status_string",
     "tsp_layer_flops",
@@ -58,11 +61,13 @@ EXPORTED = (
     "tsp_test_next_visible",
     "tsp_test_step_walk",
     "tsp_test_step_walk_desc",
+    "tsp_test_step_walk_rank",
+    "tsp_test_rank_kv_order",
     "tsp_test_tables",
     "tsp_test_work_order",
     "tsp_test_wait_timeout",
 )
-TSP_NUM_STAGES = 24
+TSP_NUM_STAGES = 25
 
 
 class TSPError(RuntimeError):
@@ -108,6 +113,12 @@ def _load() -> ctypes.CDLL:
     lib.tsp_rank_forward_qkv.restype = I
     lib.tsp_rank_forward_out.argtypes = [P, I] + [V] * 10
     lib.tsp_rank_forward_out.restype = I
+    lib.tsp_rank_backward_workspace_size.argtypes = [P, ctypes.POINTER(SZ)]
+    lib.tsp_rank_backward_workspace_size.restype = I
+    lib.tsp_rank_backward_attn.argtypes = [P, I] + [V] * 13
+    lib.tsp_rank_backward_attn.restype = I
+    lib.tsp_rank_backward_qkv.argtypes = [P, I] + [V] * 10
+    lib.tsp_rank_backward_qkv.restype = I
     lib.tsp_sync_status.argtypes = [P, V]
     lib.tsp_sync_status.restype = I
     lib.tsp_status_string.argtypes = [I]
@@ -124,6 +135,10 @@ def _load() -> ctypes.CDLL:
     lib.tsp_test_step_walk.restype = I
     lib.tsp_test_step_walk_desc.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I, ctypes.POINTER(I)]
     lib.tsp_test_step_walk_desc.restype = I
+    lib.tsp_test_step_walk_rank.argtypes = [P, I, I, ctypes.POINTER(ctypes.c_int32), I, ctypes.POINTER(I)]
+    lib.tsp_test_step_walk_rank.restype = I
+    lib.tsp_test_rank_kv_order.argtypes = [P, I, I, ctypes.POINTER(ctypes.c_int32), I64, ctypes.POINTER(I64)]
+    lib.tsp_test_rank_kv_order.restype = I
     lib.tsp_test_tables.argtypes = [P, I, ctypes.POINTER(ctypes.c_int32), I64, ctypes.POINTER(I64)]
     lib.tsp_test_tables.restype = I
     lib.tsp_test_work_order.argtypes = [P, I, I, ctypes.POINTER(ctypes.c_int32), I64, ctypes.POINTER(I64)]
@@ -403,6 +418,39 @@ def tsp_rank_forward_out(plan: Plan, rank: int, x, k, v, wo, g2, w1, w2, z, ws, 
            "tsp_rank_forward_out")
 
 
+def tsp_rank_backward_workspace_size(plan: Plan) -> int:
+    bws = ctypes.c_size_t()
+    _check(_lib.tsp_rank_backward_workspace_size(plan.handle, ctypes.byref(bws)), "tsp_rank_backward_workspace_size")
+    return bws.value
+
+
+def tsp_rank_backward_attn(plan: Plan, rank: int, dz, k, v, g2, ws, bws, dk_part, dv_part, dwo, dg2, dw1, dw2,
+                           stream=None) -> None:
+    import torch
+
+    h, F, S, L = plan.h, plan.ffn, plan.S, plan.S // plan.D
+    bf, f32, f16 = torch.bfloat16, torch.float32, torch.float16
+    _check(_lib.tsp_rank_backward_attn(plan.handle, rank, _ptr(dz, "dz", bf, (L, h)), _ptr(k, "k", f16, (S, h)),
+                                       _ptr(v, "v", f16, (S, h)), _ptr(g2, "g2", f32, (h,)), _ptr(ws, "ws"),
+                                       _ptr(bws, "bws"), _ptr(dk_part, "dk_part", f32, (S, h)),
+                                       _ptr(dv_part, "dv_part", f32, (S, h)), _ptr(dwo, "dwo", f32, (h, h)),
+                                       _ptr(dg2, "dg2", f32, (h,)), _ptr(dw1, "dw1", f32, (F, h)),
+                                       _ptr(dw2, "dw2", f32, (h, F)), _stream(stream)),
+           "tsp_rank_backward_attn")
+
+
+def tsp_rank_backward_qkv(plan: Plan, rank: int, x, g1, dk, dv, ws, bws, dx, dg1, dwqkv, stream=None) -> None:
+    import torch
+
+    h, L = plan.h, plan.S // plan.D
+    bf, f32 = torch.bfloat16, torch.float32
+    _check(_lib.tsp_rank_backward_qkv(plan.handle, rank, _ptr(x, "x", bf, (L, h)), _ptr(g1, "g1", f32, (h,)),
+                                      _ptr(dk, "dk", f32, (L, h)), _ptr(dv, "dv", f32, (L, h)), _ptr(ws, "ws"),
+                                      _ptr(bws, "bws"), _ptr(dx, "dx", bf, (L, h)), _ptr(dg1, "dg1", f32, (h,)),
+                                      _ptr(dwqkv, "dwqkv", f32, (3 * h, h)), _stream(stream)),
+           "tsp_rank_backward_qkv")
+
+
 def tsp_sync_status(plan: Plan, stream=None) -> None:
     _check(_lib.tsp_sync_status(plan.handle, _stream(stream)), "tsp_sync_status")
 
@@ -465,6 +513,24 @@ def tsp_test_step_walk(plan: Plan, kv0: int, descending: bool = False) -> np.nda
     name = "tsp_test_step_walk_desc" if descending else "tsp_test_step_walk"
     _check(fn(plan.handle, kv0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cap, ctypes.byref(n)), name)
     return out[:n.value].copy()
+
+
+def tsp_test_step_walk_rank(plan: Plan, rank: int, kv0: int) -> np.ndarray:
+    cap = plan.S // 64
+    out = np.zeros(cap, dtype=np.int32)
+    n = ctypes.c_int()
+    _check(_lib.tsp_test_step_walk_rank(plan.handle, rank, kv0, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                        cap, ctypes.byref(n)), "tsp_test_step_walk_rank")
+    return out[:n.value].copy()
+
+
+def tsp_test_rank_kv_order(plan: Plan, rank: int, num_ctas: int) -> np.ndarray:
+    n = ctypes.c_int64()
+    _lib.tsp_test_rank_kv_order(plan.handle, rank, num_ctas, None, 0, ctypes.byref(n))  # length query
+    out = np.zeros(n.value, dtype=np.int32)
+    _check(_lib.tsp_test_rank_kv_order(plan.handle, rank, num_ctas, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                       n.value, ctypes.byref(n)), "tsp_test_rank_kv_order")
+    return out
 
 
 TABLES = {"inv": 0, "qtile_maxpos": 1, "fwd_order": 2, "kv_order": 3, "q_order": 4}

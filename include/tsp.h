@@ -283,6 +283,51 @@ tsp_status tsp_rank_forward_out(tsp_plan_t plan, int rank, const void *x, const 
                                 const void *wo, const float *g2, const void *w1, const void *w2, void *z, void *ws,
                                 void *stream);
 
+/* One rank's share of the backward, after that rank's two forward calls with
+ * the same ws, k and v (the workspace keeps the rank's activations, the
+ * gathered K/V stay in k, v).  Head size 128 only.  Two calls, with the dK/dV
+ * reduce-scatter between them:
+ *
+ * tsp_rank_backward_workspace_size: bytes of one rank's backward scratch bws.
+ *
+ * tsp_rank_backward_attn: from dz (bf16 [L][h], gradient of the rank's z
+ * rows): the MLP backward (dW2, dW1 with the rank's rows as the contraction;
+ * db with its K loop in the rank's ring order), RMSNorm2 backward (dg2), the
+ * out-projection backward (dWo, dO) and the attention backward of the rank's
+ * query rows over all S keys: dQ of its rows stays in bws, and its share of
+ * dK and dV for every key goes out as fp32 partial sums into dk_part, dv_part
+ * ([S][h], rank-major local rows of the key's owner; overwritten, keys the
+ * rank's rows do not see are zero).  dwo [h][h], dg2 [h], dw1 [F][h], dw2
+ * [h][F] (fp32, overwritten) are the sums over this rank's rows only.
+ *
+ * Between the calls the caller sums dk_part and dv_part over the ranks and
+ * hands each rank its rows: a reduce-scatter of the S rows into L-row blocks
+ * (block j to rank j), since the partial rows are already in rank-major
+ * order.
+ *
+ * tsp_rank_backward_qkv: with dk, dv (fp32 [L][h], the reduced dK, dV of the
+ * rank's own rows): the QKV projection backward (dWqkv [3h][h], this rank's
+ * rows only) and RMSNorm1 backward + residual into dx (bf16 [L][h]) and dg1
+ * [h] (this rank's rows only).  x, g1 as in the forward.
+ *
+ * The caller then sums dwqkv, dwo, dw1, dw2, dg1 and dg2 over the ranks
+ * (all-reduce).  The gradient scale 2^k of a rank comes from its own max|dz|,
+ * and the dK/dV it receives are converted into that rank's fp16 domain: a sum
+ * past fp16's range there (dz of very different magnitudes across ranks)
+ * is reported as TSP_ERR_RANGE by tsp_sync_status, never silently clipped.
+ * Up to rounding the results are the layer backward's on the rank's rows
+ * (the layer takes one scale from all rows, the fixed-point dQ sum its bound
+ * from all rows, and the dK/dV partials are summed in fp32 before the fp16
+ * rounding).  Errors as for the forward calls, and TSP_ERR_UNSUPPORTED for a
+ * head size other than 128. */
+tsp_status tsp_rank_backward_workspace_size(tsp_plan_t plan, size_t *bws_bytes);
+tsp_status tsp_rank_backward_attn(tsp_plan_t plan, int rank, const void *dz, const void *k, const void *v,
+                                  const float *g2, void *ws, void *bws, float *dk_part, float *dv_part, float *dwo,
+                                  float *dg2, float *dw1, float *dw2, void *stream);
+tsp_status tsp_rank_backward_qkv(tsp_plan_t plan, int rank, const void *x, const float *g1, const float *dk,
+                                 const float *dv, void *ws, void *bws, void *dx, float *dg1, float *dwqkv,
+                                 void *stream);
+
 /* Wait for `stream`, then report TSP_ERR_CUDA for an asynchronous CUDA error,
  * TSP_ERR_TIMEOUT if a device-side wait of this plan ran out, or TSP_ERR_RANGE
  * if a value overflowed an fp16 intermediate (the flags are cleared by the
@@ -297,8 +342,9 @@ const char *tsp_status_string(tsp_status status);
  * (first in the forward) and 21 the backward's dY conversion (first in the
  * backward).  With head size 128 the attention backward is one pass, stage
  * 22 (dK, dV and the fp32 dQ sum) and stage 23 (dQ to fp16), in place of
- * stages 15 and 16. */
-#define TSP_NUM_STAGES 24
+ * stages 15 and 16.  Stage 24 is the per-rank backward's conversion of the
+ * reduced dK/dV into fp16 (tsp_rank_backward_qkv). */
+#define TSP_NUM_STAGES 25
 
 /* Per-stage timing with CUDA events.  tsp_profile_enable(plan, 1) clears the
  * record and starts bracketing every stage of later layer calls with a pair of

@@ -92,6 +92,19 @@ tsp_status tsp_test_work_order(tsp_plan_t plan, int which, int num_ctas, int32_t
  * prefix of the walk for kv0 = 0.  Output and errors as tsp_test_step_walk. */
 tsp_status tsp_test_step_walk_desc(tsp_plan_t plan, int kv0, int32_t *steps, int capacity, int *count);
 
+/* The same walk as tsp_test_step_walk_desc kept to one rank's query rows (its
+ * chunks 2D-1-rank, then rank), as the per-rank attention backward makes it.
+ * Output and errors as tsp_test_step_walk, and TSP_ERR_INVALID_ARG for a rank
+ * outside [0, D). */
+tsp_status tsp_test_step_walk_rank(tsp_plan_t plan, int rank, int kv0, int32_t *steps, int capacity, int *count);
+
+/* The per-rank attention backward's work order of `rank` for num_ctas
+ * persistent CTAs, as uploaded: key tile * heads + head for every key tile
+ * that the rank's rows see, paired in waves.  Errors as tsp_test_work_order,
+ * and TSP_ERR_INVALID_ARG for a rank outside [0, D). */
+tsp_status tsp_test_rank_kv_order(tsp_plan_t plan, int rank, int num_ctas, int32_t *out, int64_t capacity,
+                                  int64_t *count);
+
 /* Self-test of the bounded device-side wait used by every kernel: launches one
  * CTA that waits on an mbarrier nothing ever completes, with a limit of
  * `limit_cycles` SM cycles.  The wait gives up, the kernel writes 0 to

@@ -112,6 +112,60 @@ def test_descending_walk_is_a_prefix_of_one_order(h, H, F, S, D):
         assert np.array_equal(walk, full[:len(walk)]), (S, D, kv0)
 
 
+@pytest.mark.parametrize("h,H,F,S,D", [(256, 2, 1024, 1024, 2), (512, 4, 2048, 2048, 4),
+                                       (4096, 32, 16384, 32768, 8)])
+def test_rank_walk_and_order_keep_to_the_rank_rows(h, H, F, S, D):
+    """One rank's share of the single-pass backward: its walk for a key tile is
+    the whole-layer walk with every step outside the rank's L local rows left
+    out (same order), and its work order holds each (key tile, head) whose
+    walk is non-empty exactly once: the key tiles at or below the highest
+    position of the rank's rows (oracle zigzag map)."""
+    p = T.tsp_plan(h, H, F, S, D)
+    L, nq = S // D, S // 64
+    zig = O.zigzag_map(S, D).ravel()
+    rng = np.random.default_rng(S + 7 * D)
+    tiles = np.unique(np.concatenate([[0, 1, S // 256, S // 128 - 1], rng.integers(0, S // 128, 16)]))
+    for r in range(D):
+        mine = (np.arange(nq) >= r * L // 64) & (np.arange(nq) < (r + 1) * L // 64)
+        for kt in tiles:
+            full = T.tsp_test_step_walk(p, int(kt) * 128, descending=True)
+            walk = T.tsp_test_step_walk_rank(p, r, int(kt) * 128)
+            assert np.array_equal(walk, full[mine[full]]), (S, D, r, kt)
+        top = zig[r * L:(r + 1) * L].max()
+        seen = np.array([kt * H + hd for kt in range(S // 128) if kt * 128 <= top for hd in range(H)])
+        order = T.tsp_test_rank_kv_order(p, r, 148)
+        assert np.array_equal(np.sort(order), seen), (S, D, r)
+        for kt in np.unique(order // H):  # no item without steps
+            assert len(T.tsp_test_step_walk_rank(p, r, int(kt) * 128)) > 0
+        beyond = (int(top) // 128 + 1) * 128
+        if beyond < S:
+            assert len(T.tsp_test_step_walk_rank(p, r, beyond)) == 0
+    assert T.STATUS_NAMES[TT._lib.tsp_test_step_walk_rank(p.handle, D, 0, None, 0, ctypes.byref(ctypes.c_int()))] \
+        == "TSP_ERR_INVALID_ARG"
+
+
+def test_rank_backward_checks_arguments_before_enqueueing():
+    """tsp_rank_backward_attn / _qkv refuse a head size other than 128, a rank
+    outside [0, D), a NULL or a misaligned pointer before anything runs."""
+    p = T.tsp_plan(256, 2, 1024, 1024, 2)
+    V = ctypes.c_void_p
+    lib = TT._lib
+    st = lambda rc: T.STATUS_NAMES[rc]
+    good = [V(0x10000 * (i + 1)) for i in range(12)]
+    attn = lambda plan, rank, args: st(lib.tsp_rank_backward_attn(plan.handle, rank, *args[:12], V(0)))
+    qkv = lambda plan, rank, args: st(lib.tsp_rank_backward_qkv(plan.handle, rank, *args[:9], V(0)))
+    for f in (attn, qkv):
+        assert f(p, 2, good) == "TSP_ERR_INVALID_ARG" and f(p, -1, good) == "TSP_ERR_INVALID_ARG"
+        bad = list(good)
+        bad[4] = V(0)
+        assert f(p, 0, bad) == "TSP_ERR_INVALID_ARG"
+        bad = list(good)
+        bad[1] = V(0x20008)
+        assert f(p, 1, bad) == "TSP_ERR_ALIGNMENT"
+        assert f(T.tsp_plan(128, 4, 512, 1024, 2), 0, good) == "TSP_ERR_UNSUPPORTED"  # head size 32
+    assert T.tsp_rank_backward_workspace_size(p) > 0
+
+
 def _start_spread(cost, G):
     """Largest gap, over the rounds of G items, between the first and the last
     start time of a round's items when CTA i runs items i, i + G, ... at one
