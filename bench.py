@@ -513,28 +513,77 @@ def main():
         fwd()
     t_fwd = timed(fwd, args.steps)
 
-    # end to end: pinned host inputs in, results out, inside the timed region
+    # end to end: pinned host inputs in, results out, inside the timed region.
+    # Every step copies its own inputs in and its results out; the copies run
+    # on two copy streams beside the compute (inputs and outputs double-
+    # buffered: step i+1's inputs arrive and step i's results leave while
+    # step i / i+1 computes), and the timed region runs from before the first
+    # step's input copy to after the last step's result copy.
     e2e = None
     if not args.no_e2e:
-        # every result comes back: the output, dx and all weight and gain gradients
         y_host = torch.empty(S, h, dtype=bf).pin_memory()
         g_host = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in grads.items()}
+        ins = [(x, dy), (torch.empty_like(x), torch.empty_like(dy))]
+        outs = [(y, grads), (torch.empty_like(y), {k: torch.empty_like(v) for k, v in grads.items()})]
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]
+        in_ready, in_free, out_ready, out_free = ev(), ev(), ev(), ev()
 
-        def e2e_step():
-            x.copy_(x_host, non_blocking=True)
-            dy.copy_(dy_host, non_blocking=True)
-            fwd()
-            bwd()
-            y_host.copy_(y, non_blocking=True)
-            for k, v in grads.items():
-                g_host[k].copy_(v, non_blocking=True)
+        def copy_in(b):
+            with torch.cuda.stream(h2d):
+                ins[b][0].copy_(x_host, non_blocking=True)
+                ins[b][1].copy_(dy_host, non_blocking=True)
+            in_ready[b].record(h2d)
 
-        e2e_step()
-        t_e2e = timed(e2e_step, args.steps)
-        d2h = y.numel() * y.element_size() + sum(v.numel() * v.element_size() for v in grads.values())
+        def e2e_run(steps):
+            start = torch.cuda.Event()
+            start.record(stream)
+            h2d.wait_event(start)
+            d2h.wait_event(start)
+            copy_in(0)
+            for i in range(steps):
+                b, nb = i % 2, (i + 1) % 2
+                if i + 1 < steps:
+                    if i >= 1:
+                        h2d.wait_event(in_free[nb])     # step i-1 has finished reading them
+                    copy_in(nb)
+                stream.wait_event(in_ready[b])
+                if i >= 2:
+                    stream.wait_event(out_free[b])      # step i-2's results have left
+                xi, dyi = ins[b]
+                yo, go = outs[b]
+                T.tsp_layer_forward(plan, xi, g1, W["wqkv"], W["wo"], g2, W["w1"], W["w2"], yo, saved, ws, stream)
+                T.tsp_layer_backward(plan, dyi, xi, g1, W["wqkv"], W["wo"], g2, W["w1"], W["w2"], saved, ws,
+                                     go["dx"], go["dg1"], go["dwqkv"], go["dwo"], go["dg2"], go["dw1"], go["dw2"],
+                                     stream)
+                in_free[b].record(stream)
+                out_ready[b].record(stream)
+                d2h.wait_event(out_ready[b])
+                with torch.cuda.stream(d2h):
+                    y_host.copy_(yo, non_blocking=True)
+                    for k, v in go.items():
+                        g_host[k].copy_(v, non_blocking=True)
+                out_free[b].record(d2h)
+            stream.wait_stream(h2d)
+            stream.wait_stream(d2h)
+
+        e2e_run(2)
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_run(args.steps)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        T.tsp_sync_status(plan, stream)
+        t_e2e = reduce_max(a.elapsed_time(b_) / 1e3, dev)
+        d2h_bytes = y.numel() * y.element_size() + sum(v.numel() * v.element_size() for v in grads.values())
         e2e = {"value": world * S * args.steps / t_e2e, "unit": UNIT,
-               "h2d_bytes_per_step": x.numel() * 2 + dy.numel() * 2, "d2h_bytes_per_step": d2h,
-               "copied": "x, dY in; z, dx, dg1, dWqkv, dWo, dg2, dW1, dW2 out (pinned host memory)"}
+               "h2d_bytes_per_step": x.numel() * 2 + dy.numel() * 2, "d2h_bytes_per_step": d2h_bytes,
+               "copied": "x, dY in; z, dx, dg1, dWqkv, dWo, dg2, dW1, dW2 out (pinned host memory), every step; "
+                         "on two copy streams overlapping the compute (inputs and outputs double-buffered), "
+                         "timed from before the first input copy to after the last result copy"}
 
     burst, sustained, hbm, src = peaks()
     flops = stage_flops(shape)

@@ -41,6 +41,38 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for a share of the softmax's exponentials (the MUFU
+// unit needs as many cycles per 128x128 tile as the tile's two MMAs).  The
+// argument is split as x = n + f with n = round(x): adding 1.5 * 2^23 leaves
+// n in the low mantissa bits of the sum, and f = x - n lies in [-1/2, 1/2]
+// (the argument reduction of Cody and Waite, "Software Manual for the
+// Elementary Functions", 1980).  2^f is a degree-5 polynomial fitted by the
+// Remez exchange for least maximum relative error (csrc/fit_exp2.py: 2.1e-7
+// evaluated in fp32), and 2^n enters by an integer add to the exponent
+// field.  Valid for x < 128; x <= -127 (-inf included) gives 0 or a denormal
+// below 2^-126.
+__device__ __forceinline__ float exp2_poly(float x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    x = fmaxf(x, -127.0f);
+    const float t = __fadd_rn(x, kShift);
+    const float f = __fsub_rn(x, __fsub_rn(t, kShift));
+    float p = fmaf(f, 0x1.5c08e6p-10f, 0x1.3d0c52p-7f);
+    p = fmaf(p, f, 0x1.c6b6e4p-5f);
+    p = fmaf(p, f, 0x1.ebf918p-3f);
+    p = fmaf(p, f, 0x1.62e428p-1f);
+    p = fmaf(p, f, 0x1.000002p+0f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Which of a row's 128 exponentials per key tile take exp2_poly: key k of
+// the tile when k % kPolyEvery == kPolyEvery - 1 (0: none).  Measured on the
+// 7B layer at S=131072 (forward attention, ms per step, same box): none
+// 154-159, one in 8 167-175, one in 5 185-187, one in 4 190-192, one in 3
+// 190-195.  The softmax is not limited by the MUFU's rate, and each
+// polynomial costs ten issue slots where the MUFU costs one, so none is used.
+constexpr int kPolyEvery = 0;
+__host__ __device__ constexpr bool poly_key(int k) { return kPolyEvery > 0 && k % kPolyEvery == kPolyEvery - 1; }
+
 // Global position of local (rank-major) row i under the zigzag partition.
 __device__ __forceinline__ int zig_pos(int i, int L, int D, int c) {
     const int r = i / L;
@@ -375,8 +407,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int k0 = half * 64 + 2 * c;
-                        const float p0 = ex2(fmaf(s[k0], sl2, neg_m));
-                        const float p1 = ex2(fmaf(s[k0 + 1], sl2, neg_m));
+                        const float x0 = fmaf(s[k0], sl2, neg_m), x1 = fmaf(s[k0 + 1], sl2, neg_m);
+                        const float p0 = poly_key(k0) ? exp2_poly(x0) : ex2(x0);
+                        const float p1 = poly_key(k0 + 1) ? exp2_poly(x1) : ex2(x1);
                         ls[(2 * c) & 7] += p0;
                         ls[(2 * c + 1) & 7] += p1;
                         pk[c] = __uint_as_float(pack_f16(p0, p1));
@@ -445,7 +478,19 @@ cudaError_t launch_fwd_impl(const AttnDesc &a, const DevErr &err, int num_sms, c
     return cudaGetLastError();
 }
 
+__global__ void exp2_test_kernel(const float *x, float *y, int n, int which) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = which == 0 ? exp2_poly(x[i]) : ex2(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_test(const float *x, float *y, int n, int which, cudaStream_t st) {
+    if (n < 0 || (which != 0 && which != 1)) return cudaErrorInvalidValue;
+    if (n == 0) return cudaSuccess;
+    exp2_test_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n, which);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_attn_fwd(const AttnDesc &a, const DevErr &err, int num_sms, cudaStream_t st) {
     switch (a.dh) {

@@ -129,6 +129,9 @@ struct ConvBatch {
 cudaError_t launch_convert_f16(const ConvBatch &b, cudaStream_t st);
 // fp32 [rows][cols] -> fp16 times *mul (device scalar) into rows of stride
 // ldd elements (cols, ldd multiples of 8; both pointers 16-byte aligned).
+// Test hook: y = 2^x by the attention forward's polynomial (which = 0) or by
+// the MUFU approximation (which = 1), n device floats.
+cudaError_t launch_exp2_test(const float *x, float *y, int n, int which, cudaStream_t st);
 cudaError_t launch_scale_to_f16(const float *src, int64_t rows, int cols, void *dst, int64_t ldd, const float *mul,
                                 unsigned int *err, cudaStream_t st);
 

@@ -1535,6 +1535,11 @@ __global__ void wait_timeout_kernel(DevErr err, int *result) {
 }
 }  // namespace
 
+TSP_API tsp_status tsp_test_exp2(const float *x, float *y, int n, int which, void *stream) {
+    if (n < 0 || (n > 0 && (!x || !y)) || (which != 0 && which != 1)) return TSP_ERR_INVALID_ARG;
+    return cuda_status(launch_exp2_test(x, y, n, which, static_cast<cudaStream_t>(stream)));
+}
+
 TSP_API tsp_status tsp_test_wait_timeout(tsp_plan_t p, long long limit_cycles, int *result_dev, void *stream) {
     if (!p || !result_dev || limit_cycles <= 0) return TSP_ERR_INVALID_ARG;
     tsp_status st = ensure_device(p);

@@ -66,6 +66,7 @@ EXPORTED = (
     "tsp_test_tables",
     "tsp_test_work_order",
     "tsp_test_wait_timeout",
+    "tsp_test_exp2",
 )
 TSP_NUM_STAGES = 25
 
@@ -154,6 +155,8 @@ def _load() -> ctypes.CDLL:
     lib.tsp_rmsnorm_backward_noalloc.restype = I
     lib.tsp_test_wait_timeout.argtypes = [P, ctypes.c_longlong, V, V]
     lib.tsp_test_wait_timeout.restype = I
+    lib.tsp_test_exp2.argtypes = [V, V, I, I, V]
+    lib.tsp_test_exp2.restype = I
     return lib
 
 
@@ -560,3 +563,13 @@ def tsp_test_wait_timeout(plan: Plan, limit_cycles: int, result, stream=None) ->
     _check(_lib.tsp_test_wait_timeout(plan.handle, limit_cycles, _ptr(result, "result"), _stream(stream)),
            "tsp_test_wait_timeout")
 
+
+
+def tsp_test_exp2(x, y, which: int, stream=None) -> None:
+    """y = 2^x (fp32 device tensors of the same length): which 0 the
+    attention forward's polynomial, 1 the hardware approximation."""
+    import torch
+
+    n = x.numel()
+    _check(_lib.tsp_test_exp2(_ptr(x, "x", torch.float32, (n,)), _ptr(y, "y", torch.float32, (n,)), n, which,
+                              _stream(stream)), "tsp_test_exp2")

@@ -111,6 +111,13 @@ tsp_status tsp_test_rank_kv_order(tsp_plan_t plan, int rank, int num_ctas, int32
  * result_dev[0] (1 would mean the wait completed) and sets the plan's error
  * flag, so the next tsp_sync_status() reports TSP_ERR_TIMEOUT.  No memory
  * copy or tensor-core work is in flight, so giving up is safe. */
+/* y[i] = 2^x[i] for n device floats, by the polynomial exp2 that the
+ * attention forward uses for a share of its exponentials (which = 0) or by
+ * the hardware approximation it uses for the rest (which = 1).
+ * TSP_ERR_INVALID_ARG for another `which`, n < 0 or a NULL pointer with
+ * n > 0; TSP_ERR_CUDA for a failed launch. */
+tsp_status tsp_test_exp2(const float *x, float *y, int n, int which, void *stream);
+
 tsp_status tsp_test_wait_timeout(tsp_plan_t plan, long long limit_cycles, int *result_dev, void *stream);
 
 #ifdef __cplusplus

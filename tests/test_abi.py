@@ -440,3 +440,21 @@ def test_bad_phase_is_rejected():
     p = T.tsp_plan(128, 4, 512, 256, 2)
     with pytest.raises(T.TSPError):
         T.tsp_shard_schedule(p, 2)
+
+
+def test_exp2_polynomial_coefficients_are_the_fit():
+    """The polynomial in the attention forward's exp2 is the one the Remez
+    fit produces (degree 5, coefficients rounded to fp32), and the fit's
+    relative error in fp32 is what the kernel's comment and GPU test state."""
+    from folded_tensor_sequence_map_b200.csrc import fit_exp2 as F
+
+    src = open(os.path.join(ROOT, "folded_tensor_sequence_map_b200", "csrc", "attn_fwd.cu")).read()
+    body = src[src.index("float exp2_poly(float x)"):]
+    body = body[:body.index("\n}\n")]
+    used = [float.fromhex(h) for h in re.findall(r"(0x1\.[0-9a-f]+p[-+]\d+)f", body)]
+    c = F.remez_relative(5).astype(np.float32)
+    # Horner from the top coefficient: c5, c4 in the first fma, then c3 .. c0
+    assert used == [float(c[5]), float(c[4]), float(c[3]), float(c[2]), float(c[1]), float(c[0])]
+    grid = np.linspace(F.LO, F.HI, 200001)
+    err = np.abs(F.horner_f32(c, grid).astype(np.float64) / np.exp2(grid.astype(np.float32).astype(np.float64)) - 1)
+    assert err.max() <= 2.2e-7
