@@ -1,8 +1,8 @@
 """7B-shaped layer (h=4096, 32 heads x 128, FFN 16384) against the oracle.
 
 * S=8192, D=8: forward and forward+backward, every element.
-* S=32768, D=8: forward on every row (seed 2); forward+backward, every element
-  of every output and gradient (seed 3).
+* S=32768, D=8: forward+backward, every element of every output and gradient
+  (seed 3; z on every row).
 * D sweep {1, 2, 4, 8, 16} at S=4096: every D against one run of the
   unsharded oracle (the inputs are drawn in global order, so every D sees the
   same tokens and the same exact result, permuted).
@@ -64,14 +64,6 @@ def test_7b_s8192(training):
         for k in GRADS:
             assert_close(k, grads[k], go[k], report)
     print(report)
-
-
-@pytest.mark.slow
-def test_7b_s32768_forward_all_rows():
-    shape, seed = WORKLOADS["7b_s32k"]
-    inp, zig, z, _ = _run(shape, seed, False)
-    zo, _ = _oracle(shape, inp, zig, False)
-    assert_close("z", z, zo)
 
 
 @pytest.mark.slow
