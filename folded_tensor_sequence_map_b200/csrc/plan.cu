@@ -467,8 +467,9 @@ TSP_API tsp_status tsp_plan(int h, int heads, int ffn, int64_t S, int D, tsp_pla
     const int dh = h / heads;
     if (dh != 32 && dh != 64 && dh != 128) return TSP_ERR_UNSUPPORTED;
     if (h % 128 || S % 256 || (S / D) % 128 || ffn % 128 || (ffn / D) % 64) return TSP_ERR_UNSUPPORTED;
-    // Kernels that run one warp per (token, head) number their threads with
-    // 32-bit integers: heads * S * 32 (+ one block) must stay below 2^31.
+    // The RMSNorm kernels number one warp per row in 32 bits (S * 32 < 2^31);
+    // every other global index is 64-bit.  The bound below, heads * S * 32
+    // (+ one block) below 2^31, covers that with a margin.
     if (S > (int64_t(1) << 28) || static_cast<int64_t>(heads) * S * 32 + 255 > INT32_MAX) return TSP_ERR_UNSUPPORTED;
     tsp_plan_s *p = new (std::nothrow) tsp_plan_s();
     if (!p) return TSP_ERR_INVALID_ARG;
