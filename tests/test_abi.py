@@ -458,3 +458,38 @@ def test_exp2_polynomial_coefficients_are_the_fit():
     grid = np.linspace(F.LO, F.HI, 200001)
     err = np.abs(F.horner_f32(c, grid).astype(np.float64) / np.exp2(grid.astype(np.float32).astype(np.float64)) - 1)
     assert err.max() <= 2.2e-7
+
+
+@pytest.mark.parametrize("S", [32768, 131072])
+def test_rank_orders_pair_long_and_short_items(S):
+    """One rank's backward order for 148 SMs is paired in waves like the
+    layer's: in each wave the long items and the short ones come from the same
+    heads in the same order, each long item at least as long as its partner
+    (cost = the rank's query steps that see the key tile, from the oracle's
+    zigzag map).  For ranks 0 and D/2-1 the pairing narrows the spread of the
+    CTAs' start times against a head-major order; for rank D-1, whose key
+    tiles mostly share one cost, pairs cannot even out: its spread is up to
+    1.5 times the head-major order's (measured 1.0 at S=32768, 1.5 at
+    S=131072, where it is 5% of a CTA's work)."""
+    h, H, F, D, G = 4096, 32, 16384, 8, 148
+    p = T.tsp_plan(h, H, F, S, D)
+    zig = O.zigzag_map(S, D).ravel()
+    L = S // D
+    for r in (0, D // 2 - 1, D - 1):
+        smax = zig[r * L:(r + 1) * L].reshape(L // 64, 64).max(axis=1)
+        cost_kt = np.array([(smax >= kt * 128).sum() for kt in range(S // 128)])
+        up = T.tsp_test_rank_kv_order(p, r, G)
+        cost = cost_kt[up // H]
+        npairs = len(up) // 2
+        for w0 in range(0, npairs, G):
+            w1 = min(w0 + G, npairs)
+            nw = w1 - w0
+            longs, shorts = cost[2 * w0:2 * w0 + nw], cost[2 * w0 + nw:2 * w1]
+            assert np.array_equal(up[2 * w0:2 * w0 + nw] % H, up[2 * w0 + nw:2 * w1] % H), (S, r, w0)
+            assert np.all(longs >= shorts), (S, r, w0)
+        hm = np.array(sorted(up, key=lambda it: (it % H, -cost_kt[it // H], it // H)))
+        spread, spread_hm = _start_spread(cost, G), _start_spread(cost_kt[hm // H], G)
+        if r < D - 1:
+            assert spread < spread_hm, (S, r, spread, spread_hm)
+        else:
+            assert spread <= 1.6 * spread_hm, (S, r, spread, spread_hm)
