@@ -252,17 +252,50 @@ void device_orders(HostTables &t, int H, int G) {
     pair_waves(t.korder, 1, H, G);
 }
 
+// Largest gap, over the rounds of G items, between the earliest and the
+// latest start of a round's items when CTA i runs items i, i + G, ... and an
+// item takes `cost` units.
+int64_t start_spread(const std::vector<int64_t> &cost, int G) {
+    std::vector<int64_t> t(G, 0);
+    int64_t worst = 0;
+    for (size_t r0 = 0; r0 < cost.size(); r0 += G) {
+        const size_t n = std::min<size_t>(G, cost.size() - r0);
+        const auto [lo, hi] = std::minmax_element(t.begin(), t.begin() + n);
+        worst = std::max(worst, *hi - *lo);
+        for (size_t i = 0; i < n; ++i) t[i] += cost[r0 + i];
+    }
+    return worst;
+}
+
 // The backward work order of rank r for G SMs: the key tiles that its rows
 // see (its highest chunk, 2D-1-r, ends at position (2D-r) c - 1), taken from
 // the host order before pairing (a head's tiles in ascending order there, so
-// also longest first for one rank's rows), then paired in waves.
+// also longest first for one rank's rows).  Paired in waves, unless the
+// head-major order keeps the CTAs' start times closer together: for the
+// rank that holds the two middle chunks most key tiles cost the same, and
+// long-with-short pairs then differ in length.  The order does not change the
+// results.
 std::vector<int32_t> rank_kv_order(const tsp_plan_s *p, const HostTables &t, int r, int G) {
     const int64_t last = (2 * p->D - r) * p->c - 1;
     std::vector<int32_t> sub;
     for (int32_t it : t.korder)
         if (static_cast<int64_t>(it / p->H) * 128 <= last) sub.push_back(it);
-    pair_waves(sub, 1, p->H, G);
-    return sub;
+    // cost of key tile kt: the rank's 64-row steps that reach position 128 kt
+    const int64_t L = p->L, steps = L / 64, ntiles = p->S / 128;
+    std::vector<int64_t> tile_cost(ntiles, 0);
+    for (int64_t q = 0; q < steps; ++q) {
+        int32_t mx = 0;
+        for (int64_t i = 0; i < 64; ++i) mx = std::max(mx, p->zig[r * L + q * 64 + i]);
+        for (int64_t kt = 0; kt <= mx / 128 && kt < ntiles; ++kt) ++tile_cost[kt];
+    }
+    auto costs = [&](const std::vector<int32_t> &order) {
+        std::vector<int64_t> c(order.size());
+        for (size_t i = 0; i < order.size(); ++i) c[i] = tile_cost[order[i] / p->H];
+        return c;
+    };
+    std::vector<int32_t> paired = sub;
+    pair_waves(paired, 1, p->H, G);
+    return start_spread(costs(paired), G) <= start_spread(costs(sub), G) ? paired : sub;
 }
 
 // Device tables: map, inverse map, per-query-tile max position and the work
